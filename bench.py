@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Benchmark: SSM-layer decode tokens/s at batch 256, ReplaySSM replay decode
+against the conventional full-state decode, and the achieved HBM bandwidth.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload m2_serving: Mamba-2 layer, batch 256, 128 heads, headdim 64,
+d_state 128, 16 groups (8 heads share B/C), bf16 inputs, fp32 checkpoint,
+16-record window.  One benchmark step is one 16-token window of decode for the
+whole batch: 15 non-flush steps and one flush step (16 launches of the replay
+decode kernel), i.e. 4096 tokens.  Inputs are seeded and synthetic and are
+resident in HBM before timing; the 1 GiB checkpoint is far larger than L2, so
+every step streams it from HBM.
+
+Rank 0 prints one JSON line.  Under torchrun every rank runs an independent
+replica (the path has no exchange step): value = tokens of all ranks / the
+slowest rank's time.
+
+--impl reference times the CPU oracle (fp64, the machine's host cores) on a
+bounded sample of the same workload and prints the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSM-layer decode tokens/s @B=256 (replay vs full-state); achieved HBM GB/s"
+WORKLOAD = "m2_serving"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300, help="timed 16-token windows")
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=60, help="windows timed end to end")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)"
+    return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier copy measurement on this pool)"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.dev), "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def oracle_inputs(n_seq, n_steps):
+    from ssm_state_storage_b200 import workloads as wl
+    w = wl.make(WORKLOAD)
+    g = wl.Generator(w, seqs=range(n_seq))
+    A, D = g.params()
+    S0 = g.initial_state()
+    return w, A, D, S0, g.steps(n_steps)
+
+
+def oracle_time(inputs):
+    """Seconds the fp64 CPU oracle (replay decode, as it stands) takes on them."""
+    import oracle
+    w, A, D, S0, st = inputs
+    oracle.lib()
+    rp = oracle.M2Replay(S0, G=w.G, L=w.L)
+    t0 = time.perf_counter()
+    rp.decode(st["x"], st["dt"], st["Bm"], st["Cm"], A, D)
+    return time.perf_counter() - t0
+
+
+def oracle_sample(n_seq=64, n_steps=256):
+    """The oracle on a bounded sample: n_seq sequences of m2_serving, all 128
+    heads, n_steps decode steps (16 windows, 16 flushes)."""
+    secs = oracle_time(oracle_inputs(n_seq, n_steps))
+    return {"value": n_seq * n_steps / secs, "unit": "tokens/s",
+            "cores": len(os.sched_getaffinity(0)), "kind": "oracle", "seconds": secs,
+            "sample": f"{n_seq} sequences x {n_steps} decode steps x all 128 heads of "
+                      f"{WORKLOAD} (replay oracle, fp64, OpenMP over (sequence, head))"}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    os.environ.setdefault("OMP_NUM_THREADS", str(len(os.sched_getaffinity(0))))
+    n_seq, n_steps = 16, 16
+    inputs = oracle_inputs(n_seq, n_steps)
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        secs = oracle_time(inputs)
+        if i >= args.warmup:
+            per_step.append(secs)
+    tok = n_seq * n_steps
+    total = sum(per_step)
+    value = tok * len(per_step) / total
+    cb = {"value": value, "unit": "tokens/s", "cores": len(os.sched_getaffinity(0)),
+          "kind": "oracle",
+          "sample": f"each step: {n_seq} sequences x {n_steps} decode steps (one window) x all "
+                    f"128 heads of {WORKLOAD}, replay oracle in fp64"}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / len(per_step), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "batch": 256, "sample_batch": n_seq},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_ours(args, rank, world):
+    import torch
+    import torch.distributed as dist
+
+    from ssm_state_storage_b200 import bytes_model as bm
+    from ssm_state_storage_b200 import replayssm as rs
+    from ssm_state_storage_b200 import workloads as wl
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = wl.make(WORKLOAD)
+    L = w.L
+    pool = 4 * L  # distinct input steps, cycled (each step's inputs are 6 MiB)
+    g = wl.Generator(w)
+    A, D = g.params()
+    S0 = g.initial_state()
+    st = g.steps(pool)
+    Ad, Dd = A.to(dev), D.to(dev)
+    inputs = {k: v.to(dev) for k, v in st.items()}
+    layer = rs.Layer("m2", w.B, w.H, w.P, w.N, ngroups=w.G, window=L, in_dtype=w.in_dtype)
+    state = rs.ReplayState(layer, device=dev)
+    rs.replayssm_init(layer, state, S0.to(dev))
+    S_full = S0.to(dev)
+    y = torch.empty(w.B, w.H, w.P, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step_inp(t):
+        i = t % pool
+        return dict(x=inputs["x"][i], dt=inputs["dt"][i], Bm=inputs["Bm"][i],
+                    Cm=inputs["Cm"][i], A=Ad, D=Dd)
+
+    step_in = [step_inp(t) for t in range(pool)]
+
+    def replay_window(wi):
+        for j in range(L):
+            rs.replayssm_decode_step(layer, state, step_in[(wi * L + j) % pool], y, stream)
+
+    def full_window(wi):
+        for j in range(L):
+            rs.replayssm_full_decode_step(layer, S_full, step_in[(wi * L + j) % pool], y,
+                                          stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def timed(fn, n, offset):
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n):
+            fn(offset + i)
+        e1.record(stream)
+        barrier()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    for i in range(args.warmup):
+        replay_window(i)
+    dev_index = os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]
+    with ClockSampler(dev_index) as clk:
+        ms_replay = timed(replay_window, args.steps, args.warmup)
+    clocks = clk.summary()
+    if state.status() != 0:
+        raise RuntimeError(f"device status {state.status()} after the replay run")
+
+    for i in range(args.warmup):
+        full_window(i)
+    ms_full = timed(full_window, args.steps, args.warmup)
+
+    # ---- end to end: pinned host inputs in, y out, through the C ABI
+    e2e = run_e2e(args, w, layer, state, st, Ad, Dd, dev, world, rs, torch, dist)
+
+    tok_per_step = w.B * L
+    hpg = w.H // w.G
+    inb = 2 if w.in_dtype == torch.bfloat16 else 4
+    win_bytes = bm.m2_replay_window_bytes(L, w.P, w.N, hpg, inb) * w.B * w.H
+    full_bytes = bm.m2_conventional_bytes(w.P, w.N, hpg, inb) * w.B * w.H * L
+    ms_per_window = ms_replay / args.steps
+    ms_per_window_full = ms_full / args.steps
+    achieved = win_bytes / (ms_per_window * 1e-3) / 1e9
+    achieved_full = full_bytes / (ms_per_window_full * 1e-3) / 1e9
+    peak, peak_src = peaks()
+    value = world * tok_per_step * args.steps / (ms_replay * 1e-3)
+    value_full = world * tok_per_step * args.steps / (ms_full * 1e-3)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_window,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "model": "Mamba-2 SSM layer (decode step only)",
+                   "global_batch": w.B * world, "batch_per_gpu": w.B, "heads": w.H,
+                   "headdim": w.P, "d_state": w.N, "groups": w.G, "window": L,
+                   "inputs": "bf16", "checkpoint": "fp32", "parallelism": f"replicas x{world}",
+                   "step": "one 16-token window = 15 non-flush + 1 flush decode steps",
+                   "l2": "inputs larger than L2 (1 GiB checkpoint streamed every step)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "m2_decode_kernel",
+                     "peak_source": peak_src,
+                     "algorithmic_bytes_per_launch": win_bytes / L},
+        "full_state": {"value": value_full, "unit": "tokens/s", "ms_per_step": ms_per_window_full,
+                       "achieved_gbs": achieved_full, "frac": achieved_full / peak,
+                       "kernel": "m2_full_kernel"},
+        "replay_over_full": value / value_full,
+        "bytes_per_head_token": {"replay": win_bytes / (w.B * w.H * L),
+                                 "full_state": full_bytes / (w.B * w.H * L)},
+        "clocks": clocks,
+        "gpu_launches": args.steps * L,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, w, layer, state, st, Ad, Dd, dev, world, rs, torch, dist):
+    """Per decode step: H2D copy of the step's inputs from pinned host memory,
+    the decode call, D2H copy of y to pinned host memory -- pipelined over three
+    streams with double-buffered device inputs/outputs."""
+    L = w.L
+    pool = st["x"].shape[0]
+    host = {k: v.pin_memory() for k, v in st.items()}
+    keys = ("x", "dt", "Bm", "Cm")
+    dbuf = [{k: torch.empty_like(host[k][0], device=dev) for k in keys} for _ in range(2)]
+    ydev = [torch.empty(w.B, w.H, w.P, device=dev) for _ in range(2)]
+    yhost = [torch.empty(w.B, w.H, w.P).pin_memory() for _ in range(2)]
+    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_yfree = [torch.cuda.Event() for _ in range(2)]
+    ev_infree = [torch.cuda.Event() for _ in range(2)]
+    for e in ev_yfree + ev_infree:
+        e.record(s_cmp)
+    n_steps = args.e2e_steps * L
+    h2d = sum(host[k][0].numel() * host[k][0].element_size() for k in keys)
+    d2h = yhost[0].numel() * 4
+
+    def run(n, t0):
+        for t in range(t0, t0 + n):
+            i = t % 2
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_infree[i])
+                for k in keys:
+                    dbuf[i][k].copy_(host[k][t % pool], non_blocking=True)
+                ev_in[i].record(s_in)
+            s_cmp.wait_event(ev_in[i])
+            s_cmp.wait_event(ev_yfree[i])
+            inp = dict(dbuf[i], A=Ad, D=Dd)
+            rs.replayssm_decode_step(layer, state, inp, ydev[i], s_cmp)
+            ev_done[i].record(s_cmp)
+            ev_infree[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[i])
+                yhost[i].copy_(ydev[i], non_blocking=True)
+                ev_yfree[i].record(s_out)
+
+    run(2 * L, 0)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    run(n_steps, 0)
+    s_in.wait_stream(s_out)
+    e1.record(s_in)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if state.status() != 0:
+        raise RuntimeError(f"device status {state.status()} after the e2e run")
+    return {"value": world * w.B * n_steps / (ms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d * L, "d2h_bytes_per_step": d2h * L,
+            "steps": args.e2e_steps, "pipelined": "H2D / decode / D2H on three streams"}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,64 @@
+"""Algorithmic HBM bytes of the decode paths (the roofline numerators).
+
+Counts the bytes a step must move at minimum given the storage layout, not
+what the hardware happens to move:
+  conventional (full-state) step, per head-token:
+      read + write the fp32 state, read the step inputs (x, dt, the group's
+      B and C shared by its heads), write y.
+  replay step with k records after the append (k = 1..window), per head-token:
+      read h0, read the k-1 buffered records (x, dt and the group's B; C of
+      past records is never needed), read the step inputs, append the record
+      (not on the flush step, whose buffer empties), write y, and on the flush
+      step write h0 once.
+[sitech.ge, "NVIDIA ו-Dao AI Lab הציגו ReplaySSM…", §Reducing state traffic and
+simplifying rollback]: a 16-token window costs 16 state reads and 16 writes
+conventionally, against one checkpoint write for ReplaySSM.
+"""
+from __future__ import annotations
+
+
+def m2_sizes(P, N, hpg, in_bytes):
+    state = P * N * 4
+    x = P * in_bytes
+    dt_in = in_bytes
+    bc_share = 2 * N * in_bytes / hpg      # B and C of the group, per head
+    b_share = N * in_bytes / hpg
+    y = P * 4
+    return state, x, dt_in, bc_share, b_share, y
+
+
+def m2_conventional_bytes(P, N, hpg, in_bytes):
+    state, x, dt_in, bc, _, y = m2_sizes(P, N, hpg, in_bytes)
+    return 2 * state + x + dt_in + bc + y
+
+
+def m2_replay_bytes(k, L, P, N, hpg, in_bytes):
+    """Bytes of one replay step for one head whose buffer holds k records
+    after the append (the buffered dt is stored as fp32)."""
+    state, x, dt_in, bc, b_share, y = m2_sizes(P, N, hpg, in_bytes)
+    rec_read = x + 4 + b_share
+    flush = k == L
+    append = 0 if flush else (x + 4 + bc)
+    return state + (k - 1) * rec_read + (x + dt_in + bc) + append + y + (state if flush else 0)
+
+
+def m2_replay_window_bytes(L, P, N, hpg, in_bytes):
+    return sum(m2_replay_bytes(k, L, P, N, hpg, in_bytes) for k in range(1, L + 1))
+
+
+def gdn_conventional_bytes(DK, DV, in_bytes):
+    state = DK * DV * 4
+    return 2 * state + (2 * DK + DV) * in_bytes + 8 + DV * 4
+
+
+def gdn_replay_bytes(k, L, DK, DV, in_bytes):
+    state = DK * DV * 4
+    rec_read = (DK + DV) * in_bytes + 8   # k, v, alpha, beta of a past record
+    cur = (2 * DK + DV) * in_bytes + 8    # q, k, v, alpha, beta of this step
+    flush = k == L
+    append = 0 if flush else cur
+    return state + (k - 1) * rec_read + cur + append + DV * 4 + (state if flush else 0)
+
+
+def gdn_replay_window_bytes(L, DK, DV, in_bytes):
+    return sum(gdn_replay_bytes(k, L, DK, DV, in_bytes) for k in range(1, L + 1))

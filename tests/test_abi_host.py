@@ -1,0 +1,88 @@
+"""The C-ABI library loads and exports every entry point the header declares;
+host-side validation answers without touching a GPU (no compute calls here)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+import torch
+
+from ssm_state_storage_b200 import replayssm as rs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(HEADER_DIR):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(HEADER_DIR, fn)).read()
+            names |= set(re.findall(r"^[A-Za-z_][\w \*]*?\b(replayssm_\w+)\s*\(", txt, re.M))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from ssm_state_storage_b200 import build
+    build.build()
+    return rs.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 12
+    for n in sorted(names):
+        assert hasattr(lib, n), n
+    assert names <= set(rs.ENTRY_POINTS), names - set(rs.ENTRY_POINTS)
+
+
+def _m2(**kw):
+    base = dict(kind="m2", batch=256, nheads=128, headdim=64, dstate=128, ngroups=16)
+    base.update(kw)
+    return rs.Layer(**base)
+
+
+def test_validation_and_sizes(lib):
+    L = _m2()
+    assert rs.replayssm_validate(L) == 0
+    assert L.capacity() == 16
+    assert _m2(draft_max=4).capacity() == 19
+    assert L.nbytes("h0") == 256 * 128 * 64 * 128 * 4
+    assert L.nbytes("buf0") == 256 * 128 * 16 * 64 * 2
+    assert L.nbytes("buf2") == 256 * 16 * 16 * 128 * 2
+    assert L.nbytes("len") == 256 * 128 * 4
+    assert _m2(read_fmt="nvfp4").nbytes("rc") == 256 * 128 * 64 * 64
+    assert _m2(read_fmt="nvfp4").nbytes("rc_scale") == 256 * 128 * 64 * 8
+    assert rs.replayssm_validate(_m2(headdim=96)) == 2          # shape
+    assert rs.replayssm_validate(_m2(ngroups=3)) == 2            # H % G
+    assert rs.replayssm_validate(_m2(window=17)) == 5            # capacity
+    assert rs.replayssm_validate(_m2(draft_max=5)) == 5
+    assert rs.replayssm_validate(_m2(read_fmt="fp8", ckpt_fmt="fp8")) == 1
+    g = rs.Layer("gdn", 8, 32, 128, 128)
+    assert rs.replayssm_validate(g) == 0 and g.capacity() == 16
+    assert rs.replayssm_validate(rs.Layer("gdn", 8, 32, 64, 128)) == 2
+    assert rs.replayssm_validate(rs.Layer("gdn", 8, 32, 128, 128, draft_max=2)) == 8
+    assert rs.replayssm_status_string(9) == "buffer state out of range"
+
+
+def test_null_arguments_rejected_before_launch(lib):
+    L = _m2(batch=2)
+    d = L.desc()
+    st = rs.State()
+    si = rs.StepIn()
+    # no CUDA call is made: every check fails first
+    assert lib.replayssm_decode_step(C.byref(d), C.byref(st), C.byref(si), None, None) == 1
+    assert lib.replayssm_decode_step(None, C.byref(st), C.byref(si), None, None) == 1
+    assert lib.replayssm_flush(C.byref(d), None, None, 0, None) == 1
+    assert lib.replayssm_verify_commit(C.byref(d), C.byref(st), None, C.byref(si), 1, None,
+                                       None) in (1, 5)
+    assert lib.replayssm_quantize(7, 1, 1, 16, None, None, None, None, None) == 1
+
+
+def test_cpu_tensors_are_refused():
+    """The binding refuses host tensors for device arguments: there is no CPU path."""
+    L = _m2(batch=1, nheads=8, ngroups=1)
+    x = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(rs.ReplayError):
+        rs._step_in(L, dict(x=x, dt=x[..., 0], Bm=x, Cm=x, A=torch.zeros(8), D=torch.zeros(8)))

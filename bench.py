@@ -46,6 +46,12 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=60, help="windows timed end to end")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only-main", action="store_true",
+                    help="skip the Gated DeltaNet and speculative-verify measurements")
+    ap.add_argument("--batch", type=int, default=256,
+                    help="sequences of m2_serving (profiling captures use a smaller batch)")
+    ap.add_argument("--sub-steps", type=int, default=60,
+                    help="timed windows / rounds of the secondary measurements")
     return ap.parse_args()
 
 
@@ -183,7 +189,7 @@ def run_ours(args, rank, world):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    w = wl.make(WORKLOAD)
+    w = wl.make(WORKLOAD, B=args.batch)
     L = w.L
     pool = 4 * L  # distinct input steps, cycled (each step's inputs are 6 MiB)
     g = wl.Generator(w)
@@ -290,6 +296,14 @@ def run_ours(args, rank, world):
         "gpu_launches": args.steps * L,
         "e2e": e2e,
     }
+    if not args.only_main:
+        # free the m2_serving buffers before the other workloads
+        del state, S_full, inputs, step_in, y
+        torch.cuda.empty_cache()
+        line["gdn"] = bench_gdn(args, dev, peak, rs, bm, wl, torch)
+        torch.cuda.empty_cache()
+        line["verify"] = bench_verify(args, dev, peak, rs, bm, wl, torch)
+        torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample()
     if rank == 0:
@@ -357,6 +371,170 @@ def run_e2e(args, w, layer, state, st, Ad, Dd, dev, world, rs, torch, dist):
     return {"value": world * w.B * n_steps / (ms * 1e-3), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d * L, "d2h_bytes_per_step": d2h * L,
             "steps": args.e2e_steps, "pipelined": "H2D / decode / D2H on three streams"}
+
+
+def _events_ms(fn, n, stream, torch, dev):
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1)
+
+
+def bench_gdn(args, dev, peak, rs, bm, wl, torch):
+    """gdn_serving: Gated DeltaNet, batch 256, 32 heads, 128 x 128 state."""
+    w = wl.make("gdn_serving")
+    L, pool = w.L, 4 * w.L
+    g = wl.Generator(w)
+    S0 = g.initial_state()
+    st = {k: v.to(dev) for k, v in g.steps(pool).items()}
+    layer = rs.Layer("gdn", w.B, w.H, w.P, w.N, window=L, in_dtype=w.in_dtype)
+    state = rs.ReplayState(layer, device=dev)
+    rs.replayssm_init(layer, state, S0.to(dev))
+    S = S0.to(dev)
+    o = torch.empty(w.B, w.H, w.P, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    step_in = [{k: st[k][t] for k in st} for t in range(pool)]
+
+    def replay_window(wi):
+        for j in range(L):
+            rs.replayssm_decode_step(layer, state, step_in[(wi * L + j) % pool], o, stream)
+
+    def full_window(wi):
+        for j in range(L):
+            rs.replayssm_full_decode_step(layer, S, step_in[(wi * L + j) % pool], o, stream=stream)
+
+    n = args.sub_steps
+    for i in range(3):
+        replay_window(i)
+        full_window(i)
+    ms_r = _events_ms(replay_window, n, stream, torch, dev)
+    ms_f = _events_ms(full_window, n, stream, torch, dev)
+    if state.status() != 0:
+        raise RuntimeError(f"device status {state.status()} after the GDN run")
+    inb = 2
+    wb = bm.gdn_replay_window_bytes(L, w.N, w.P, inb) * w.B * w.H
+    fb = bm.gdn_conventional_bytes(w.N, w.P, inb) * w.B * w.H * L
+    ach_r = wb / (ms_r / n * 1e-3) / 1e9
+    ach_f = fb / (ms_f / n * 1e-3) / 1e9
+    tok = w.B * L * n
+    return {"workload": "gdn_serving", "value": tok / (ms_r * 1e-3), "unit": "tokens/s",
+            "ms_per_window": ms_r / n,
+            "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
+                         "frac": ach_r / peak, "kernel": "gdn_kernel<decode>"},
+            "full_state": {"value": tok / (ms_f * 1e-3), "unit": "tokens/s",
+                           "achieved_gbs": ach_f, "frac": ach_f / peak,
+                           "kernel": "gdn_kernel<full>"},
+            "replay_over_full": ms_f / ms_r,
+            "bytes_per_head_token": {"replay": wb / (w.B * w.H * L),
+                                     "full_state": fb / (w.B * w.H * L)},
+            "gpu_launches": n * L}
+
+
+def bench_verify(args, dev, peak, rs, bm, wl, torch):
+    """m2_verify: Mamba-2 m2_serving heads at batch 512, 4 drafts per round,
+    acceptance ~ U{0..4}; replay verify/commit against snapshot-and-restore
+    decoding of the full state."""
+    w = wl.make("m2_verify")
+    pool = 16
+    g = wl.Generator(w)
+    A, D = g.params()
+    S0 = g.initial_state()
+    rd = g.rounds(pool)
+    acc_host = rd["acc"].clone()
+    rd = {k: v.to(dev) for k, v in rd.items()}
+    Ad, Dd = A.to(dev), D.to(dev)
+    layer = rs.Layer("m2", w.B, w.H, w.P, w.N, ngroups=w.G, window=w.L, draft_max=w.n_draft,
+                     in_dtype=w.in_dtype)
+    state = rs.ReplayState(layer, device=dev)
+    rs.replayssm_init(layer, state, S0.to(dev))
+    y = torch.empty(w.B, w.n_draft, w.H, w.P, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    drafts = [dict(x=rd["x"][r], dt=rd["dt"][r], Bm=rd["Bm"][r], Cm=rd["Cm"][r], A=Ad, D=Dd)
+              for r in range(pool)]
+    n = args.sub_steps
+
+    def replay_round(r):
+        rs.replayssm_verify_commit(layer, state, rd["acc"][(r - 1) % pool] if r else None,
+                                   drafts[r % pool], y, stream)
+
+    for r in range(3):
+        replay_round(r)
+    rs.replayssm_commit(layer, state, rd["acc"][2 % pool], Ad, stream)
+    torch.cuda.synchronize(dev)
+    lens0 = state.len[:, 0].cpu().long()
+    def timed_round(r):
+        # timed round r evaluates draft set r+3; its predecessor's acceptance
+        # (set r+2) is committed first, except for r = 0 (already committed)
+        rs.replayssm_verify_commit(layer, state, rd["acc"][(r + 2) % pool] if r else None,
+                                   drafts[(r + 3) % pool], y, stream)
+
+    ms_r = _events_ms(timed_round, n, stream, torch, dev)
+    if state.status() != 0:
+        raise RuntimeError(f"device status {state.status()} after the verify run")
+    # algorithmic bytes: replay the length bookkeeping on the host
+    hpg = w.H // w.G
+    st_b, x_b, dt_b, bc_b, b_b, y_b = bm.m2_sizes(w.P, w.N, hpg, 2)
+    lens = lens0.clone()
+    total = 0.0
+    for r in range(n):
+        a = acc_host[(r + 2) % pool].long() if r else torch.zeros_like(lens)
+        n1 = lens + a
+        fold = n1 >= w.L
+        nb = torch.where(fold, torch.zeros_like(n1), n1)
+        per = (st_b + n1 * (x_b + 4 + b_b) + w.n_draft * ((x_b + dt_b + bc_b) + (x_b + 4 + bc_b))
+               + w.n_draft * y_b + fold.double() * st_b)
+        total += float(per.double().sum()) * w.H
+        lens = nb
+    ach_r = total / (ms_r * 1e-3) / 1e9
+    committed = float(sum(acc_host[(r + 2) % pool].sum() for r in range(1, n)))
+
+    # snapshot-and-restore conventional decoding of the full state
+    fl = rs.Layer("m2", w.B, w.H, w.P, w.N, ngroups=w.G, window=w.L, in_dtype=w.in_dtype)
+    S = S0.to(dev)
+    snap = torch.empty_like(S)
+    ysn = torch.empty(w.B, w.n_draft, w.H, w.P, device=dev)
+    junk = torch.empty(w.B, w.H, w.P, device=dev)
+
+    def snap_round(r):
+        i = r % pool
+        snap.copy_(S)
+        for d in range(w.n_draft):
+            inp = dict(x=rd["x"][i][:, d], dt=rd["dt"][i][:, d], Bm=rd["Bm"][i][:, d],
+                       Cm=rd["Cm"][i][:, d], A=Ad, D=Dd)
+            rs.replayssm_full_decode_step(fl, S, inp, ysn[:, d], stream=stream)
+        S.copy_(snap)
+        for d in range(w.n_draft):
+            inp = dict(x=rd["x"][i][:, d], dt=rd["dt"][i][:, d], Bm=rd["Bm"][i][:, d],
+                       Cm=rd["Cm"][i][:, d], A=Ad, D=Dd)
+            rs.replayssm_full_decode_step(fl, S, inp, junk, limit=rd["acc"][i], step_index=d,
+                                          stream=stream)
+
+    for r in range(2):
+        snap_round(r)
+    ms_s = _events_ms(snap_round, n, stream, torch, dev)
+    conv = bm.m2_conventional_bytes(w.P, w.N, hpg, 2)
+    snap_bytes = 0.0
+    for r in range(n):
+        a = acc_host[r % pool].double()
+        snap_bytes += float((4 * st_b + (w.n_draft + a) * conv).sum()) * w.H
+    ach_s = snap_bytes / (ms_s * 1e-3) / 1e9
+    rounds = n
+    return {"workload": "m2_verify", "rounds_per_s": rounds / (ms_r * 1e-3),
+            "ms_per_round": ms_r / rounds,
+            "drafts_evaluated_per_s": w.B * w.n_draft * rounds / (ms_r * 1e-3),
+            "committed_tokens_per_s": committed / (ms_r * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
+                         "frac": ach_r / peak, "kernel": "m2_verify_kernel"},
+            "snapshot_restore": {"rounds_per_s": rounds / (ms_s * 1e-3), "ms_per_round": ms_s / rounds,
+                                 "achieved_gbs": ach_s, "frac": ach_s / peak,
+                                 "kernels": "cudaMemcpyAsync x2 + m2_full_kernel x8"},
+            "replay_over_snapshot": ms_s / ms_r,
+            "gpu_launches": rounds}
 
 
 def main():

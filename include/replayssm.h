@@ -159,6 +159,9 @@ int32_t replayssm_capacity(const rssm_desc *desc);
  * invalid desc. */
 size_t replayssm_state_bytes(const rssm_desc *desc, int32_t which);
 const char *replayssm_status_string(rssm_status s);
+/* Text of the CUDA error behind the calling thread's most recent
+ * RSSM_ERR_CUDA return ("no error" if there was none).  Host only. */
+const char *replayssm_last_cuda_error(void);
 
 /* Start a state from a full state S0 (same layout as h0; device pointer):
  * h0 <- S0 (rounded to ckpt_fmt when set), len <- 0, read copy built from h0,

@@ -34,6 +34,7 @@ rssm_status check_desc(const rssm_desc *d) {
   if (d->kind == RSSM_MAMBA2) {
     if (d->ngroups <= 0 || d->nheads % d->ngroups != 0) return RSSM_ERR_SHAPE;
     if (!m2_supported(d->headdim, d->dstate)) return RSSM_ERR_SHAPE;
+    if (!m2_heads_supported(d->nheads / d->ngroups)) return RSSM_ERR_SHAPE;
     if ((int64_t)d->batch * d->ngroups > INT32_MAX) return RSSM_ERR_SHAPE;
   } else {
     if (!gdn_supported(d->dstate, d->headdim)) return RSSM_ERR_SHAPE;
@@ -63,7 +64,13 @@ rssm_status check_state(const rssm_desc *d, const rssm_state *s) {
 }
 
 inline cudaStream_t to_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
-inline rssm_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RSSM_OK : RSSM_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+inline rssm_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return RSSM_OK;
+  g_last_cuda_error = e;
+  return RSSM_ERR_CUDA;
+}
 
 inline int64_t stride_or(int64_t s, int64_t dense) { return s != 0 ? s : dense; }
 
@@ -213,6 +220,8 @@ const char *replayssm_status_string(rssm_status s) {
   }
 }
 
+const char *replayssm_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
+
 rssm_status replayssm_init(const rssm_desc *d, rssm_state *s, const float *S0, void *stream) {
   rssm_status st = check_desc(d);
   if (st != RSSM_OK) return st;
@@ -279,6 +288,7 @@ rssm_status replayssm_verify_commit(const rssm_desc *d, rssm_state *s,
   if (d->read_fmt != RSSM_FMT_NONE || d->ckpt_fmt != RSSM_FMT_NONE) return RSSM_ERR_UNSUPPORTED;
   if ((st = check_state(d, s)) != RSSM_OK) return st;
   if (n_draft < 1 || n_draft > d->draft_max) return RSSM_ERR_CAPACITY;
+  if (d->nheads / d->ngroups > 8) return RSSM_ERR_UNSUPPORTED;  // one CTA per group
   if (!y) return RSSM_ERR_INVALID_ARG;
   if ((st = check_m2_inputs(drafts, true)) != RSSM_OK) return st;
   M2Params p = m2_params(d, s);

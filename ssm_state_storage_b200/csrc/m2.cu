@@ -24,24 +24,34 @@
 // registers with 128-bit loads: lane (rs = lane/8, c8 = lane%8) of warp w holds
 // rows w*P/8 + rs + 4*rho and columns 32*s + 4*c8, so each quarter-warp reads
 // one 128-byte line and the row sums need only 3 shuffle levels.
+#include <type_traits>
+
 #include "codec.cuh"
 #include "common.cuh"
 #include "internal.h"
+#include "pipeline.cuh"
 
 namespace rssm {
 namespace {
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
 
 __device__ __forceinline__ float sum8(float v) {  // over the 8 lanes of a quarter-warp
   v += __shfl_xor_sync(0xffffffffu, v, 1);
   v += __shfl_xor_sync(0xffffffffu, v, 2);
   v += __shfl_xor_sync(0xffffffffu, v, 4);
   return v;
+}
+
+// Dot product of C4 float4 pairs summed as a balanced tree.
+template <int C4>
+__device__ __forceinline__ float tree_dot(const float4 (&a)[C4], const float4 (&b)[C4]) {
+  float d[C4];
+#pragma unroll
+  for (int s = 0; s < C4; ++s) d[s] = (a[s].x * b[s].x + a[s].y * b[s].y) + (a[s].z * b[s].z + a[s].w * b[s].w);
+#pragma unroll
+  for (int w = 1; w < C4; w <<= 1)
+#pragma unroll
+    for (int s = 0; s + w < C4; s += 2 * w) d[s] += d[s + w];
+  return d[0];
 }
 
 template <int P, int N>
@@ -97,7 +107,7 @@ __device__ __forceinline__ void load_read_view(const M2Params &p, size_t bh, int
 template <int P, int N>
 __device__ __forceinline__ void quantize_tile(const M2Params &p, size_t bh, int fmt, bool roundtrip,
                                               float4 (&v)[P / 32][N / 32], float *s_red, int warp,
-                                              int lane, int rs, int c8) {
+                                              int lane, int rs, int c8, int bar_threads = 0) {
   using T = Tile<P, N>;
   if (fmt == 1) {
     uint8_t *rc = p.rc + bh * (size_t)(P * N);
@@ -129,7 +139,8 @@ __device__ __forceinline__ void quantize_tile(const M2Params &p, size_t bh, int 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) s_red[warp] = m;
-  __syncthreads();
+  if (bar_threads) bar_sync(2, bar_threads);  // the consumer warps only
+  else __syncthreads();
   float amax = s_red[0];
 #pragma unroll
   for (int w = 1; w < 8; ++w) amax = fmaxf(amax, s_red[w]);
@@ -182,28 +193,59 @@ __device__ __forceinline__ void store_tile(float *tile, int warp, int rs, int c8
       st_stream(tile + (size_t)T::row(warp, rs, rho) * N + T::col(c8, s), v[rho][s]);
 }
 
-// Decay weights of k records by warp 0 (lane i owns record i):
-//   s_wdt[i] = exp(A * sum_{i<m<k} dt_m) * dt_i,  *s_lam = exp(A * sum_{m<k} dt_m).
-// Each lane sums its suffix in a fixed order, so results do not depend on timing.
-__device__ __forceinline__ void decay_weights(const float *s_dt, int k, float A, float *s_wdt,
-                                              float *s_lam, int lane) {
+// Decay weights of k records for one head, by one warp (lane i owns record i):
+//   wdt[i] = exp(A * sum_{i<m<k} dt_m) * dt_i,   *lam = exp(A * sum_{m<k} dt_m).
+// The suffix sums come from a shuffle scan (fixed association order, so the
+// result does not depend on timing); every dt term is non-negative, so no
+// cancellation occurs.  Sums, products and exponentials are taken in fp64 (a
+// handful per head; B200 runs fp64 at half the fp32 rate): an fp32 exp(A s)
+// would carry a relative error of about |A s| * 2^-24 into every weight.
+__device__ __forceinline__ void decay_weights_scan(const float *dt, int k, float A, float *wdt,
+                                                   float *lam, int lane) {
+  const double mine = lane < k ? (double)dt[lane] : 0.0;
+  double s = lane + 1 < k ? (double)dt[lane + 1] : 0.0;  // suffix of the records after this one
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double t = __shfl_down_sync(0xffffffffu, s, o);
+    if (lane + o < 32) s += t;
+  }
+  const double a = A;
+  if (lane < k) wdt[lane] = (float)(exp(a * s) * mine);
+  if (lane == 0) *lam = (float)exp(a * (s + mine));
+}
+
+__device__ __forceinline__ void decay_weights(const float *dt, int k, float A, float *wdt,
+                                              float *lam, int lane) {
+  const double a = A;
   if (lane < k) {
-    float s = 0.f;
-    for (int m = lane + 1; m < k; ++m) s += s_dt[m];
-    s_wdt[lane] = expf(A * s) * s_dt[lane];
+    double s = 0.0;
+    for (int m = lane + 1; m < k; ++m) s += dt[m];
+    wdt[lane] = (float)(exp(a * s) * (double)dt[lane]);
   }
   if (lane == 0) {
-    float t = 0.f;
-    for (int m = 0; m < k; ++m) t += s_dt[m];
-    *s_lam = expf(A * t);
+    double t = 0.0;
+    for (int m = 0; m < k; ++m) t += dt[m];
+    *lam = (float)exp(a * t);
   }
 }
 
 // h <- lam * h + sum_{i<k} (wdt_i x_i[r]) B_i[cols]  -- the fold, in registers.
-template <int P, int N>
+// x: the head's records [k][P] (input dtype); B: the group's records [k][N] fp32.
+template <typename TB>
+__device__ __forceinline__ float4 ld4_smem(const TB *p) {
+  if constexpr (sizeof(TB) == 4) {
+    return *reinterpret_cast<const float4 *>(p);
+  } else {
+    const uint2 raw = *reinterpret_cast<const uint2 *>(p);
+    const TB *e = reinterpret_cast<const TB *>(&raw);
+    return make_float4(to_f32(e[0]), to_f32(e[1]), to_f32(e[2]), to_f32(e[3]));
+  }
+}
+
+template <int P, int N, typename TI, typename TB = float>
 __device__ __forceinline__ void fold_regs(float4 (&hv)[P / 32][N / 32], float lam, int k,
-                                          const float *s_wdt, const float (*s_x)[P],
-                                          const float (*s_B)[N], int warp, int rs, int c8) {
+                                          const float *wdt, const TI *x, const TB *Bs,
+                                          int warp, int rs, int c8) {
   using T = Tile<P, N>;
 #pragma unroll
   for (int rho = 0; rho < T::RPT; ++rho) {
@@ -216,10 +258,10 @@ __device__ __forceinline__ void fold_regs(float4 (&hv)[P / 32][N / 32], float la
       hv[rho][s].w *= lam;
     }
     for (int i = 0; i < k; ++i) {
-      const float xw = s_wdt[i] * s_x[i][r];
+      const float xw = wdt[i] * to_f32(x[i * P + r]);
 #pragma unroll
       for (int s = 0; s < T::C4; ++s) {
-        const float4 bb = *reinterpret_cast<const float4 *>(&s_B[i][T::col(c8, s)]);
+        const float4 bb = ld4_smem<TB>(&Bs[i * N + T::col(c8, s)]);
         hv[rho][s].x = fmaf(xw, bb.x, hv[rho][s].x);
         hv[rho][s].y = fmaf(xw, bb.y, hv[rho][s].y);
         hv[rho][s].z = fmaf(xw, bb.z, hv[rho][s].z);
@@ -229,157 +271,786 @@ __device__ __forceinline__ void fold_regs(float4 (&hv)[P / 32][N / 32], float la
   }
 }
 
+// The fold with the record loop outermost: each B_i fragment (fp32 in shared
+// memory) is loaded once and used for all of the thread's rows.
+template <int P, int N, typename TI>
+__device__ __forceinline__ void fold_regs_hoisted(float4 (&hv)[P / 32][N / 32], float lam, int k,
+                                                  const float *wdt, const TI *x, const float *Bf,
+                                                  int warp, int rs, int c8) {
+  using T = Tile<P, N>;
+#pragma unroll
+  for (int rho = 0; rho < T::RPT; ++rho)
+#pragma unroll
+    for (int s = 0; s < T::C4; ++s) {
+      hv[rho][s].x *= lam;
+      hv[rho][s].y *= lam;
+      hv[rho][s].z *= lam;
+      hv[rho][s].w *= lam;
+    }
+  // two accumulation chains (even / odd records): shorter rounding chains and
+  // independent FMA streams
+  float4 acc[T::RPT][T::C4];
+#pragma unroll
+  for (int rho = 0; rho < T::RPT; ++rho)
+#pragma unroll
+    for (int s = 0; s < T::C4; ++s) acc[rho][s] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = 0; i < k; ++i) {
+    float4 bb[T::C4];
+#pragma unroll
+    for (int s = 0; s < T::C4; ++s)
+      bb[s] = *reinterpret_cast<const float4 *>(&Bf[i * N + T::col(c8, s)]);
+    const float w = wdt[i];
+    const bool odd = i & 1;
+#pragma unroll
+    for (int rho = 0; rho < T::RPT; ++rho) {
+      const float xw = w * to_f32(x[i * P + T::row(warp, rs, rho)]);
+#pragma unroll
+      for (int s = 0; s < T::C4; ++s) {
+        float4 &d = odd ? acc[rho][s] : hv[rho][s];
+        d.x = fmaf(xw, bb[s].x, d.x);
+        d.y = fmaf(xw, bb[s].y, d.y);
+        d.z = fmaf(xw, bb[s].z, d.z);
+        d.w = fmaf(xw, bb[s].w, d.w);
+      }
+    }
+  }
+#pragma unroll
+  for (int rho = 0; rho < T::RPT; ++rho)
+#pragma unroll
+    for (int s = 0; s < T::C4; ++s) {
+      hv[rho][s].x += acc[rho][s].x;
+      hv[rho][s].y += acc[rho][s].y;
+      hv[rho][s].z += acc[rho][s].z;
+      hv[rho][s].w += acc[rho][s].w;
+    }
+}
+
 // After a fold: round the checkpoint (qmode 3/4), store it, refresh the read
-// copy (qmode 1/2).
+// copy (qmode 1/2).  NVFP4 variants synchronise the CTA.
 template <int P, int N, int QM>
 __device__ __forceinline__ void commit_checkpoint(const M2Params &p, size_t bh, float *dst,
                                                   float4 (&hv)[P / 32][N / 32], float *s_red,
-                                                  int warp, int lane, int rs, int c8) {
-  if constexpr (QM >= 3) quantize_tile<P, N>(p, bh, QM - 2, true, hv, s_red, warp, lane, rs, c8);
+                                                  int warp, int lane, int rs, int c8,
+                                                  int bar_threads = 0) {
+  if constexpr (QM >= 3)
+    quantize_tile<P, N>(p, bh, QM - 2, true, hv, s_red, warp, lane, rs, c8, bar_threads);
   store_tile<P, N>(dst, warp, rs, c8, hv);
-  if constexpr (QM == 1 || QM == 2) quantize_tile<P, N>(p, bh, QM, false, hv, s_red, warp, lane, rs, c8);
+  if constexpr (QM == 1 || QM == 2)
+    quantize_tile<P, N>(p, bh, QM, false, hv, s_red, warp, lane, rs, c8, bar_threads);
+}
+
+// Heads handled by one CTA: the whole group when it has at most 8 heads,
+// otherwise chunks of 8 (the host requires H/G <= 8 or a multiple of 8).
+__host__ __device__ __forceinline__ int head_chunk(int hpg) { return hpg <= 8 ? hpg : 8; }
+
+// Copy `count` elements of T from global to shared memory as fp32, 16 bytes
+// per load (both ends 16-byte aligned, count a multiple of 16 / sizeof(T)).
+template <typename T>
+__device__ __forceinline__ void stage_f32(float *dst, const T *src, int count, int tid) {
+  constexpr int V = 16 / sizeof(T);
+  const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+  for (int v = tid; v < count / V; v += kThreads) {
+    const uint4 raw = s4[v];
+    const T *e = reinterpret_cast<const T *>(&raw);
+#pragma unroll
+    for (int j = 0; j < V; ++j) dst[v * V + j] = to_f32(e[j]);
+  }
+}
+
+// Copy `bytes` (multiple of 16) from global to shared memory unchanged.
+__device__ __forceinline__ void stage_raw(void *dst, const void *src, int bytes, int tid) {
+  const uint4 *s4 = static_cast<const uint4 *>(src);
+  uint4 *d4 = static_cast<uint4 *>(dst);
+  for (int v = tid; v < bytes / 16; v += kThreads) d4[v] = s4[v];
+}
+
+__host__ __device__ __forceinline__ int pad4(int n) { return (n + 3) & ~3; }
+
+// Shared-memory layout of the decode / fold kernels (floats unless noted):
+//   B [L][N] | C [N] | bc [pad4(L)] | dt [hc][L] | wdt [hc][L] | lam [pad4(hc)]
+//   | red [2][8] (tile maxima, alternating between consecutive heads) | x [hc][L][P] (input dtype)
+struct DecodeSmem {
+  float *B, *C, *bc, *dt, *wdt, *lam, *red;
+  void *x;
+  __host__ __device__ static size_t bytes(int L, int hc, int P, int N, int es) {
+    const size_t f = (size_t)L * N + N + pad4(L) + 2 * pad4(hc * L) + pad4(hc) + 16;
+    return f * 4 + (size_t)hc * L * P * es;
+  }
+  __device__ DecodeSmem(unsigned char *base, int L, int hc, int N) {
+    float *f = reinterpret_cast<float *>(base);
+    B = f;
+    C = B + L * N;
+    bc = C + N;
+    dt = bc + pad4(L);
+    wdt = dt + pad4(hc * L);
+    lam = wdt + pad4(hc * L);
+    red = lam + pad4(hc);
+    x = red + 16;
+  }
+};
+
+// ------------------------------------------------------------- row helpers
+// One row of a P x N head tile as seen by one lane of the decode kernel:
+// columns 32 s + 4 c8 (s < N/32), four values each.
+
+template <int P, int N, int QM>
+__device__ __forceinline__ void view_row(const unsigned char *t, int r, int c8, float sg,
+                                         float4 (&v)[N / 32]) {
+#pragma unroll
+  for (int s = 0; s < N / 32; ++s) {
+    const int c = 32 * s + 4 * c8;
+    if constexpr (QM == 1) {
+      const uint32_t w = *reinterpret_cast<const uint32_t *>(t + r * N + c);
+      v[s] = make_float4(e4m3_decode(w & 0xFF), e4m3_decode((w >> 8) & 0xFF),
+                         e4m3_decode((w >> 16) & 0xFF), e4m3_decode(w >> 24));
+    } else if constexpr (QM == 2) {
+      const uint32_t w = *reinterpret_cast<const uint16_t *>(t + r * (N / 2) + c / 2);
+      const float sb = e4m3_decode(t[P * N / 2 + r * (N / 16) + c / 16]);
+      v[s] = make_float4(nvfp4_value(w & 0xF, sb, sg), nvfp4_value((w >> 4) & 0xF, sb, sg),
+                         nvfp4_value((w >> 8) & 0xF, sb, sg), nvfp4_value((w >> 12) & 0xF, sb, sg));
+    } else {
+      v[s] = *reinterpret_cast<const float4 *>(t + (r * N + c) * 4);
+    }
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void load_row(const float *tile, int r, int c8, float4 (&v)[N / 32]) {
+#pragma unroll
+  for (int s = 0; s < N / 32; ++s) v[s] = ld_stream(tile + (size_t)r * N + 32 * s + 4 * c8);
+}
+
+template <int N>
+__device__ __forceinline__ void store_row(float *tile, int r, int c8, const float4 (&v)[N / 32]) {
+#pragma unroll
+  for (int s = 0; s < N / 32; ++s) st_stream(tile + (size_t)r * N + 32 * s + 4 * c8, v[s]);
+}
+
+// The fold of RGC register-held rows of one head:
+//   v[u] <- lam v[u] + sum_{i<k} (w_i x_i[rows[u]]) B_i[cols],
+// record loop outermost so that each B_i fragment (fp32 in shared memory) is
+// loaded once and feeds 4 * RGC * (N/32) independent FMAs.
+template <int P, int N, typename TI, int RGC>
+__device__ __forceinline__ void fold_rows(float4 (&v)[RGC][N / 32], float lam, int k,
+                                          const float *w, const TI *x, const int (&rows)[RGC],
+                                          const float *Bf, int c8) {
+#pragma unroll
+  for (int u = 0; u < RGC; ++u)
+#pragma unroll
+    for (int s = 0; s < N / 32; ++s)
+      v[u][s] = make_float4(lam * v[u][s].x, lam * v[u][s].y, lam * v[u][s].z, lam * v[u][s].w);
+  for (int i = 0; i < k; ++i) {
+    float4 bb[N / 32];
+#pragma unroll
+    for (int s = 0; s < N / 32; ++s)
+      bb[s] = *reinterpret_cast<const float4 *>(&Bf[i * N + 32 * s + 4 * c8]);
+    const float wi = w[i];
+#pragma unroll
+    for (int u = 0; u < RGC; ++u) {
+      const float xw = wi * to_f32(x[i * P + rows[u]]);
+#pragma unroll
+      for (int s = 0; s < N / 32; ++s) {
+        v[u][s].x = fmaf(xw, bb[s].x, v[u][s].x);
+        v[u][s].y = fmaf(xw, bb[s].y, v[u][s].y);
+        v[u][s].z = fmaf(xw, bb[s].z, v[u][s].z);
+        v[u][s].w = fmaf(xw, bb[s].w, v[u][s].w);
+      }
+    }
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void fp8_roundtrip_row(float4 (&v)[N / 32]) {
+#pragma unroll
+  for (int s = 0; s < N / 32; ++s)
+    v[s] = make_float4(e4m3_decode(e4m3_encode(v[s].x)), e4m3_decode(e4m3_encode(v[s].y)),
+                       e4m3_decode(e4m3_encode(v[s].z)), e4m3_decode(e4m3_encode(v[s].w)));
+}
+
+template <int N>
+__device__ __forceinline__ void fp8_codes_row(uint8_t *rc_tile, int r, int c8,
+                                              const float4 (&v)[N / 32]) {
+#pragma unroll
+  for (int s = 0; s < N / 32; ++s) {
+    const uint32_t w = e4m3_encode(v[s].x) | (e4m3_encode(v[s].y) << 8) |
+                       (e4m3_encode(v[s].z) << 16) | (e4m3_encode(v[s].w) << 24);
+    *reinterpret_cast<uint32_t *>(rc_tile + (size_t)r * N + 32 * s + 4 * c8) = w;
+  }
+}
+
+template <int N>
+__device__ __forceinline__ float absmax_row(const float4 (&v)[N / 32]) {
+  float m = 0.f;
+#pragma unroll
+  for (int s = 0; s < N / 32; ++s)
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(v[s].x), fabsf(v[s].y)), fmaxf(fabsf(v[s].z), fabsf(v[s].w))));
+  return m;
+}
+
+// NVFP4 of one row given the tile scale: block maxima over the 4 lanes that
+// share a 16-column block, then codes (written) or deq(Q(v)) (roundtrip).
+template <int P, int N>
+__device__ __forceinline__ void nvfp4_row(float4 (&v)[N / 32], float sg, bool roundtrip,
+                                          uint8_t *rc_tile, uint8_t *sc_tile, int r, int c8) {
+#pragma unroll
+  for (int s = 0; s < N / 32; ++s) {
+    const int c = 32 * s + 4 * c8;
+    float bm = fmaxf(fmaxf(fabsf(v[s].x), fabsf(v[s].y)), fmaxf(fabsf(v[s].z), fabsf(v[s].w)));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+    const uint32_t scode = nvfp4_block_code(bm, sg);
+    const float d = nvfp4_step(scode, sg);
+    const uint32_t lo = nvfp4_pack2(v[s].x, v[s].y, d), hi = nvfp4_pack2(v[s].z, v[s].w, d);
+    if (roundtrip) {
+      const float sb = e4m3_decode(scode);
+      v[s] = make_float4(nvfp4_value(lo & 0xF, sb, sg), nvfp4_value(lo >> 4, sb, sg),
+                         nvfp4_value(hi & 0xF, sb, sg), nvfp4_value(hi >> 4, sb, sg));
+    } else {
+      *reinterpret_cast<uint16_t *>(rc_tile + (size_t)r * (N / 2) + c / 2) = (uint16_t)(lo | (hi << 8));
+      if ((c8 & 3) == 0) sc_tile[(size_t)r * (N / 16) + c / 16] = (uint8_t)scode;
+    }
+  }
 }
 
 // =============================================================== decode step
+// Persistent, warp-specialised kernel: one CTA per SM walks work items
+// (sequence, group, head chunk) in a static round-robin.  Warp 8 is the
+// producer: for each item it reads the buffer length, bulk-copies the
+// item's buffered records (the group's B records, every head's x records)
+// into one of two record buffers, then streams the item's checkpoint tiles
+// (or read-copy tiles) into a ring of NS shared-memory slots, each slot's
+// arrival tracked by an mbarrier.  Warps 0-7 consume: per item they add this
+// step's record, form the B_i.C_k dots and every head's decay weights, then
+// for each head pull the tile from the ring into registers, release the slot,
+// write y and, on the flush step, fold the tile and write it back.
+// HBM traffic therefore overlaps all per-item setup work.
 
-template <int P, int N, typename TI, int QM>
-__global__ void __launch_bounds__(kThreads, 2) m2_decode_kernel(const M2Params p) {
+// Byte layout of the decode kernel's shared memory (host and device agree).
+// Per record buffer rb (NR = 1 to 3 of them): the group's B records
+// [L][N] and every head's x records [hc][L][P] (input dtype; slot k-1 holds
+// this step's record), plus a small "stage" block of fp32 values written by
+// the producer warp: C_k [N], dt records [hc][L], A [hc], D [hc], header.
+struct DecodeLayout {
+  int NS, NR, hc, L, tile_bytes, tile_stride, stage_floats, scratch_floats;
+  int off_bars, off_recB, off_recX, off_stage, off_scr, off_ring, total;
+
+  __host__ __device__ static int align128(int v) { return (v + 127) & ~127; }
+
+  __host__ static DecodeLayout make(int P, int N, int hc, int L, int es, int qm, int budget) {
+    DecodeLayout d;
+    d.hc = hc;
+    d.L = L;
+    d.tile_bytes = qm == 1 ? P * N : qm == 2 ? P * N / 2 + P * N / 16 : P * N * 4;
+    d.tile_stride = align128(d.tile_bytes);
+    d.stage_floats = N + pad4(hc * L) + 2 * pad4(hc) + 4;
+    d.scratch_floats = 2 * pad4(L) + 2 * pad4(hc * L) + pad4(hc) + 32 + L * N + hc * P;
+    const int rec_b = L * N * es, rec_x = hc * L * P * es;
+    // Prefer three record buffers (the stager then runs two items ahead, which
+    // hides its two dependent memory round trips) as long as the ring keeps
+    // at least 3 slots; fall back to fewer buffers for large tiles.
+    for (d.NR = 3; d.NR >= 1; --d.NR) {
+      int o = 0;
+      d.off_bars = o;
+      o += align128(8 * (2 * 8 + 2 * 4));  // room for up to 8 slots and 4 record buffers
+      d.off_recB = o;
+      o += align128(d.NR * rec_b);
+      d.off_recX = o;
+      o += align128(d.NR * rec_x);
+      d.off_stage = o;
+      o += align128(d.NR * d.stage_floats * 4);
+      d.off_scr = o;
+      o += align128(2 * d.scratch_floats * 4);
+      d.off_ring = o;
+      const int room = budget - o;
+      d.NS = room / d.tile_stride;
+      if (d.NS > 8) d.NS = 8;
+      if (d.NS >= (d.NR == 1 ? 2 : 3)) {
+        d.total = o + d.NS * d.tile_stride;
+        return d;
+      }
+    }
+    d.NS = 0;
+    return d;
+  }
+};
+
+// Read view of a head tile held in shared memory (fp32, FP8 or NVFP4 codes).
+template <int P, int N, int QM>
+__device__ __forceinline__ void view_from_smem(const unsigned char *t, float sg, int warp, int rs,
+                                               int c8, float4 (&v)[P / 32][N / 32]) {
   using T = Tile<P, N>;
-  constexpr int RPT = T::RPT, C4 = T::C4;
-  __shared__ __align__(16) float s_B[kMaxCap][N];
-  __shared__ __align__(16) float s_x[kMaxCap][P];
-  __shared__ __align__(16) float s_C[N];
-  __shared__ float s_bc[kMaxCap], s_dt[kMaxCap], s_wdt[kMaxCap], s_coef[kMaxCap];
-  __shared__ float s_lam, s_red[8];
-  __shared__ int s_k;
+#pragma unroll
+  for (int rho = 0; rho < T::RPT; ++rho)
+#pragma unroll
+    for (int s = 0; s < T::C4; ++s) {
+      const int r = T::row(warp, rs, rho), c = T::col(c8, s);
+      if constexpr (QM == 1) {
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(t + r * N + c);
+        v[rho][s] = make_float4(e4m3_decode(w & 0xFF), e4m3_decode((w >> 8) & 0xFF),
+                                e4m3_decode((w >> 16) & 0xFF), e4m3_decode(w >> 24));
+      } else if constexpr (QM == 2) {
+        const uint32_t w = *reinterpret_cast<const uint16_t *>(t + r * (N / 2) + c / 2);
+        const float sb = e4m3_decode(t[P * N / 2 + r * (N / 16) + c / 16]);
+        v[rho][s] = make_float4(nvfp4_value(w & 0xF, sb, sg), nvfp4_value((w >> 4) & 0xF, sb, sg),
+                                nvfp4_value((w >> 8) & 0xF, sb, sg),
+                                nvfp4_value((w >> 12) & 0xF, sb, sg));
+      } else {
+        v[rho][s] = *reinterpret_cast<const float4 *>(t + (r * N + c) * 4);
+      }
+    }
+}
+
+struct DecodeSmemPtrs {
+  uint64_t *full, *empty, *rfull, *rempty;
+  unsigned char *ring;
+  unsigned char *recB, *recX;
+  float *stage, *scr;
+  __device__ DecodeSmemPtrs(unsigned char *smem, const DecodeLayout &lay) {
+    full = reinterpret_cast<uint64_t *>(smem + lay.off_bars);
+    empty = full + 8;
+    rfull = empty + 8;
+    rempty = rfull + 4;
+    ring = smem + lay.off_ring;
+    recB = smem + lay.off_recB;
+    recX = smem + lay.off_recX;
+    stage = reinterpret_cast<float *>(smem + lay.off_stage);
+    scr = reinterpret_cast<float *>(smem + lay.off_scr);
+  }
+};
+
+// Stage block of record buffer rb: C [N] | dt [hc][L] | A [hc] | D [hc] | hdr [4]
+// (hdr: n0, bad, gscale (NVFP4 tile scales are read per head by consumers)).
+struct Stage {
+  float *C, *dt, *A, *D;
+  int *hdr;
+  __device__ Stage(float *base, int N, int hc, int L) {
+    C = base;
+    dt = C + N;
+    A = dt + pad4(hc * L);
+    D = A + pad4(hc);
+    hdr = reinterpret_cast<int *>(D + pad4(hc));
+  }
+};
+
+__device__ __forceinline__ void item_coords(const M2Params &p, int item, int nchunk, int hc, int &b,
+                                            int &g, int &chunk, int &h_first) {
+  const int bg_i = item / nchunk;
+  chunk = item - bg_i * nchunk;
+  b = bg_i / p.G;
+  g = bg_i - b * p.G;
+  h_first = g * p.hpg + chunk * hc;
+}
+
+// Stager warp: for item `it` wait until its record buffer is free, then stage
+// the small per-item inputs.  Every global load of the item is issued first
+// into registers (none depends on the buffer length: all `window` dt slots
+// are read), so the item costs one memory latency; then the values are
+// written to shared memory, and lane 0 bulk-copies the buffered records and
+// arrives on the buffer's barrier.
+template <int P, int N, typename TI>
+__device__ __forceinline__ bool stage_item(const M2Params &p, const DecodeLayout &lay,
+                                           const DecodeSmemPtrs &S, int item, int it, int nchunk,
+                                           int lane) {
+  constexpr int NPL = N / 32;          // B and C values per lane
+  constexpr int XPL = 8 * P / 32;      // x values per lane (up to 8 heads)
+  constexpr int DPL = 8 * 16 / 32;     // dt slots per lane (up to 8 heads x 16)
+  const int hc = lay.hc, L = lay.L;
+  const int rb = it % lay.NR;
+  const uint32_t rphase = (it / lay.NR) & 1;
+  bool ok = true;
+  if (lane == 0) ok = mbar_wait(&S.rempty[rb], rphase ^ 1);
+  if (!__shfl_sync(0xffffffffu, (int)ok, 0)) return false;
+  int b, g, chunk, h_first;
+  item_coords(p, item, nchunk, hc, b, g, chunk, h_first);
+  const size_t bh0 = (size_t)b * p.H + h_first;
+  const TI *__restrict__ Bin = static_cast<const TI *>(p.Bm) + b * p.bs_B + (size_t)g * N;
+  const TI *__restrict__ Cin = static_cast<const TI *>(p.Cm) + b * p.bs_C + (size_t)g * N;
+  const TI *__restrict__ xin = static_cast<const TI *>(p.x) + b * p.bs_x + (size_t)h_first * P;
+
+  // ---- phase 1: every load of the item, independent of one another
+  const int my_len = lane < hc ? __ldcg(&p.len[bh0 + lane]) : 0;
+  const float my_A = lane < hc ? p.A[h_first + lane] : 0.f;
+  const float my_D = lane < hc ? p.D[h_first + lane] : 0.f;
+  const float my_dt = lane < hc ? ld_in<TI>(p.dt, b * p.bs_dt + h_first + lane) : 0.f;
+  TI bv[NPL], cv[NPL], xv[XPL];
+  float dtv[DPL];
+#pragma unroll
+  for (int u = 0; u < NPL; ++u) {
+    bv[u] = Bin[lane + 32 * u];
+    cv[u] = Cin[lane + 32 * u];
+  }
+#pragma unroll
+  for (int u = 0; u < XPL; ++u) {
+    const int e = lane + 32 * u;
+    xv[u] = e < hc * P ? xin[e] : TI{};
+  }
+#pragma unroll
+  for (int u = 0; u < DPL; ++u) {
+    const int e = lane + 32 * u, j = e / L, i = e - j * L;
+    dtv[u] = e < hc * L ? __ldcg(&p.dtbuf[(bh0 + j) * p.cap + i]) : 0.f;
+  }
+
+  // ---- phase 2: buffer length and its checks
+  const int n0 = __shfl_sync(0xffffffffu, my_len, 0);
+  const bool bad = __any_sync(0xffffffffu, (lane < hc && my_len != n0) || n0 < 0 || n0 >= L);
+  const int k = min(max(n0 + 1, 1), L);  // copies stay in bounds even for a bad length
+
+  // ---- phase 3: shared-memory writes
+  Stage st(S.stage + rb * lay.stage_floats, N, hc, L);
+  TI *rB = reinterpret_cast<TI *>(S.recB) + (size_t)rb * L * N;
+  TI *rX = reinterpret_cast<TI *>(S.recX) + (size_t)rb * hc * L * P;
+#pragma unroll
+  for (int u = 0; u < NPL; ++u) {
+    rB[(k - 1) * N + lane + 32 * u] = bv[u];
+    st.C[lane + 32 * u] = to_f32(cv[u]);
+  }
+#pragma unroll
+  for (int u = 0; u < XPL; ++u) {
+    const int e = lane + 32 * u, j = e / P, q = e - j * P;
+    if (e < hc * P) rX[(j * L + k - 1) * P + q] = xv[u];
+  }
+#pragma unroll
+  for (int u = 0; u < DPL; ++u) {
+    const int e = lane + 32 * u, j = e / L, i = e - j * L;
+    const float cur = __shfl_sync(0xffffffffu, my_dt, j < 32 ? j : 0);
+    if (e < hc * L) st.dt[e] = i == k - 1 ? cur : dtv[u];
+  }
+  if (lane < hc) {
+    st.A[lane] = my_A;
+    st.D[lane] = my_D;
+  }
+  if (lane == 0) {
+    st.hdr[0] = n0;
+    st.hdr[1] = bad;
+  }
+  fence_proxy_async_smem();  // these generic writes precede later bulk copies into the buffer
+  __syncwarp();
+  if (lane == 0) {
+    const uint32_t bytesB = (k - 1) * N * sizeof(TI), bytesX = (k - 1) * P * sizeof(TI);
+    mbar_arrive_expect_tx(&S.rfull[rb], bytesB + hc * bytesX);
+    if (k > 1) {
+      const size_t bg = (size_t)b * p.G + g;
+      bulk_g2s(rB, static_cast<const TI *>(p.Bbuf) + bg * p.cap * N, bytesB, &S.rfull[rb]);
+      for (int j = 0; j < hc; ++j)
+        bulk_g2s(rX + (size_t)j * L * P, static_cast<const TI *>(p.xbuf) + (bh0 + j) * p.cap * P,
+                 bytesX, &S.rfull[rb]);
+    }
+  }
+  return true;
+}
+
+template <int P, int N, typename TI>
+__device__ __forceinline__ void decode_stager(const M2Params &p, const DecodeLayout &lay,
+                                              const DecodeSmemPtrs &S, volatile int *abort_flag,
+                                              int nitems, int nchunk, int lane) {
+  int it = 0;
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+    // warp-uniform view of the abort flag: every lane takes the same branch
+    const bool abort_now = __any_sync(0xffffffffu, *abort_flag != 0);
+    if (abort_now || !stage_item<P, N, TI>(p, lay, S, item, it, nchunk, lane)) {
+      if (lane == 0 && !abort_now) {
+        report(p.status, RSSM_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      return;  // nothing of ours is in flight: a wait gave up before any copy
+    }
+  }
+}
+
+// Tile producer (one lane): streams the items' checkpoint (or read-copy)
+// tiles into the ring, waiting only for free slots.
+template <int P, int N, int QM>
+__device__ __forceinline__ void decode_tiles(const M2Params &p, const DecodeLayout &lay,
+                                             const DecodeSmemPtrs &S, volatile int *abort_flag,
+                                             int nitems, int nchunk) {
+  const int hc = lay.hc;
+  int slot = 0;
+  uint32_t sphase = 0;
+  uint32_t issued = 0, parity = 0;  // per slot: a copy was issued / its phase parity
+  bool failed = false;
+  for (int item = blockIdx.x; item < nitems && !failed; item += gridDim.x) {
+    int b, g, chunk, h_first;
+    item_coords(p, item, nchunk, hc, b, g, chunk, h_first);
+    const size_t bh0 = (size_t)b * p.H + h_first;
+    for (int j = 0; j < hc; ++j) {
+      if (*abort_flag || !mbar_wait(&S.empty[slot], sphase ^ 1)) {
+        failed = true;
+        break;
+      }
+      mbar_arrive_expect_tx(&S.full[slot], lay.tile_bytes);
+      unsigned char *dst = S.ring + slot * lay.tile_stride;
+      const size_t bh = bh0 + j;
+      if constexpr (QM == 1) {
+        bulk_g2s(dst, p.rc + bh * (size_t)(P * N), P * N, &S.full[slot]);
+      } else if constexpr (QM == 2) {
+        bulk_g2s(dst, p.rc + bh * (size_t)(P * N / 2), P * N / 2, &S.full[slot]);
+        bulk_g2s(dst + P * N / 2, p.rc_scale + bh * (size_t)(P * N / 16), P * N / 16,
+                 &S.full[slot]);
+      } else {
+        bulk_g2s(dst, p.h0 + bh * (size_t)(P * N), P * N * 4, &S.full[slot]);
+      }
+      issued |= 1u << slot;
+      parity = (parity & ~(1u << slot)) | (sphase << slot);
+      if (++slot == lay.NS) {
+        slot = 0;
+        sphase ^= 1;
+      }
+    }
+  }
+  if (failed) {
+    if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+    *abort_flag = 1;
+    // do not leave the CTA with bulk copies still landing in its memory
+    for (int s = 0; s < lay.NS; ++s)
+      if (issued & (1u << s)) mbar_wait(&S.full[s], (parity >> s) & 1u);
+  }
+}
+
+constexpr int kDecodeThreads = kThreads + 64;  // 8 consumer warps, tile producer, stager
+
+template <int P, int N, typename TI, int QM, int WPH>
+__global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Params p,
+                                                                  const DecodeLayout lay) {
+  using T = Tile<P, N>;
+  constexpr int C4 = T::C4;
+  constexpr bool kReadCopy = (QM == 1 || QM == 2);
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int abort_word;
+  volatile int *abort_flag = &abort_word;
+  const DecodeSmemPtrs S(smem, lay);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, rs = lane >> 3, c8 = lane & 7;
-  const int b = blockIdx.x / p.G, g = blockIdx.x - b * p.G;
-  const int h_first = g * p.hpg;
-  const size_t bh0 = (size_t)b * p.H + h_first;
+  const int hc = lay.hc, nchunk = p.hpg / hc;
+  const int nitems = p.B * p.G * nchunk;
+  const int L = lay.L;
 
   if (tid == 0) {
-    const int n0 = p.len[bh0];
-    bool ok = n0 >= 0 && n0 < p.L;
-    for (int j = 1; j < p.hpg; ++j) ok = ok && p.len[bh0 + j] == n0;
-    if (!ok) report(p.status, RSSM_ERR_STATE);
-    s_k = ok ? n0 + 1 : -1;
+    for (int s = 0; s < 8; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], WPH);  // consumer warps reading each tile
+    }
+    for (int r = 0; r < 4; ++r) {
+      mbar_init(&S.rfull[r], 1);
+      mbar_init(&S.rempty[r], 8);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
   }
   __syncthreads();
-  const int k = s_k;
-  if (k < 0) return;
-  const bool flush = (k == p.L);
-
-  // ---- group records: B_0..B_{k-1} (the last one is this step's), C_k
-  const size_t bg = (size_t)b * p.G + g;
-  const TI *Bin = static_cast<const TI *>(p.Bm) + b * p.bs_B + (size_t)g * N;
-  const TI *Cin = static_cast<const TI *>(p.Cm) + b * p.bs_C + (size_t)g * N;
-  TI *Bb = static_cast<TI *>(p.Bbuf) + bg * p.cap * N;
-  TI *Cb = static_cast<TI *>(p.Cbuf) + bg * p.cap * N;
-  for (int idx = tid; idx < k * N; idx += kThreads) {
-    const int i = idx / N, n = idx - i * N;
-    s_B[i][n] = to_f32(i == k - 1 ? Bin[n] : Bb[(size_t)i * N + n]);
+  if (warp == 8) {
+    if (lane == 0) decode_tiles<P, N, QM>(p, lay, S, abort_flag, nitems, nchunk);
+    return;
   }
-  for (int n = tid; n < N; n += kThreads) {
-    const TI cv = Cin[n];
-    s_C[n] = to_f32(cv);
-    if (!flush) {  // append; a flush empties the buffer, so its record is not kept
-      Bb[(size_t)(k - 1) * N + n] = Bin[n];
-      Cb[(size_t)(k - 1) * N + n] = cv;
-    }
+  if (warp == 9) {
+    decode_stager<P, N, TI>(p, lay, S, abort_flag, nitems, nchunk, lane);
+    return;
   }
-  __syncthreads();
-  for (int i = warp; i < k; i += 8) {
-    float acc = 0.f;
-    for (int n = lane; n < N; n += 32) acc += s_B[i][n] * s_C[n];
-    acc = warp_sum(acc);
-    if (lane == 0) s_bc[i] = acc;
-  }
-  float4 c4[C4];
-#pragma unroll
-  for (int s = 0; s < C4; ++s) c4[s] = *reinterpret_cast<const float4 *>(&s_C[T::col(c8, s)]);
 
-  for (int j = 0; j < p.hpg; ++j) {
-    const int h = h_first + j;
-    const size_t bh = bh0 + j;
-    float *tile = p.h0 + bh * (size_t)(P * N);
+  // Consumers.  Control flow stays uniform across the 256 consumer threads:
+  // every branch depends only on values read from shared memory after the
+  // same barrier or on bar.red.or results, and a thread whose bounded wait
+  // ran out keeps going through every barrier (its data is garbage, the
+  // status word says so) until the next item boundary, where all consumers
+  // leave together.
+  //
+  // Heads are processed HPQ = 8 / WPH at a time (one ring slot each, the rest
+  // of the ring keeps loading ahead), WPH warps per head; a warp owns
+  // RW = P / WPH rows of the tile, RG = RW / 4 row groups (quarter-warp rs
+  // takes row 4g + rs, lane c8 columns 32s + 4c8).  A warp first pulls its
+  // rows into registers (then the slot is released), so the outputs and the
+  // fold run while the producer already refills the slot.
+  constexpr int HPQ = 8 / WPH, RW = P / WPH, RG = RW / 4;
+  constexpr int RGC = RG < 4 ? RG : 4;  // row groups held in registers at once
+  const int hq = warp / WPH, sub = warp - hq * WPH;
+  int it = 0;
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+    const int rb = it % lay.NR;
+    const uint32_t rphase = (it / lay.NR) & 1;
+    float *scr = S.scr + (it & 1) * lay.scratch_floats;
+    double *bc = reinterpret_cast<double *>(scr);  // B_i.C_k, fp64
+    float *wdt = scr + 2 * pad4(L);
+    float *coef = wdt + pad4(hc * L);
+    float *lam = coef + pad4(hc * L);
+    float *red = lam + pad4(hc);
+    float *Bf = red + 32;  // fp32 copy of the group's B records [k][N]
+    float *z = Bf + L * N;  // buffered-record and skip terms of y [hc][P]
+    int b, g, chunk, h_first;
+    item_coords(p, item, nchunk, hc, b, g, chunk, h_first);
+    const size_t bh0 = (size_t)b * p.H + h_first;
+    const Stage st(S.stage + rb * lay.stage_floats, N, hc, L);
+    const TI *rB = reinterpret_cast<const TI *>(S.recB) + (size_t)rb * L * N;
+    const TI *rX = reinterpret_cast<const TI *>(S.recX) + (size_t)rb * hc * L * P;
 
-    // ---- checkpoint (or read copy) into registers; the partial C dots
-    float4 hv[RPT][C4];
-    float part[RPT];
-    if constexpr (QM == 1 || QM == 2) {
-      float4 rv[RPT][C4];
-      load_read_view<P, N, QM>(p, bh, warp, rs, c8, rv);
-      if (flush) load_tile<P, N>(tile, warp, rs, c8, hv);
-#pragma unroll
-      for (int rho = 0; rho < RPT; ++rho) {
-        float a = 0.f;
-#pragma unroll
-        for (int s = 0; s < C4; ++s) a += dot4(rv[rho][s], c4[s]);
-        part[rho] = a;
-      }
-    } else {
-      load_tile<P, N>(tile, warp, rs, c8, hv);
-#pragma unroll
-      for (int rho = 0; rho < RPT; ++rho) {
-        float a = 0.f;
-#pragma unroll
-        for (int s = 0; s < C4; ++s) a += dot4(hv[rho][s], c4[s]);
-        part[rho] = a;
-      }
+    const bool got = mbar_wait(&S.rfull[rb], rphase);
+    if (!got) {
+      report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
     }
-
-    // ---- head records: x_0..x_{k-1}, dt_0..dt_{k-1}; append this step's
-    const TI *xin = static_cast<const TI *>(p.x) + b * p.bs_x + (size_t)h * P;
-    TI *xb = static_cast<TI *>(p.xbuf) + bh * p.cap * P;
-    for (int idx = tid; idx < k * P; idx += kThreads) {
-      const int i = idx / P, q = idx - i * P;
-      if (i == k - 1) {
-        const TI xv = xin[q];
-        s_x[i][q] = to_f32(xv);
-        if (!flush) xb[(size_t)i * P + q] = xv;
-      } else {
-        s_x[i][q] = to_f32(xb[(size_t)i * P + q]);
+    if (bar_or(1, kThreads, !got || *abort_flag)) break;  // uniform exit
+    const int n0 = st.hdr[0];
+    if (st.hdr[1]) {  // uniform: every consumer reads the same staged header
+      if (tid == 0) report(p.status, RSSM_ERR_STATE);
+      // skip the item, keeping the ring in step with the producer
+      for (int q0 = 0; q0 < hc; q0 += HPQ) {
+        const uint32_t pos = (uint32_t)it * hc + q0 + hq;
+        if (!mbar_wait(&S.full[pos % lay.NS], (pos / lay.NS) & 1)) {
+          report(p.status, RSSM_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[pos % lay.NS]);
       }
-    }
-    if (tid < k) {
-      float d;
-      if (tid == k - 1) {
-        d = ld_in<TI>(p.dt, b * p.bs_dt + h);
-        if (!flush) p.dtbuf[bh * p.cap + tid] = d;
-      } else {
-        d = p.dtbuf[bh * p.cap + tid];
-      }
-      s_dt[tid] = d;
-    }
-    __syncthreads();
-    if (warp == 0) {
-      decay_weights(s_dt, k, p.A[h], s_wdt, &s_lam, lane);
+      fence_proxy_async_smem();
       __syncwarp();
-      if (lane < k) s_coef[lane] = s_wdt[lane] * s_bc[lane];
+      if (lane == 0) mbar_arrive(&S.rempty[rb]);
+      continue;
     }
-    __syncthreads();
+    const int k = n0 + 1;
+    const bool flush = (k == L);
 
-    // ---- output: y = Lam (h C) + sum_i w_i (B_i.C) x_i + D x_k
-    const float lam = s_lam, Dh = p.D[h];
-    float *yout = p.y + b * p.bs_y + (size_t)h * P;
+    // ---- append this step's record to the global buffer (a flush empties
+    // the buffer, so its record is not kept); one CTA per group writes B, C
+    if (!flush) {
+      const size_t bg = (size_t)b * p.G + g;
+      if (chunk == 0) {
+        for (int n = tid; n < N; n += kThreads) {
+          static_cast<TI *>(p.Bbuf)[(bg * p.cap + k - 1) * N + n] = rB[(k - 1) * N + n];
+          static_cast<TI *>(p.Cbuf)[(bg * p.cap + k - 1) * N + n] = from_f32<TI>(st.C[n]);
+        }
+      }
+      for (int e = tid; e < hc * P; e += kThreads) {
+        const int j = e / P, q = e - j * P;
+        static_cast<TI *>(p.xbuf)[((bh0 + j) * p.cap + k - 1) * P + q] = rX[(j * L + k - 1) * P + q];
+      }
+      if (tid < hc) p.dtbuf[(bh0 + tid) * p.cap + k - 1] = st.dt[tid * L + k - 1];
+    }
+    // ---- fp32 B records (for the fold), B_i.C_k dots, decay weights
+    if (flush)
+      for (int e = tid; e < k * N; e += kThreads) Bf[e] = to_f32(rB[e]);
+    {
+      // 16 threads per record, fp64 (these dots of N rounded products would
+      // otherwise dominate the output error when the inputs are fp32); the
+      // loop bound is the same for every thread so that all 32 lanes of each
+      // warp reach the full-mask shuffles
+      constexpr int PER = N / 16;
+      for (int base = 0; base < k; base += kThreads / 16) {
+        const int i = base + (tid >> 4), c0 = (tid & 15) * PER;
+        double acc = 0.0;
+        if (i < k) {
 #pragma unroll
-    for (int rho = 0; rho < RPT; ++rho) {
-      const int r = T::row(warp, rs, rho);
-      float acc = lam * part[rho];
-      for (int i = c8; i < k; i += 8) acc = fmaf(s_coef[i], s_x[i][r], acc);
-      acc = sum8(acc);
-      if (c8 == 0) yout[r] = fmaf(Dh, s_x[k - 1][r], acc);
+          for (int e = 0; e < PER; ++e)
+            acc = fma((double)to_f32(rB[i * N + c0 + e]), (double)st.C[c0 + e], acc);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+        if (i < k && (tid & 15) == 0) bc[i] = acc;
+      }
     }
+    for (int j = warp; j < hc; j += 8)
+      decay_weights_scan(st.dt + j * L, k, st.A[j], wdt + j * L, lam + j, lane);
+    bar_sync(1, kThreads);
+    // everything of y but the checkpoint term, per row:
+    //   z[j][r] = sum_i w_i (B_i . C_k) x_i[r] + D x_k[r]
+    // (threads run along r, so the record reads are conflict-free)
+    for (int e = tid; e < hc * P; e += kThreads) {
+      const int j = e / P, r = e - j * P;
+      const TI *xr = rX + j * L * P + r;
+      float acc = 0.f;
+      for (int i = 0; i < k; ++i)
+        acc = fmaf((float)((double)wdt[j * L + i] * bc[i]), to_f32(xr[i * P]), acc);
+      z[e] = fmaf(st.D[j], to_f32(xr[(k - 1) * P]), acc);
+    }
+    bar_sync(1, kThreads);
 
-    // ---- flush: fold the window into the checkpoint and write it once
-    if (flush) {
-      fold_regs<P, N>(hv, lam, k, s_wdt, s_x, s_B, warp, rs, c8);
-      commit_checkpoint<P, N, QM>(p, bh, tile, hv, s_red, warp, lane, rs, c8);
+    float4 c4[C4];
+#pragma unroll
+    for (int s = 0; s < C4; ++s) c4[s] = *reinterpret_cast<const float4 *>(&st.C[T::col(c8, s)]);
+
+    // ---- heads: HPQ at a time, WPH warps each, row groups of 4 rows
+    for (int q0 = 0; q0 < hc; q0 += HPQ) {
+      const int j = q0 + hq, h = h_first + j;
+      const size_t bh = bh0 + j;
+      const uint32_t pos = (uint32_t)it * hc + j;  // producer's issue order
+      const int sl = pos % lay.NS;
+      if (!mbar_wait(&S.full[sl], (pos / lay.NS) & 1)) {
+        report(p.status, RSSM_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      const unsigned char *t = S.ring + sl * lay.tile_stride;
+      const float sg = QM == 2 ? p.rc_gscale[bh] : 1.0f;
+      const float lm = lam[j];
+      const float *wj = wdt + j * L, *zj = z + j * P;
+      const TI *xj = rX + j * L * P;
+      float *yout = p.y + b * p.bs_y + (size_t)h * P;
+      float *tile = p.h0 + bh * (size_t)(P * N);
+      float amax = 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < RG; c0 += RGC) {
+        float4 v[RGC][C4];
+#pragma unroll
+        for (int u = 0; u < RGC; ++u) view_row<P, N, QM>(t, sub * RW + 4 * (c0 + u) + rs, c8, sg, v[u]);
+        if (c0 + RGC == RG) {  // all of this warp's rows are in registers
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.empty[sl]);
+        }
+        int rows[RGC];
+#pragma unroll
+        for (int u = 0; u < RGC; ++u) rows[u] = sub * RW + 4 * (c0 + u) + rs;
+#pragma unroll
+        for (int u = 0; u < RGC; ++u) {
+          const float a = sum8(tree_dot<C4>(v[u], c4));
+          if (c8 == 0) yout[rows[u]] = fmaf(lm, a, zj[rows[u]]);
+        }
+        if (flush) {
+          if constexpr (kReadCopy) {
+#pragma unroll
+            for (int u = 0; u < RGC; ++u) load_row<N>(tile, rows[u], c8, v[u]);
+          }
+          fold_rows<P, N, TI, RGC>(v, lm, k, wj, xj, rows, Bf, c8);
+#pragma unroll
+          for (int u = 0; u < RGC; ++u) {
+            if constexpr (QM == 3) fp8_roundtrip_row<N>(v[u]);
+            store_row<N>(tile, rows[u], c8, v[u]);
+            if constexpr (QM == 1) fp8_codes_row<N>(p.rc + bh * (size_t)(P * N), rows[u], c8, v[u]);
+            if constexpr (QM == 2 || QM == 4) amax = fmaxf(amax, absmax_row<N>(v[u]));
+          }
+        }
+      }
+      if constexpr (QM == 2 || QM == 4) {
+        if (flush) {
+          // NVFP4 needs the whole tile's maximum: combine the WPH warps of
+          // this head, then requantise the rows just written (each thread
+          // rereads exactly the elements it stored)
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+          if (lane == 0) red[hq * 8 + sub] = amax;
+          bar_sync(2 + hq, WPH * 32);
+          float tmax = 0.f;
+          for (int w2 = 0; w2 < WPH; ++w2) tmax = fmaxf(tmax, red[hq * 8 + w2]);
+          const float sgn = nvfp4_tile_scale(tmax);
+          for (int g4 = 0; g4 < RG; ++g4) {
+            const int r = sub * RW + 4 * g4 + rs;
+            float4 v[C4];
+            load_row<N>(tile, r, c8, v);
+            nvfp4_row<P, N>(v, sgn, QM == 4, p.rc + bh * (size_t)(P * N / 2),
+                            p.rc_scale + bh * (size_t)(P * N / 16), r, c8);
+            if constexpr (QM == 4) store_row<N>(tile, r, c8, v);
+          }
+          if constexpr (QM == 2)
+            if (sub == 0 && lane == 0) p.rc_gscale[bh] = sgn;
+          bar_sync(2 + hq, WPH * 32);  // red[] of this head is reused next round
+        }
+      }
     }
-    __syncthreads();  // s_x, s_dt, s_wdt, s_coef, s_lam are reused by the next head
+    // the producer refills this record buffer next: order our reads of it
+    // (generic proxy) before its bulk copies (async proxy)
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.rempty[rb]);
+    if (tid < hc) p.len[bh0 + tid] = flush ? 0 : k;
   }
-  if (tid < p.hpg) p.len[bh0 + tid] = flush ? 0 : k;
 }
 
 // ====================================================== fold-only kernels
@@ -391,77 +1062,64 @@ template <int P, int N, typename TI, int QM, int MODE>
 __global__ void __launch_bounds__(kThreads, 2) m2_fold_kernel(const M2Params p) {
   using T = Tile<P, N>;
   constexpr int RPT = T::RPT, C4 = T::C4;
-  __shared__ __align__(16) float s_B[kMaxCap][N];
-  __shared__ __align__(16) float s_x[kMaxCap][P];
-  __shared__ float s_dt[kMaxCap], s_wdt[kMaxCap];
-  __shared__ float s_lam, s_red[8];
-  __shared__ int s_n, s_do;
-
+  extern __shared__ __align__(16) unsigned char smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, rs = lane >> 3, c8 = lane & 7;
-  const int b = blockIdx.x / p.G, g = blockIdx.x - b * p.G;
-  const int h_first = g * p.hpg;
+  const int hc = head_chunk(p.hpg), nchunk = p.hpg / hc;
+  const int bg_i = blockIdx.x / nchunk, chunk = blockIdx.x - bg_i * nchunk;
+  const int b = bg_i / p.G, g = bg_i - b * p.G;
+  const int h_first = g * p.hpg + chunk * hc;
   const size_t bh0 = (size_t)b * p.H + h_first;
+  const int LC = p.cap;  // records here may exceed the window after a verify round
+  DecodeSmem S(smem_raw, LC, hc, N);
+  TI *s_x = static_cast<TI *>(S.x);
 
-  if (tid == 0) {
-    const int n0 = p.len[bh0];
-    bool ok = true;
-    for (int j = 1; j < p.hpg; ++j) ok = ok && p.len[bh0 + j] == n0;
-    int n = n0, act = 0;
-    if (MODE == kFoldCommit) {
-      const int a = p.acc[b];
-      ok = ok && n0 >= 0 && n0 < p.L && a >= 0 && a <= p.draft_max && n0 + a <= p.cap;
-      n = n0 + a;
-      act = n >= p.L;
-    } else if (MODE == kFoldFlush) {
-      ok = ok && n0 >= 0 && n0 <= p.cap;
-      act = n0 >= p.L || (p.force && n0 > 0);
-    } else {
-      ok = ok && n0 >= 0 && n0 <= p.cap;
-      act = 1;
-    }
-    if (!ok) report(p.status, RSSM_ERR_STATE);
-    s_n = ok ? n : -1;
-    s_do = act;
+  const int n0 = p.len[bh0];
+  bool bad = false;
+  if (tid > 0 && tid < hc) bad = p.len[bh0 + tid] != n0;
+  int n = n0, act = 0;
+  if (MODE == kFoldCommit) {
+    const int a = p.acc[b];
+    if (tid == 0) bad = n0 < 0 || n0 >= p.L || a < 0 || a > p.draft_max || n0 + a > p.cap;
+    n = n0 + a;
+    act = n >= p.L;
+  } else {
+    if (tid == 0) bad = n0 < 0 || n0 > p.cap;
+    act = MODE == kFoldMaterialize ? 1 : (n0 >= p.L || (p.force && n0 > 0));
   }
-  __syncthreads();
-  const int n = s_n;
-  if (n < 0) return;
-  if (!s_do) {
-    if (MODE == kFoldCommit && tid < p.hpg) p.len[bh0 + tid] = n;
+  if (__syncthreads_or(bad)) {
+    if (tid == 0) report(p.status, RSSM_ERR_STATE);
     return;
   }
-
-  const size_t bg = (size_t)b * p.G + g;
-  const TI *Bb = static_cast<const TI *>(p.Bbuf) + bg * p.cap * N;
-  for (int idx = tid; idx < n * N; idx += kThreads) {
-    const int i = idx / N, c = idx - i * N;
-    s_B[i][c] = to_f32(Bb[(size_t)i * N + c]);
+  if (!act) {
+    if (MODE == kFoldCommit && tid < hc) p.len[bh0 + tid] = n;
+    return;
   }
-  for (int j = 0; j < p.hpg; ++j) {
-    const int h = h_first + j;
+  const size_t bg = (size_t)b * p.G + g;
+  stage_f32<TI>(S.B, static_cast<const TI *>(p.Bbuf) + bg * p.cap * N, n * N, tid);
+  for (int j = 0; j < hc; ++j)
+    stage_raw(s_x + j * LC * P, static_cast<const TI *>(p.xbuf) + (bh0 + j) * p.cap * P,
+              n * P * (int)sizeof(TI), tid);
+  for (int e = tid; e < hc * n; e += kThreads) {
+    const int j = e / n, i = e - j * n;
+    S.dt[j * LC + i] = p.dtbuf[(bh0 + j) * p.cap + i];
+  }
+  __syncthreads();
+  for (int j = warp; j < hc; j += 8)
+    decay_weights(S.dt + j * LC, n, p.A[h_first + j], S.wdt + j * LC, S.lam + j, lane);
+  __syncthreads();
+  for (int j = 0; j < hc; ++j) {
     const size_t bh = bh0 + j;
     float *tile = p.h0 + bh * (size_t)(P * N);
     float4 hv[RPT][C4];
     load_tile<P, N>(tile, warp, rs, c8, hv);
-    const TI *xb = static_cast<const TI *>(p.xbuf) + bh * p.cap * P;
-    for (int idx = tid; idx < n * P; idx += kThreads) {
-      const int i = idx / P, q = idx - i * P;
-      s_x[i][q] = to_f32(xb[(size_t)i * P + q]);
-    }
-    if (tid < n) s_dt[tid] = p.dtbuf[bh * p.cap + tid];
-    __syncthreads();
-    if (warp == 0) decay_weights(s_dt, n, p.A[h], s_wdt, &s_lam, lane);
-    __syncthreads();
-    const float lam = n > 0 ? s_lam : 1.0f;
-    fold_regs<P, N>(hv, lam, n, s_wdt, s_x, s_B, warp, rs, c8);
+    fold_regs<P, N, TI>(hv, S.lam[j], n, S.wdt + j * LC, s_x + j * LC * P, S.B, warp, rs, c8);
     if constexpr (MODE == kFoldMaterialize) {
       store_tile<P, N>(p.S_out + bh * (size_t)(P * N), warp, rs, c8, hv);
     } else {
-      commit_checkpoint<P, N, QM>(p, bh, tile, hv, s_red, warp, lane, rs, c8);
+      commit_checkpoint<P, N, QM>(p, bh, tile, hv, S.red + 8 * (j & 1), warp, lane, rs, c8);
     }
-    __syncthreads();
   }
-  if (MODE != kFoldMaterialize && tid < p.hpg) p.len[bh0 + tid] = 0;
+  if (MODE != kFoldMaterialize && tid < hc) p.len[bh0 + tid] = 0;
 }
 
 // ================================================ conventional full step
@@ -521,182 +1179,268 @@ __global__ void __launch_bounds__(kThreads, 2) m2_full_kernel(const M2Params p) 
 // 1. optional commit of the previous round (len += a; fold when >= L),
 // 2. drafts written to slots len..len+nd-1,
 // 3. draft d's output from h0 and records 0..len+d, output-only.
+// One CTA per (sequence, group); the host requires H/G <= 8.
+
+constexpr int kMD = 4;  // most drafts per round
+
+struct VerifySmem {
+  float *Bb, *Bd, *Cd, *dtb, *dtd, *wdt, *lamf, *coef, *lam, *red;
+  double *bc;
+  void *xb, *xd;
+  // Bb [cap][N] | Bd [4][N] | Cd [4][N] | bc [4][cap+4] | dtb [hc][cap] | dtd [hc][4]
+  // | wdt [hc][cap] | lamf [pad4(hc)] | coef [hc][4][cap+4] | lam [hc][4] | red [8]
+  // | xb [hc][cap][P] | xd [hc][4][P] (input dtype)
+  __host__ __device__ static size_t bytes(int cap, int hc, int P, int N, int es) {
+    const int R = cap + kMD;
+    const size_t f = (size_t)cap * N + 2 * kMD * N + 2 * pad4(kMD * R) + pad4(hc * cap) +
+                     hc * kMD + pad4(hc * cap) + pad4(hc) + pad4(hc * kMD * R) + hc * kMD + 8;
+    return f * 4 + (size_t)hc * (cap + kMD) * P * es;
+  }
+  __device__ VerifySmem(unsigned char *base, int cap, int hc, int N, int P, int es) {
+    const int R = cap + kMD;
+    float *f = reinterpret_cast<float *>(base);
+    Bb = f;
+    Bd = Bb + cap * N;
+    Cd = Bd + kMD * N;
+    bc = reinterpret_cast<double *>(Cd + kMD * N);
+    dtb = Cd + kMD * N + 2 * pad4(kMD * R);
+    dtd = dtb + pad4(hc * cap);
+    wdt = dtd + hc * kMD;
+    lamf = wdt + pad4(hc * cap);
+    coef = lamf + pad4(hc);
+    lam = coef + pad4(hc * kMD * R);
+    red = lam + hc * kMD;
+    xb = red + 8;
+    xd = static_cast<unsigned char *>(xb) + (size_t)hc * cap * P * es;
+  }
+};
 
 template <int P, int N, typename TI>
 __global__ void __launch_bounds__(kThreads, 2) m2_verify_kernel(const M2Params p) {
   using T = Tile<P, N>;
   constexpr int RPT = T::RPT, C4 = T::C4;
-  constexpr int MD = 4;  // most drafts per round
-  __shared__ __align__(16) float s_Bb[kMaxCap][N];  // buffered records (fold / output prefix)
-  __shared__ __align__(16) float s_Bd[MD][N];       // drafts
-  __shared__ __align__(16) float s_Cd[MD][N];
-  __shared__ __align__(16) float s_xb[kMaxCap][P];
-  __shared__ __align__(16) float s_xd[MD][P];
-  __shared__ float s_dtb[kMaxCap], s_dtd[MD];
-  __shared__ float s_bc[MD][kMaxCap + MD];
-  __shared__ float s_coef[MD][kMaxCap + MD];
-  __shared__ float s_wdt[kMaxCap];
-  __shared__ float s_lam[MD], s_lamf, s_red[8];
-  __shared__ int s_n1, s_fold;
-
+  extern __shared__ __align__(16) unsigned char smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, rs = lane >> 3, c8 = lane & 7;
   const int b = blockIdx.x / p.G, g = blockIdx.x - b * p.G;
-  const int h_first = g * p.hpg;
+  const int hc = p.hpg, cap = p.cap, R = cap + kMD;
+  const int h_first = g * hc;
   const size_t bh0 = (size_t)b * p.H + h_first;
   const int nd = p.n_draft;
+  VerifySmem S(smem_raw, cap, hc, N, P, (int)sizeof(TI));
+  TI *s_xb = static_cast<TI *>(S.xb);
+  TI *s_xd = static_cast<TI *>(S.xd);
 
-  if (tid == 0) {
-    const int n0 = p.len[bh0];
-    bool ok = n0 >= 0 && n0 < p.L;
-    for (int j = 1; j < p.hpg; ++j) ok = ok && p.len[bh0 + j] == n0;
-    const int a = p.acc ? p.acc[b] : 0;
-    ok = ok && a >= 0 && a <= p.draft_max && n0 + a <= p.cap;
-    const int n1 = n0 + a;
-    const int fold = n1 >= p.L;
-    const int nb = fold ? 0 : n1;
-    ok = ok && nb + nd <= p.cap;
-    if (!ok) report(p.status, RSSM_ERR_STATE);
-    s_n1 = ok ? n1 : -1;
-    s_fold = fold;
-  }
-  __syncthreads();
-  const int n1 = s_n1;
-  if (n1 < 0) return;
-  const bool fold = s_fold;
+  float4 cur[RPT][C4];
+  load_tile<P, N>(p.h0 + bh0 * (size_t)(P * N), warp, rs, c8, cur);
+
+  const int n0 = p.len[bh0];
+  const int a = p.acc ? p.acc[b] : 0;
+  const int n1 = n0 + a;
+  const bool fold = n1 >= p.L;
   const int nb = fold ? 0 : n1;  // committed records the drafts follow
-
-  const size_t bg = (size_t)b * p.G + g;
-  TI *Bb = static_cast<TI *>(p.Bbuf) + bg * p.cap * N;
-  TI *Cb = static_cast<TI *>(p.Cbuf) + bg * p.cap * N;
-  for (int idx = tid; idx < n1 * N; idx += kThreads) {
-    const int i = idx / N, c = idx - i * N;
-    s_Bb[i][c] = to_f32(Bb[(size_t)i * N + c]);
+  bool bad = tid == 0 && (n0 < 0 || n0 >= p.L || a < 0 || a > p.draft_max || n1 > cap ||
+                          nb + nd > cap);
+  if (tid > 0 && tid < hc) bad = p.len[bh0 + tid] != n0;
+  if (__syncthreads_or(bad)) {
+    if (tid == 0) report(p.status, RSSM_ERR_STATE);
+    return;
   }
-  __syncthreads();  // with a fold the drafts land on slots just read
-  for (int idx = tid; idx < nd * N; idx += kThreads) {
-    const int d = idx / N, c = idx - d * N;
-    const TI bv = static_cast<const TI *>(p.Bm)[b * p.bs_B + ((size_t)d * p.G + g) * N + c];
-    const TI cv = static_cast<const TI *>(p.Cm)[b * p.bs_C + ((size_t)d * p.G + g) * N + c];
-    s_Bd[d][c] = to_f32(bv);
-    s_Cd[d][c] = to_f32(cv);
-    Bb[(size_t)(nb + d) * N + c] = bv;
-    Cb[(size_t)(nb + d) * N + c] = cv;
+
+  // ---- stage buffered records 0..n1-1 and the drafts
+  const size_t bg = (size_t)b * p.G + g;
+  TI *Bb = static_cast<TI *>(p.Bbuf) + bg * cap * N;
+  TI *Cb = static_cast<TI *>(p.Cbuf) + bg * cap * N;
+  TI *xbuf = static_cast<TI *>(p.xbuf);
+  stage_f32<TI>(S.Bb, Bb, n1 * N, tid);
+  for (int j = 0; j < hc; ++j)
+    stage_raw(s_xb + j * cap * P, xbuf + (bh0 + j) * cap * P, n1 * P * (int)sizeof(TI), tid);
+  for (int e = tid; e < hc * n1; e += kThreads) {
+    const int j = e / n1, i = e - j * n1;
+    S.dtb[j * cap + i] = p.dtbuf[(bh0 + j) * cap + i];
+  }
+  const TI *Bin = static_cast<const TI *>(p.Bm) + b * p.bs_B;
+  const TI *Cin = static_cast<const TI *>(p.Cm) + b * p.bs_C;
+  for (int e = tid; e < nd * N; e += kThreads) {
+    const int d = e / N, c = e - d * N;
+    S.Bd[e] = to_f32(Bin[((size_t)d * p.G + g) * N + c]);
+    S.Cd[e] = to_f32(Cin[((size_t)d * p.G + g) * N + c]);
+  }
+  const TI *xin = static_cast<const TI *>(p.x) + b * p.bs_x;
+  for (int e = tid; e < hc * nd * P; e += kThreads) {
+    const int j = e / (nd * P), rem = e - j * (nd * P), d = rem / P, q = rem - d * P;
+    s_xd[(j * kMD + d) * P + q] = xin[((size_t)d * p.H + h_first + j) * P + q];
+  }
+  for (int e = tid; e < hc * nd; e += kThreads) {
+    const int j = e / nd, d = e - j * nd;
+    S.dtd[j * kMD + d] = ld_in<TI>(p.dt, b * p.bs_dt + (int64_t)d * p.H + h_first + j);
   }
   __syncthreads();
-  // bc[d][i] = B_i . C_d over the output record list (nb committed + drafts 0..d)
-  for (int pair = warp; pair < nd * (nb + nd); pair += 8) {
-    const int d = pair / (nb + nd), i = pair - d * (nb + nd);
+
+  // ---- drafts into their slots (after the reads above: with a fold they
+  // overwrite records just staged); B.C dots; decay weights and coefficients
+  for (int e = tid; e < nd * N; e += kThreads) {
+    const int d = e / N, c = e - d * N;
+    Bb[(size_t)(nb + d) * N + c] = Bin[((size_t)d * p.G + g) * N + c];
+    Cb[(size_t)(nb + d) * N + c] = Cin[((size_t)d * p.G + g) * N + c];
+  }
+  for (int e = tid; e < hc * nd * P; e += kThreads) {
+    const int j = e / (nd * P), rem = e - j * (nd * P), d = rem / P, q = rem - d * P;
+    xbuf[((bh0 + j) * cap + nb + d) * P + q] = s_xd[(j * kMD + d) * P + q];
+  }
+  for (int e = tid; e < hc * nd; e += kThreads) {
+    const int j = e / nd, d = e - j * nd;
+    p.dtbuf[(bh0 + j) * cap + nb + d] = S.dtd[j * kMD + d];
+  }
+  for (int pr = warp; pr < nd * (nb + nd); pr += 8) {
+    const int d = pr / (nb + nd), i = pr - d * (nb + nd);
     if (i <= nb + d) {
-      const float *Bi = i < nb ? s_Bb[i] : s_Bd[i - nb];
-      float acc = 0.f;
-      for (int c = lane; c < N; c += 32) acc += Bi[c] * s_Cd[d][c];
-      acc = warp_sum(acc);
-      if (lane == 0) s_bc[d][i] = acc;
+      const float *Bi = i < nb ? S.Bb + i * N : S.Bd + (i - nb) * N;
+      double acc = 0.0;
+      for (int c = lane; c < N; c += 32) acc = fma((double)Bi[c], (double)S.Cd[d * N + c], acc);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) S.bc[d * R + i] = acc;
     }
   }
-
-  for (int j = 0; j < p.hpg; ++j) {
-    const int h = h_first + j;
-    const size_t bh = bh0 + j;
-    float *tile = p.h0 + bh * (size_t)(P * N);
-    float4 hv[RPT][C4];
-    load_tile<P, N>(tile, warp, rs, c8, hv);
-    const TI *xb_src = static_cast<const TI *>(p.xbuf) + bh * p.cap * P;
-    TI *xb = static_cast<TI *>(p.xbuf) + bh * p.cap * P;
-    for (int idx = tid; idx < n1 * P; idx += kThreads) {
-      const int i = idx / P, q = idx - i * P;
-      s_xb[i][q] = to_f32(xb_src[(size_t)i * P + q]);
-    }
-    if (tid < n1) s_dtb[tid] = p.dtbuf[bh * p.cap + tid];
-    __syncthreads();  // buffered x read before the drafts overwrite their slots
-    for (int idx = tid; idx < nd * P; idx += kThreads) {
-      const int d = idx / P, q = idx - d * P;
-      const TI xv = static_cast<const TI *>(p.x)[b * p.bs_x + ((size_t)d * p.H + h) * P + q];
-      s_xd[d][q] = to_f32(xv);
-      xb[(size_t)(nb + d) * P + q] = xv;
-    }
-    if (tid < nd) {
-      const float dv = ld_in<TI>(p.dt, b * p.bs_dt + (int64_t)tid * p.H + h);
-      s_dtd[tid] = dv;
-      p.dtbuf[bh * p.cap + nb + tid] = dv;
-    }
-    __syncthreads();
-    const float A = p.A[h];
-    if (warp == 0) {
-      if (fold) decay_weights(s_dtb, n1, A, s_wdt, &s_lamf, lane);
-      // draft d: records (nb committed, then drafts 0..d); lane i owns record i
-      for (int d = 0; d < nd; ++d) {
-        const int kd = nb + d + 1;
-        if (lane < kd) {
-          float s = 0.f;
-          for (int m = lane + 1; m < kd; ++m) s += m < nb ? s_dtb[m] : s_dtd[m - nb];
-          const float dti = lane < nb ? s_dtb[lane] : s_dtd[lane - nb];
-          s_coef[d][lane] = expf(A * s) * dti * s_bc[d][lane];
-        }
-        if (lane == 0) {
-          float t = 0.f;
-          for (int m = 0; m < kd; ++m) t += m < nb ? s_dtb[m] : s_dtd[m - nb];
-          s_lam[d] = expf(A * t);
-        }
+  __syncthreads();
+  for (int j = warp; j < hc; j += 8) {
+    const float A = p.A[h_first + j];
+    const float *dtb = S.dtb + j * cap, *dtd = S.dtd + j * kMD;
+    if (fold) decay_weights(dtb, n1, A, S.wdt + j * cap, S.lamf + j, lane);
+    for (int d = 0; d < nd; ++d) {
+      const int kd = nb + d + 1;
+      if (lane < kd) {
+        double s = 0.0;
+        for (int m = lane + 1; m < kd; ++m) s += m < nb ? dtb[m] : dtd[m - nb];
+        const double dti = lane < nb ? dtb[lane] : dtd[lane - nb];
+        S.coef[(j * kMD + d) * R + lane] = (float)(exp((double)A * s) * dti * S.bc[d * R + lane]);
+      }
+      if (lane == 0) {
+        double t = 0.0;
+        for (int m = 0; m < kd; ++m) t += m < nb ? dtb[m] : dtd[m - nb];
+        S.lam[j * kMD + d] = (float)exp((double)A * t);
       }
     }
-    __syncthreads();
+  }
+  __syncthreads();
+
+  // ---- head loop: optional fold, then the draft outputs from one tile read
+  for (int j = 0; j < hc; ++j) {
+    const int h = h_first + j;
+    const size_t bh = bh0 + j;
+    float4 nxt[RPT][C4];
+    if (j + 1 < hc) load_tile<P, N>(p.h0 + (bh + 1) * (size_t)(P * N), warp, rs, c8, nxt);
     if (fold) {
-      fold_regs<P, N>(hv, s_lamf, n1, s_wdt, s_xb, s_Bb, warp, rs, c8);
-      commit_checkpoint<P, N, 0>(p, bh, tile, hv, s_red, warp, lane, rs, c8);
+      fold_regs<P, N, TI>(cur, S.lamf[j], n1, S.wdt + j * cap, s_xb + j * cap * P, S.Bb, warp,
+                          rs, c8);
+      store_tile<P, N>(p.h0 + bh * (size_t)(P * N), warp, rs, c8, cur);
     }
     const float Dh = p.D[h];
+    const TI *xbj = s_xb + j * cap * P, *xdj = s_xd + j * kMD * P;
 #pragma unroll
     for (int rho = 0; rho < RPT; ++rho) {
       const int r = T::row(warp, rs, rho);
       for (int d = 0; d < nd; ++d) {
-        float a = 0.f;
+        float acc = 0.f;
 #pragma unroll
         for (int s = 0; s < C4; ++s)
-          a += dot4(hv[rho][s], *reinterpret_cast<const float4 *>(&s_Cd[d][T::col(c8, s)]));
-        a *= s_lam[d];
+          acc += dot4(cur[rho][s], *reinterpret_cast<const float4 *>(&S.Cd[d * N + T::col(c8, s)]));
+        acc *= S.lam[j * kMD + d];
+        const float *cf = S.coef + (j * kMD + d) * R;
         for (int i = c8; i <= nb + d; i += 8) {
-          const float xi = i < nb ? s_xb[i][r] : s_xd[i - nb][r];
-          a = fmaf(s_coef[d][i], xi, a);
+          const float xi = i < nb ? to_f32(xbj[i * P + r]) : to_f32(xdj[(i - nb) * P + r]);
+          acc = fmaf(cf[i], xi, acc);
         }
-        a = sum8(a);
+        acc = sum8(acc);
         if (c8 == 0)
-          p.y[b * p.bs_y + ((size_t)d * p.H + h) * P + r] = fmaf(Dh, s_xd[d][r], a);
+          p.y[b * p.bs_y + ((size_t)d * p.H + h) * P + r] = fmaf(Dh, to_f32(xdj[d * P + r]), acc);
       }
     }
-    __syncthreads();
+    if (j + 1 < hc) {
+#pragma unroll
+      for (int rho = 0; rho < RPT; ++rho)
+#pragma unroll
+        for (int s = 0; s < C4; ++s) cur[rho][s] = nxt[rho][s];
+    }
   }
-  if (tid < p.hpg) p.len[bh0 + tid] = nb;
+  if (tid < hc) p.len[bh0 + tid] = nb;
 }
 
 // ================================================================= launchers
 
-template <int P, int N, typename TI>
-cudaError_t decode_qm(const M2Params &p, cudaStream_t s) {
-  const dim3 grid((unsigned)(p.B * p.G)), block(kThreads);
+template <typename K>
+cudaError_t launch_dyn(K kernel, unsigned grid, size_t smem, cudaStream_t s, const M2Params &p) {
+  if (smem > 48 * 1024) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  kernel<<<grid, kThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n > 0 ? n : 148;
+}
+
+// Heads per decode work item: the whole group up to 8 heads, else chunks of 8
+// (per-item setup is amortised over as many heads as the ring allows).
+__host__ __forceinline__ int decode_chunk(int hpg) {
+  // a power of two (1, 2, 4 or 8) dividing the group: the consumer warps split
+  // evenly over the heads in flight
+  for (int c = 8; c > 1; c >>= 1)
+    if (hpg % c == 0) return c;
+  return 1;
+}
+
+template <typename K>
+cudaError_t launch_decode(K kernel, const M2Params &p, const DecodeLayout &lay, cudaStream_t s) {
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+  if (e != cudaSuccess) return e;
+  const int nitems = p.B * p.G * (p.hpg / lay.hc);
+  const int grid = nitems < sm_count() ? nitems : sm_count();
+  kernel<<<grid, kDecodeThreads, lay.total, s>>>(p, lay);
+  return cudaGetLastError();
+}
+
+template <int P, int N, typename TI, int WPH>
+cudaError_t decode_wph(const M2Params &p, const DecodeLayout &lay, cudaStream_t s) {
   switch (p.qmode) {
-    case 0: m2_decode_kernel<P, N, TI, 0><<<grid, block, 0, s>>>(p); break;
-    case 1: m2_decode_kernel<P, N, TI, 1><<<grid, block, 0, s>>>(p); break;
-    case 2: m2_decode_kernel<P, N, TI, 2><<<grid, block, 0, s>>>(p); break;
-    case 3: m2_decode_kernel<P, N, TI, 3><<<grid, block, 0, s>>>(p); break;
-    case 4: m2_decode_kernel<P, N, TI, 4><<<grid, block, 0, s>>>(p); break;
+    case 0: return launch_decode(m2_decode_kernel<P, N, TI, 0, WPH>, p, lay, s);
+    case 1: return launch_decode(m2_decode_kernel<P, N, TI, 1, WPH>, p, lay, s);
+    case 2: return launch_decode(m2_decode_kernel<P, N, TI, 2, WPH>, p, lay, s);
+    case 3: return launch_decode(m2_decode_kernel<P, N, TI, 3, WPH>, p, lay, s);
+    case 4: return launch_decode(m2_decode_kernel<P, N, TI, 4, WPH>, p, lay, s);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+}
+
+template <int P, int N, typename TI>
+cudaError_t decode_qm(const M2Params &p, cudaStream_t s) {
+  const int hc = decode_chunk(p.hpg);
+  const DecodeLayout lay = DecodeLayout::make(P, N, hc, p.L, (int)sizeof(TI), p.qmode, 220 * 1024);
+  if (lay.NS < 2) return cudaErrorInvalidConfiguration;
+  // two heads in flight (4 warps each) when the item has at least two heads
+  return hc >= 2 ? decode_wph<P, N, TI, 4>(p, lay, s) : decode_wph<P, N, TI, 8>(p, lay, s);
 }
 
 template <int P, int N, typename TI, int MODE>
 cudaError_t fold_qm(const M2Params &p, cudaStream_t s) {
-  const dim3 grid((unsigned)(p.B * p.G)), block(kThreads);
+  const int hc = head_chunk(p.hpg);
+  const unsigned grid = (unsigned)(p.B * p.G * (p.hpg / hc));
+  const size_t smem = DecodeSmem::bytes(p.cap, hc, P, N, sizeof(TI));
   switch (MODE == kFoldMaterialize ? 0 : p.qmode) {
-    case 0: m2_fold_kernel<P, N, TI, 0, MODE><<<grid, block, 0, s>>>(p); break;
-    case 1: m2_fold_kernel<P, N, TI, 1, MODE><<<grid, block, 0, s>>>(p); break;
-    case 2: m2_fold_kernel<P, N, TI, 2, MODE><<<grid, block, 0, s>>>(p); break;
-    case 3: m2_fold_kernel<P, N, TI, 3, MODE><<<grid, block, 0, s>>>(p); break;
-    case 4: m2_fold_kernel<P, N, TI, 4, MODE><<<grid, block, 0, s>>>(p); break;
+    case 0: return launch_dyn(m2_fold_kernel<P, N, TI, 0, MODE>, grid, smem, s, p);
+    case 1: return launch_dyn(m2_fold_kernel<P, N, TI, 1, MODE>, grid, smem, s, p);
+    case 2: return launch_dyn(m2_fold_kernel<P, N, TI, 2, MODE>, grid, smem, s, p);
+    case 3: return launch_dyn(m2_fold_kernel<P, N, TI, 3, MODE>, grid, smem, s, p);
+    case 4: return launch_dyn(m2_fold_kernel<P, N, TI, 4, MODE>, grid, smem, s, p);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 template <int P, int N, typename TI>
@@ -711,10 +1455,10 @@ cudaError_t fold_mode(const M2Params &p, int mode, cudaStream_t s) {
 
 template <typename F>
 cudaError_t dispatch_shape(int P, int N, int bf16, F &&f) {
-#define RSSM_M2_CASE(PP, NN)                                   \
-  if (P == PP && N == NN)                                      \
-    return bf16 ? f(std::integral_constant<int, PP>{}, std::integral_constant<int, NN>{}, \
-                    __nv_bfloat16{})                           \
+#define RSSM_M2_CASE(PP, NN)                                                                    \
+  if (P == PP && N == NN)                                                                       \
+    return bf16 ? f(std::integral_constant<int, PP>{}, std::integral_constant<int, NN>{},       \
+                    __nv_bfloat16{})                                                            \
                 : f(std::integral_constant<int, PP>{}, std::integral_constant<int, NN>{}, 0.0f);
   RSSM_M2_CASE(64, 64)
   RSSM_M2_CASE(64, 128)
@@ -727,6 +1471,12 @@ cudaError_t dispatch_shape(int P, int N, int bf16, F &&f) {
 }  // namespace
 
 bool m2_supported(int P, int N) { return (P == 64 || P == 128) && (N == 64 || N == 128); }
+
+bool m2_heads_supported(int hpg) { return hpg <= 8 || hpg % 8 == 0; }
+
+size_t m2_verify_smem(int cap, int hpg, int P, int N, int es) {
+  return VerifySmem::bytes(cap, hpg, P, N, es);
+}
 
 cudaError_t m2_launch_decode(const M2Params &p, cudaStream_t s) {
   if (p.B * p.G == 0) return cudaSuccess;
@@ -754,9 +1504,11 @@ cudaError_t m2_launch_full(const M2Params &p, cudaStream_t s) {
 cudaError_t m2_launch_verify(const M2Params &p, cudaStream_t s) {
   if (p.B * p.G == 0) return cudaSuccess;
   return dispatch_shape(p.P, p.N, p.in_bf16, [&](auto PP, auto NN, auto ti) {
-    m2_verify_kernel<decltype(PP)::value, decltype(NN)::value, decltype(ti)>
-        <<<(unsigned)(p.B * p.G), kThreads, 0, s>>>(p);
-    return cudaGetLastError();
+    using TI = decltype(ti);
+    const size_t smem = VerifySmem::bytes(p.cap, p.hpg, decltype(PP)::value, decltype(NN)::value,
+                                          sizeof(TI));
+    return launch_dyn(m2_verify_kernel<decltype(PP)::value, decltype(NN)::value, TI>,
+                      (unsigned)(p.B * p.G), smem, s, p);
   });
 }
 

@@ -55,6 +55,7 @@ ENTRY_POINTS = {
     "replayssm_capacity": (C.c_int32, [C.POINTER(Desc)]),
     "replayssm_state_bytes": (C.c_size_t, [C.POINTER(Desc), C.c_int32]),
     "replayssm_status_string": (C.c_char_p, [C.c_int]),
+    "replayssm_last_cuda_error": (C.c_char_p, []),
     "replayssm_init": (C.c_int, [C.POINTER(Desc), C.POINTER(State), C.c_void_p, C.c_void_p]),
     "replayssm_decode_step": (C.c_int, [C.POINTER(Desc), C.POINTER(State), C.POINTER(StepIn),
                                         C.c_void_p, C.c_void_p]),
@@ -97,7 +98,10 @@ class ReplayError(RuntimeError):
 
 def _ok(rc: int, what: str):
     if rc != RSSM_OK:
-        raise ReplayError(f"{what}: {STATUS_NAMES.get(rc, rc)} (status {rc})")
+        extra = ""
+        if rc == 6:
+            extra = f": {lib().replayssm_last_cuda_error().decode()}"
+        raise ReplayError(f"{what}: {STATUS_NAMES.get(rc, rc)} (status {rc}){extra}")
 
 
 # ------------------------------------------------------------------- layer spec

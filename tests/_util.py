@@ -33,6 +33,36 @@ def per_step_rel_err(got, ref):
     return max(rel_err(g, r) for g, r in zip(got, ref))
 
 
+class Worst(float):
+    """A float (the error) that also describes where the worst element is."""
+
+    def __new__(cls, value, where):
+        obj = super().__new__(cls, value)
+        obj.where = where
+        return obj
+
+    def __repr__(self):
+        return f"{float(self):.3e} ({self.where})"
+
+
+def worst_step_err(got, ref):
+    """per_step_rel_err plus the step, index and values of the worst element."""
+    best = Worst(0.0, "")
+    for t, (g, r) in enumerate(zip(got, ref)):
+        g = np.asarray(g, np.float64)
+        r = np.asarray(r, np.float64)
+        rms = np.sqrt(np.mean(r * r)) if r.size else 0.0
+        den = np.maximum(np.abs(r), 1e-2 * rms)
+        den = np.where(den == 0, 1.0, den)
+        e = np.abs(g - r) / den
+        i = int(np.argmax(e))
+        if e.flat[i] > best:
+            idx = np.unravel_index(i, r.shape)
+            best = Worst(float(e.flat[i]), f"step {t} index {tuple(int(v) for v in idx)} got "
+                         f"{g.flat[i]:.9g} ref {r.flat[i]:.9g} rms {rms:.4g}")
+    return best
+
+
 def read_kv(name):
     out = {}
     with open(os.path.join(GOLDEN, name)) as f:

@@ -543,7 +543,7 @@ struct DecodeLayout {
     d.tile_bytes = qm == 1 ? P * N : qm == 2 ? P * N / 2 + P * N / 16 : P * N * 4;
     d.tile_stride = align128(d.tile_bytes);
     d.stage_floats = N + pad4(hc * L) + 2 * pad4(hc) + 4;
-    d.scratch_floats = 2 * pad4(L) + 2 * pad4(hc * L) + pad4(hc) + 32 + L * N + hc * P;
+    d.scratch_floats = 2 * pad4(L) + pad4(hc * L) + pad4(hc) + 32 + L * N + hc * P;
     const int rec_b = L * N * es, rec_x = hc * L * P * es;
     // Prefer three record buffers (the stager then runs two items ahead, which
     // hides its two dependent memory round trips) as long as the ring keeps
@@ -869,8 +869,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
     float *scr = S.scr + (it & 1) * lay.scratch_floats;
     double *bc = reinterpret_cast<double *>(scr);  // B_i.C_k, fp64
     float *wdt = scr + 2 * pad4(L);
-    float *coef = wdt + pad4(hc * L);
-    float *lam = coef + pad4(hc * L);
+    float *lam = wdt + pad4(hc * L);
     float *red = lam + pad4(hc);
     float *Bf = red + 32;  // fp32 copy of the group's B records [k][N]
     float *z = Bf + L * N;  // buffered-record and skip terms of y [hc][P]

@@ -110,6 +110,11 @@ typedef struct {
  *            buf[2] v  [B][H][cap][DV] in_dtype
  *            buf[3] alpha [B][H][cap]  fp32
  *            buf[4] beta  [B][H][cap]  fp32
+ *            buf[5] u  [B][H][cap][DV] fp32: per record i, the delta-rule
+ *                   correction u_i = beta_i (v_i - (state before i)^T k_i)
+ *                   expressed from h0 and records 0..i (see replayssm_decode_step);
+ *                   it depends only on h0 and those records, so it is computed
+ *                   once, when record i is appended, and read by later steps
  * len [B][H] int32: records buffered per (sequence, head).  Slots >= len are
  * free (they may hold rejected drafts).  rc/rc_scale/rc_gscale are the read
  * copy (read_fmt != NONE): FP8 codes [B][H][P][N]; NVFP4 codes
@@ -117,7 +122,7 @@ typedef struct {
  * [B][H][P][N/16], fp32 tile scales [B][H].  status: one int32. */
 typedef struct {
   float *h0;
-  void *buf[5];
+  void *buf[6];
   int32_t *len;
   uint8_t *rc;
   uint8_t *rc_scale;
@@ -142,14 +147,14 @@ typedef struct {
 /* Which buffer replayssm_state_bytes sizes. */
 typedef enum {
   RSSM_BYTES_H0 = 0,
-  RSSM_BYTES_BUF0 = 1, /* .. RSSM_BYTES_BUF0 + 4 for buf[0..4] */
-  RSSM_BYTES_LEN = 6,
-  RSSM_BYTES_RC = 7,
-  RSSM_BYTES_RC_SCALE = 8,
-  RSSM_BYTES_RC_GSCALE = 9,
-  RSSM_BYTES_STATUS = 10,
-  RSSM_BYTES_FULL_STATE = 11, /* conventional state, same layout as h0 */
-  RSSM_BYTES_Y = 12           /* one step's output */
+  RSSM_BYTES_BUF0 = 1, /* .. RSSM_BYTES_BUF0 + 5 for buf[0..5] */
+  RSSM_BYTES_LEN = 7,
+  RSSM_BYTES_RC = 8,
+  RSSM_BYTES_RC_SCALE = 9,
+  RSSM_BYTES_RC_GSCALE = 10,
+  RSSM_BYTES_STATUS = 11,
+  RSSM_BYTES_FULL_STATE = 12, /* conventional state, same layout as h0 */
+  RSSM_BYTES_Y = 13           /* one step's output */
 } rssm_bytes_which;
 
 /* Host-only helpers (no CUDA calls). */
@@ -173,7 +178,11 @@ rssm_status replayssm_init(const rssm_desc *desc, rssm_state *state, const float
  * append the step's record at slot len; y from h0 (or its read copy) and the
  * len+1 buffered records; if len+1 == window, fold the records into h0, write
  * h0 (and the read copy) once and set len = 0, else len += 1.  Requires
- * 0 <= len < window on entry (else RSSM_ERR_STATE in the status word). */
+ * 0 <= len < window on entry (else RSSM_ERR_STATE in the status word).
+ * GDN: with gamma/R the products of the record alphas, the step evaluates
+ * z = h0^T k and h0^T q once, u = beta (v - gamma z - sum_j R_j (k_j.k) u_j)
+ * from the earlier records' cached u_j, and o = scale (gamma h0^T q +
+ * sum_i R_i (k_i.q) u_i); u is appended with the record. */
 rssm_status replayssm_decode_step(const rssm_desc *desc, rssm_state *state,
                                   const rssm_step_in *in, float *y, void *stream);
 

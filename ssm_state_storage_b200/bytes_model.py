@@ -52,11 +52,15 @@ def gdn_conventional_bytes(DK, DV, in_bytes):
 
 
 def gdn_replay_bytes(k, L, DK, DV, in_bytes):
+    """Gated DeltaNet replay step as the kernel runs it: every past record
+    contributes its key, its cached u (fp32) and its alpha; this step reads
+    q, k, v, alpha, beta, appends them with its u (not on the flush step),
+    writes the output, and on the flush step writes the checkpoint."""
     state = DK * DV * 4
-    rec_read = (DK + DV) * in_bytes + 8   # k, v, alpha, beta of a past record
-    cur = (2 * DK + DV) * in_bytes + 8    # q, k, v, alpha, beta of this step
+    rec_read = DK * in_bytes + DV * 4 + 4
+    cur = (2 * DK + DV) * in_bytes + 8
     flush = k == L
-    append = 0 if flush else cur
+    append = 0 if flush else cur + DV * 4
     return state + (k - 1) * rec_read + cur + append + DV * 4 + (state if flush else 0)
 
 

@@ -47,7 +47,7 @@ rssm_status check_desc(const rssm_desc *d) {
 
 rssm_status check_state(const rssm_desc *d, const rssm_state *s) {
   if (!s || !s->h0 || !s->len || !s->status) return RSSM_ERR_INVALID_ARG;
-  const int nbuf = d->kind == RSSM_MAMBA2 ? 4 : 5;
+  const int nbuf = d->kind == RSSM_MAMBA2 ? 4 : 6;
   for (int i = 0; i < nbuf; ++i)
     if (!s->buf[i]) return RSSM_ERR_INVALID_ARG;
   if (!aligned16(s->h0)) return RSSM_ERR_ALIGNMENT;
@@ -143,6 +143,7 @@ GDNParams gdn_params(const rssm_desc *d, const rssm_state *s) {
     p.vbuf = s->buf[2];
     p.abuf = static_cast<float *>(s->buf[3]);
     p.bbuf = static_cast<float *>(s->buf[4]);
+    p.ubuf = static_cast<float *>(s->buf[5]);
     p.len = s->len;
     p.status = s->status;
   }
@@ -192,6 +193,7 @@ size_t replayssm_state_bytes(const rssm_desc *d, int32_t which) {
     case RSSM_BYTES_BUF0 + 2: return m2 ? B * G * cap * N * es : B * H * cap * P * es;
     case RSSM_BYTES_BUF0 + 3: return m2 ? B * G * cap * N * es : B * H * cap * 4;
     case RSSM_BYTES_BUF0 + 4: return m2 ? 0 : B * H * cap * 4;
+    case RSSM_BYTES_BUF0 + 5: return m2 ? 0 : B * H * cap * P * 4;
     case RSSM_BYTES_LEN: return B * H * 4;
     case RSSM_BYTES_RC:
       return d->read_fmt == RSSM_FMT_FP8 ? B * H * P * N

@@ -29,6 +29,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "pipeline.cuh"
 
 namespace rssm {
 namespace {
@@ -277,11 +278,439 @@ cudaError_t launch_dt(const GDNParams &p, cudaStream_t s) {
 
 }  // namespace
 
+// ============================================================ decode step
+// Persistent, warp-specialised replay decode step (one CTA of 320 threads
+// per SM).  Work item = one (sequence, head).  Warp 8 streams the item's
+// checkpoint as two 32 KiB half-tiles (rows 0-63, 64-127) with bulk copies
+// into a ring of shared-memory slots; warp 9 stages the item's small inputs
+// and bulk-copies its buffered k and u records, up to NR items ahead; warps
+// 0-3 consume half-tile 0 and warps 4-7 half-tile 1 (16 rows x 4 columns per
+// thread, held in registers so the slot is freed at once).
+//
+// With R_i = prod_{i<m<k} alpha_m, gamma = prod_{m<k} alpha_m (records
+// 0..k-1, record k-1 = this step's) and the cached u_0..u_{k-2}:
+//   z  = h0^T k_{k-1},   zq = h0^T q
+//   u_{k-1} = beta_{k-1} (v_{k-1} - gamma z - sum_{j<k-1} R_j (k_j.k_{k-1}) u_j)
+//   o  = scale (gamma zq + sum_{i<k} R_i (k_i.q) u_i)
+//   flush (k = window): h0 <- gamma h0 + sum_{i<k} R_i k_i u_i^T.
+
+namespace {
+
+constexpr int kHalfRows = DKc / 2;                       // rows per half-tile
+constexpr int kHalfBytes = kHalfRows * DVc * 4;          // 32 KiB
+
+struct GdnLayout {
+  int NS, NR, L;
+  int off_bars, off_recK, off_recU, off_stage, off_db, off_single, off_ring, total;
+  int stage_floats, db_floats;
+  __host__ static int a128(int v) { return (v + 127) & ~127; }
+  __host__ static GdnLayout make(int L, int es, int budget) {
+    GdnLayout d;
+    d.L = L;
+    // stage: q, kc, v [128] fp32 | alpha [L] | beta | hdr(2 ints)
+    d.stage_floats = 3 * 128 + ((L + 3) & ~3) + 4;
+    // per item, double-buffered: R [L] | kk [L] | kq [L] | gamma,pad [4] | Kf [L][128]
+    d.db_floats = 3 * ((L + 3) & ~3) + 4 + L * 128;
+    for (d.NR = 3; d.NR >= 1; --d.NR) {
+      int o = 0;
+      d.off_bars = o;
+      o += a128(8 * (2 * 8 + 2 * 4));
+      d.off_recK = o;
+      o += a128(d.NR * L * DKc * es);
+      d.off_recU = o;
+      o += a128(d.NR * L * DVc * 4);
+      d.off_stage = o;
+      o += a128(d.NR * d.stage_floats * 4);
+      d.off_db = o;
+      o += a128(2 * d.db_floats * 4);
+      d.off_single = o;  // part [8][2][128] | z [2][128] | ucur [128]
+      o += a128((8 * 2 * 128 + 2 * 128 + 128) * 4);
+      d.off_ring = o;
+      d.NS = (budget - o) / kHalfBytes;
+      if (d.NS > 8) d.NS = 8;
+      if (d.NS >= 4) {
+        d.total = o + d.NS * kHalfBytes;
+        return d;
+      }
+    }
+    d.NS = 0;
+    return d;
+  }
+};
+
+struct GdnPtrs {
+  uint64_t *full, *empty, *rfull, *rempty;
+  unsigned char *recK, *ring;
+  float *recU, *stage, *db, *part, *z, *ucur;
+  __device__ GdnPtrs(unsigned char *smem, const GdnLayout &l) {
+    full = reinterpret_cast<uint64_t *>(smem + l.off_bars);
+    empty = full + 8;
+    rfull = empty + 8;
+    rempty = rfull + 4;
+    recK = smem + l.off_recK;
+    recU = reinterpret_cast<float *>(smem + l.off_recU);
+    stage = reinterpret_cast<float *>(smem + l.off_stage);
+    db = reinterpret_cast<float *>(smem + l.off_db);
+    part = reinterpret_cast<float *>(smem + l.off_single);
+    z = part + 8 * 2 * 128;
+    ucur = z + 2 * 128;
+    ring = smem + l.off_ring;
+  }
+};
+
+// Stager warp: all loads of item `it` first (none depends on the length:
+// every alpha slot of the window is read), then shared-memory writes, then
+// (lane 0) the bulk copies of the buffered k and u records.
+template <typename TI>
+__device__ __forceinline__ bool gdn_stage(const GDNParams &p, const GdnLayout &lay,
+                                          const GdnPtrs &S, int item, int it, int lane) {
+  const int L = lay.L;
+  const int rb = it % lay.NR;
+  const uint32_t rphase = (it / lay.NR) & 1;
+  bool ok = true;
+  if (lane == 0) ok = mbar_wait(&S.rempty[rb], rphase ^ 1);
+  if (!__shfl_sync(0xffffffffu, (int)ok, 0)) return false;
+  const int b = item / p.H, h = item - (item / p.H) * p.H;
+  const size_t bh = (size_t)item;
+  const TI *qin = static_cast<const TI *>(p.q) + b * p.bs_q + (size_t)h * DKc;
+  const TI *kin = static_cast<const TI *>(p.k) + b * p.bs_k + (size_t)h * DKc;
+  const TI *vin = static_cast<const TI *>(p.v) + b * p.bs_v + (size_t)h * DVc;
+  const int n0 = __ldcg(&p.len[bh]);
+  const float a_cur = p.alpha[b * p.bs_a + h], b_cur = p.beta[b * p.bs_b + h];
+  const float a_rec = lane < L ? __ldcg(&p.abuf[bh * p.cap + lane]) : 0.f;
+  TI qv[4], kv[4], vv[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    qv[u] = qin[lane + 32 * u];
+    kv[u] = kin[lane + 32 * u];
+    vv[u] = vin[lane + 32 * u];
+  }
+  const bool bad = n0 < 0 || n0 >= L;
+  const int k = min(max(n0 + 1, 1), L);  // copies stay in bounds even for a bad length
+  float *st = S.stage + rb * lay.stage_floats;
+  TI *rK = reinterpret_cast<TI *>(S.recK) + (size_t)rb * L * DKc;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int c = lane + 32 * u;
+    st[c] = to_f32(qv[u]);
+    st[128 + c] = to_f32(kv[u]);
+    st[256 + c] = to_f32(vv[u]);
+    rK[(k - 1) * DKc + c] = kv[u];
+  }
+  float *alpha = st + 384;
+  if (lane < k) alpha[lane] = lane == k - 1 ? a_cur : a_rec;
+  float *tail = alpha + ((L + 3) & ~3);
+  if (lane == 0) {
+    tail[0] = b_cur;
+    reinterpret_cast<int *>(tail)[1] = n0;
+    reinterpret_cast<int *>(tail)[2] = bad;
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    const uint32_t bytesK = (k - 1) * DKc * sizeof(TI), bytesU = (k - 1) * DVc * 4;
+    mbar_arrive_expect_tx(&S.rfull[rb], bytesK + bytesU);
+    if (k > 1) {
+      bulk_g2s(rK, static_cast<const TI *>(p.kbuf) + bh * p.cap * DKc, bytesK, &S.rfull[rb]);
+      bulk_g2s(S.recU + (size_t)rb * L * DVc, p.ubuf + bh * p.cap * DVc, bytesU, &S.rfull[rb]);
+    }
+  }
+  return true;
+}
+
+template <typename TI>
+__global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNParams p,
+                                                                   const GdnLayout lay) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int abort_word;
+  volatile int *abort_flag = &abort_word;
+  const GdnPtrs S(smem, lay);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nitems = p.B * p.H;
+  const int L = lay.L;
+
+  if (tid == 0) {
+    for (int s = 0; s < 8; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 4);  // the 4 consumer warps of a half-tile
+    }
+    for (int r = 0; r < 4; ++r) {
+      mbar_init(&S.rfull[r], 1);
+      mbar_init(&S.rempty[r], 8);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == 8) {  // tile producer: half-tiles in (item, half) order
+    if (lane != 0) return;
+    int slot = 0;
+    uint32_t sphase = 0, issued = 0, parity = 0;
+    bool failed = false;
+    for (int item = blockIdx.x; item < nitems && !failed; item += gridDim.x) {
+      for (int half = 0; half < 2; ++half) {
+        if (*abort_flag || !mbar_wait(&S.empty[slot], sphase ^ 1)) {
+          failed = true;
+          break;
+        }
+        mbar_arrive_expect_tx(&S.full[slot], kHalfBytes);
+        bulk_g2s(S.ring + slot * kHalfBytes,
+                 p.h0 + (size_t)item * DKc * DVc + (size_t)half * kHalfRows * DVc, kHalfBytes,
+                 &S.full[slot]);
+        issued |= 1u << slot;
+        parity = (parity & ~(1u << slot)) | (sphase << slot);
+        if (++slot == lay.NS) {
+          slot = 0;
+          sphase ^= 1;
+        }
+      }
+    }
+    if (failed) {
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+      for (int s = 0; s < lay.NS; ++s)
+        if (issued & (1u << s)) mbar_wait(&S.full[s], (parity >> s) & 1u);
+    }
+    return;
+  }
+  if (warp == 9) {  // stager
+    int it = 0;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+      const bool abort_now = __any_sync(0xffffffffu, *abort_flag != 0);
+      if (abort_now || !gdn_stage<TI>(p, lay, S, item, it, lane)) {
+        if (lane == 0 && !abort_now) {
+          report(p.status, RSSM_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        return;
+      }
+    }
+    return;
+  }
+
+  // Consumers (uniform control flow, as in the Mamba-2 kernel).  Warp w
+  // holds rows 16w..16w+15 (local rows 16(w%4).. of half-tile w/4) and
+  // columns 4*lane..4*lane+3.
+  const int half = warp >> 2, row0 = 16 * warp;
+  int it = 0;
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+    const int rb = it % lay.NR;
+    const uint32_t rphase = (it / lay.NR) & 1;
+    const int b = item / p.H, h = item - (item / p.H) * p.H;
+    const size_t bh = (size_t)item;
+    const float *st = S.stage + rb * lay.stage_floats;
+    const float *qs = st, *ks = st + 128, *vs = st + 256, *alpha = st + 384;
+    const float *tail = alpha + ((L + 3) & ~3);
+    const TI *rK = reinterpret_cast<const TI *>(S.recK) + (size_t)rb * L * DKc;
+    const float *rU = S.recU + (size_t)rb * L * DVc;
+    float *db = S.db + (it & 1) * lay.db_floats;
+    float *R = db, *kk = db + ((L + 3) & ~3), *kq = kk + ((L + 3) & ~3);
+    float *gam = kq + ((L + 3) & ~3);
+    float *Kf = gam + 4;
+
+    const bool got = mbar_wait(&S.rfull[rb], rphase);
+    if (!got) {
+      report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    if (bar_or(1, kThreads, !got || *abort_flag)) break;
+    const int n0 = reinterpret_cast<const int *>(tail)[1];
+    const int pos = 2 * it + half;  // this warp's half-tile in the producer's order
+    if (reinterpret_cast<const int *>(tail)[2]) {
+      if (tid == 0) report(p.status, RSSM_ERR_STATE);
+      if (!mbar_wait(&S.full[pos % lay.NS], (pos / lay.NS) & 1)) {
+        report(p.status, RSSM_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.empty[pos % lay.NS]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.rempty[rb]);
+      continue;
+    }
+    const int k = n0 + 1;
+    const bool flush = (k == L);
+    const float beta = tail[0];
+
+    // ---- P1: appends, decay ratios, k_j.k and k_i.q, fp32 keys for the fold
+    if (!flush) {
+      TI *qb = static_cast<TI *>(p.qbuf) + (bh * p.cap + k - 1) * DKc;
+      TI *kb = static_cast<TI *>(p.kbuf) + (bh * p.cap + k - 1) * DKc;
+      TI *vb = static_cast<TI *>(p.vbuf) + (bh * p.cap + k - 1) * DVc;
+      if (tid < 128) {
+        qb[tid] = from_f32<TI>(qs[tid]);
+        kb[tid] = rK[(k - 1) * DKc + tid];
+      } else {
+        vb[tid - 128] = from_f32<TI>(vs[tid - 128]);
+      }
+      if (tid == 0) {
+        p.abuf[bh * p.cap + k - 1] = alpha[k - 1];
+        p.bbuf[bh * p.cap + k - 1] = beta;
+      }
+    }
+    if (warp == 0) {  // R_i = prod_{i<m<k} alpha_m (lane i), gamma, in fp64
+      double r = 1.0;
+      for (int m = lane + 1; m < k; ++m) r *= alpha[m];
+      if (lane < k) R[lane] = (float)r;
+      if (lane == 0) gam[0] = (float)(r * alpha[0]);
+    }
+    {
+      // 2k-1 dot products of 128: k_j.k_{k-1} (j < k-1) then k_i.q (i < k);
+      // 16 threads per dot, trip count uniform across each warp
+      const int ndot = 2 * k - 1;
+      for (int base = 0; base < ndot; base += kThreads / 16) {
+        const int d = base + (tid >> 4), c0 = (tid & 15) * 8;
+        double acc = 0.0;
+        if (d < ndot) {
+          const int i = d < k - 1 ? d : d - (k - 1);
+          const float *other = d < k - 1 ? ks : qs;
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            acc = fma((double)to_f32(rK[i * DKc + c0 + e]), (double)other[c0 + e], acc);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+        if (d < ndot && (tid & 15) == 0) {
+          if (d < k - 1) kk[d] = (float)acc;
+          else kq[d - (k - 1)] = (float)acc;
+        }
+      }
+    }
+    if (flush)
+      for (int e = tid; e < k * DKc; e += kThreads) Kf[e] = to_f32(rK[e]);
+
+    // ---- P2: this warp's 16 rows into registers; partial h0^T k and h0^T q
+    const int sl = pos % lay.NS;
+    if (!mbar_wait(&S.full[sl], (pos / lay.NS) & 1)) {
+      report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    float4 hv[16];
+    const float *tile = reinterpret_cast<const float *>(S.ring + sl * kHalfBytes);
+#pragma unroll
+    for (int rho = 0; rho < 16; ++rho)
+      hv[rho] = *reinterpret_cast<const float4 *>(tile + (16 * (warp & 3) + rho) * DVc + 4 * lane);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.empty[sl]);
+    {
+      float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float4 k4 = *reinterpret_cast<const float4 *>(&ks[row0 + 4 * t]);
+        const float4 q4 = *reinterpret_cast<const float4 *>(&qs[row0 + 4 * t]);
+        const float kr[4] = {k4.x, k4.y, k4.z, k4.w}, qr[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 x = hv[4 * t + e];
+          pk.x = fmaf(kr[e], x.x, pk.x);
+          pk.y = fmaf(kr[e], x.y, pk.y);
+          pk.z = fmaf(kr[e], x.z, pk.z);
+          pk.w = fmaf(kr[e], x.w, pk.w);
+          pq.x = fmaf(qr[e], x.x, pq.x);
+          pq.y = fmaf(qr[e], x.y, pq.y);
+          pq.z = fmaf(qr[e], x.z, pq.z);
+          pq.w = fmaf(qr[e], x.w, pq.w);
+        }
+      }
+      *reinterpret_cast<float4 *>(&S.part[(warp * 2 + 0) * 128 + 4 * lane]) = pk;
+      *reinterpret_cast<float4 *>(&S.part[(warp * 2 + 1) * 128 + 4 * lane]) = pq;
+    }
+    bar_sync(1, kThreads);
+    // ---- P3: z = h0^T k, zq = h0^T q (fixed summation order over the warps)
+    {
+      const int vsel = tid >> 7, c = tid & 127;
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) acc += S.part[(w * 2 + vsel) * 128 + c];
+      S.z[vsel * 128 + c] = acc;
+    }
+    bar_sync(1, kThreads);
+    // ---- P4: u of this record, the output (one column per thread)
+    if (tid < 128) {
+      const int c = tid;
+      const float g = gam[0];
+      float acc = vs[c] - g * S.z[c];
+      for (int j = 0; j < k - 1; ++j) acc = fmaf(-R[j] * kk[j], rU[j * DVc + c], acc);
+      const float u = beta * acc;
+      float o = g * S.z[128 + c];
+      for (int i = 0; i < k - 1; ++i) o = fmaf(R[i] * kq[i], rU[i * DVc + c], o);
+      o = fmaf(kq[k - 1], u, o);  // R_{k-1} = 1
+      p.y[b * p.bs_y + (size_t)h * DVc + c] = p.scale * o;
+      if (!flush) p.ubuf[(bh * p.cap + k - 1) * DVc + c] = u;
+      S.ucur[c] = u;
+    }
+    // ---- P5 (flush): h0 <- gamma h0 + sum_i R_i k_i u_i^T, written once
+    if (flush) {
+      bar_sync(1, kThreads);
+      const float g = gam[0];
+#pragma unroll
+      for (int rho = 0; rho < 16; ++rho) {
+        hv[rho].x *= g;
+        hv[rho].y *= g;
+        hv[rho].z *= g;
+        hv[rho].w *= g;
+      }
+      for (int i = 0; i < k; ++i) {
+        const float4 ui = *reinterpret_cast<const float4 *>(
+            i < k - 1 ? &rU[i * DVc + 4 * lane] : &S.ucur[4 * lane]);
+        const float ri = R[i];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float4 k4 = *reinterpret_cast<const float4 *>(&Kf[i * DKc + row0 + 4 * t]);
+          const float kr[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float w = ri * kr[e];
+            hv[4 * t + e].x = fmaf(w, ui.x, hv[4 * t + e].x);
+            hv[4 * t + e].y = fmaf(w, ui.y, hv[4 * t + e].y);
+            hv[4 * t + e].z = fmaf(w, ui.z, hv[4 * t + e].z);
+            hv[4 * t + e].w = fmaf(w, ui.w, hv[4 * t + e].w);
+          }
+        }
+      }
+      float *dst = p.h0 + bh * (DKc * DVc);
+#pragma unroll
+      for (int rho = 0; rho < 16; ++rho)
+        st_stream(dst + (size_t)(row0 + rho) * DVc + 4 * lane, hv[rho]);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.rempty[rb]);
+    if (tid == 0) p.len[bh] = flush ? 0 : k;
+  }
+}
+
+int gdn_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n > 0 ? n : 148;
+}
+
+template <typename TI>
+cudaError_t gdn_launch_persistent(const GDNParams &p, cudaStream_t s) {
+  const GdnLayout lay = GdnLayout::make(p.L, (int)sizeof(TI), 220 * 1024);
+  if (lay.NS < 4) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(gdn_decode_kernel<TI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+  if (e != cudaSuccess) return e;
+  const int nitems = p.B * p.H;
+  const int grid = nitems < gdn_sm_count() ? nitems : gdn_sm_count();
+  gdn_decode_kernel<TI><<<grid, kThreads + 64, lay.total, s>>>(p, lay);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 bool gdn_supported(int DK, int DV) { return DK == DKc && DV == DVc; }
 
 cudaError_t gdn_launch_decode(const GDNParams &p, cudaStream_t s) {
   if (p.B * p.H == 0) return cudaSuccess;
-  return launch_dt<kGdnDecode>(p, s);
+  return p.in_bf16 ? gdn_launch_persistent<__nv_bfloat16>(p, s) : gdn_launch_persistent<float>(p, s);
 }
 
 cudaError_t gdn_launch_fold(const GDNParams &p, int mode, cudaStream_t s) {

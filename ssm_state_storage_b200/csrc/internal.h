@@ -45,7 +45,7 @@ struct GDNParams {
   float scale;
   float *h0;
   void *qbuf, *kbuf, *vbuf;
-  float *abuf, *bbuf;
+  float *abuf, *bbuf, *ubuf;
   int32_t *len;
   int32_t *status;
   const void *q, *k, *v;

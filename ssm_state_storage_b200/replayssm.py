@@ -28,8 +28,8 @@ STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "unsu
 KIND = {"m2": 0, "gdn": 1}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 FMT = {"none": 0, "fp8": 1, "nvfp4": 2}
-BYTES = {"h0": 0, "buf0": 1, "buf1": 2, "buf2": 3, "buf3": 4, "buf4": 5, "len": 6, "rc": 7,
-         "rc_scale": 8, "rc_gscale": 9, "status": 10, "full_state": 11, "y": 12}
+BYTES = {"h0": 0, "buf0": 1, "buf1": 2, "buf2": 3, "buf3": 4, "buf4": 5, "buf5": 6, "len": 7,
+         "rc": 8, "rc_scale": 9, "rc_gscale": 10, "status": 11, "full_state": 12, "y": 13}
 
 
 class Desc(C.Structure):
@@ -40,7 +40,7 @@ class Desc(C.Structure):
 
 
 class State(C.Structure):
-    _fields_ = [("h0", C.c_void_p), ("buf", C.c_void_p * 5), ("len", C.c_void_p),
+    _fields_ = [("h0", C.c_void_p), ("buf", C.c_void_p * 6), ("len", C.c_void_p),
                 ("rc", C.c_void_p), ("rc_scale", C.c_void_p), ("rc_gscale", C.c_void_p),
                 ("status", C.c_void_p)]
 
@@ -164,7 +164,8 @@ class ReplayState:
                         torch.zeros(B, H, cap, N, dtype=dt_in, device=device),
                         torch.zeros(B, H, cap, P, dtype=dt_in, device=device),
                         torch.zeros(B, H, cap, dtype=f32, device=device),
-                        torch.zeros(B, H, cap, dtype=f32, device=device)]
+                        torch.zeros(B, H, cap, dtype=f32, device=device),
+                        torch.zeros(B, H, cap, P, dtype=f32, device=device)]
         for i, t in enumerate(self.buf):
             assert t.numel() * t.element_size() == layer.nbytes(f"buf{i}")
         assert self.h0.numel() * 4 == layer.nbytes("h0")
@@ -182,7 +183,7 @@ class ReplayState:
     def cstate(self) -> State:
         s = State()
         s.h0 = self.h0.data_ptr()
-        for i in range(5):
+        for i in range(6):
             s.buf[i] = self.buf[i].data_ptr() if i < len(self.buf) else None
         s.len = self.len.data_ptr()
         s.rc = self.rc.data_ptr() if self.rc is not None else None

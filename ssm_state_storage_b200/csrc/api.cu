@@ -295,6 +295,12 @@ rssm_status replayssm_verify_commit(const rssm_desc *d, rssm_state *s,
   if ((st = check_m2_inputs(drafts, true)) != RSSM_OK) return st;
   M2Params p = m2_params(d, s);
   m2_inputs(p, drafts, n_draft);
+  // the kernel bulk-copies draft rows of x, B and C: each row must start on
+  // a 16-byte boundary
+  const int64_t es = (int64_t)es_of(d);
+  if (!aligned16(drafts->in[0]) || !aligned16(drafts->in[2]) || !aligned16(drafts->in[3]) ||
+      (p.bs_x * es) % 16 || (p.bs_B * es) % 16 || (p.bs_C * es) % 16)
+    return RSSM_ERR_ALIGNMENT;
   p.y = y;
   p.acc = accepted_prev;
   p.n_draft = n_draft;

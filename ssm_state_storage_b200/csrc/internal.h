@@ -67,7 +67,6 @@ cudaError_t m2_launch_full(const M2Params &p, cudaStream_t s);
 cudaError_t m2_launch_verify(const M2Params &p, cudaStream_t s);
 bool m2_supported(int P, int N);
 bool m2_heads_supported(int hpg);  // heads per group: <= 8 or a multiple of 8
-size_t m2_verify_smem(int cap, int hpg, int P, int N, int es);
 
 cudaError_t gdn_launch_decode(const GDNParams &p, cudaStream_t s);
 cudaError_t gdn_launch_fold(const GDNParams &p, int mode, cudaStream_t s);

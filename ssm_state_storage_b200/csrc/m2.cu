@@ -758,12 +758,14 @@ __device__ __forceinline__ void decode_stager(const M2Params &p, const DecodeLay
 }
 
 // Tile producer (one lane): streams the items' checkpoint (or read-copy)
-// tiles into the ring, waiting only for free slots.
+// tiles into a ring of NS slots, hc heads per item, waiting only for free
+// slots.  On a failed wait it marks the CTA aborted and waits (bounded) for
+// the copies it has in flight before returning.
 template <int P, int N, int QM>
-__device__ __forceinline__ void decode_tiles(const M2Params &p, const DecodeLayout &lay,
-                                             const DecodeSmemPtrs &S, volatile int *abort_flag,
+__device__ __forceinline__ void stream_tiles(const M2Params &p, uint64_t *full, uint64_t *empty,
+                                             unsigned char *ring, int NS, int tile_stride,
+                                             int tile_bytes, int hc, volatile int *abort_flag,
                                              int nitems, int nchunk) {
-  const int hc = lay.hc;
   int slot = 0;
   uint32_t sphase = 0;
   uint32_t issued = 0, parity = 0;  // per slot: a copy was issued / its phase parity
@@ -773,25 +775,24 @@ __device__ __forceinline__ void decode_tiles(const M2Params &p, const DecodeLayo
     item_coords(p, item, nchunk, hc, b, g, chunk, h_first);
     const size_t bh0 = (size_t)b * p.H + h_first;
     for (int j = 0; j < hc; ++j) {
-      if (*abort_flag || !mbar_wait(&S.empty[slot], sphase ^ 1)) {
+      if (*abort_flag || !mbar_wait(&empty[slot], sphase ^ 1)) {
         failed = true;
         break;
       }
-      mbar_arrive_expect_tx(&S.full[slot], lay.tile_bytes);
-      unsigned char *dst = S.ring + slot * lay.tile_stride;
+      mbar_arrive_expect_tx(&full[slot], tile_bytes);
+      unsigned char *dst = ring + slot * tile_stride;
       const size_t bh = bh0 + j;
       if constexpr (QM == 1) {
-        bulk_g2s(dst, p.rc + bh * (size_t)(P * N), P * N, &S.full[slot]);
+        bulk_g2s(dst, p.rc + bh * (size_t)(P * N), P * N, &full[slot]);
       } else if constexpr (QM == 2) {
-        bulk_g2s(dst, p.rc + bh * (size_t)(P * N / 2), P * N / 2, &S.full[slot]);
-        bulk_g2s(dst + P * N / 2, p.rc_scale + bh * (size_t)(P * N / 16), P * N / 16,
-                 &S.full[slot]);
+        bulk_g2s(dst, p.rc + bh * (size_t)(P * N / 2), P * N / 2, &full[slot]);
+        bulk_g2s(dst + P * N / 2, p.rc_scale + bh * (size_t)(P * N / 16), P * N / 16, &full[slot]);
       } else {
-        bulk_g2s(dst, p.h0 + bh * (size_t)(P * N), P * N * 4, &S.full[slot]);
+        bulk_g2s(dst, p.h0 + bh * (size_t)(P * N), P * N * 4, &full[slot]);
       }
       issued |= 1u << slot;
       parity = (parity & ~(1u << slot)) | (sphase << slot);
-      if (++slot == lay.NS) {
+      if (++slot == NS) {
         slot = 0;
         sphase ^= 1;
       }
@@ -800,10 +801,17 @@ __device__ __forceinline__ void decode_tiles(const M2Params &p, const DecodeLayo
   if (failed) {
     if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
     *abort_flag = 1;
-    // do not leave the CTA with bulk copies still landing in its memory
-    for (int s = 0; s < lay.NS; ++s)
-      if (issued & (1u << s)) mbar_wait(&S.full[s], (parity >> s) & 1u);
+    for (int s = 0; s < NS; ++s)
+      if (issued & (1u << s)) mbar_wait(&full[s], (parity >> s) & 1u);
   }
+}
+
+template <int P, int N, int QM>
+__device__ __forceinline__ void decode_tiles(const M2Params &p, const DecodeLayout &lay,
+                                             const DecodeSmemPtrs &S, volatile int *abort_flag,
+                                             int nitems, int nchunk) {
+  stream_tiles<P, N, QM>(p, S.full, S.empty, S.ring, lay.NS, lay.tile_stride, lay.tile_bytes,
+                         lay.hc, abort_flag, nitems, nchunk);
 }
 
 constexpr int kDecodeThreads = kThreads + 64;  // 8 consumer warps, tile producer, stager
@@ -1175,194 +1183,457 @@ __global__ void __launch_bounds__(kThreads, 2) m2_full_kernel(const M2Params p) 
 }
 
 // ============================================================ verify round
-// 1. optional commit of the previous round (len += a; fold when >= L),
-// 2. drafts written to slots len..len+nd-1,
-// 3. draft d's output from h0 and records 0..len+d, output-only.
-// One CTA per (sequence, group); the host requires H/G <= 8.
+// Persistent speculative-verify kernel, structured like the decode kernel.
+// Work item = (sequence, group, chunk) with hc = (H/G)/nchunk heads; nchunk
+// is 1 unless the staged records of all the group's heads do not fit in
+// shared memory beside the tile ring.  Per item:
+//   1. commit of the previous round: n1 = len + accepted; when n1 >= window
+//      the n1 buffered records are folded into h0 (written once) and the
+//      drafts follow an empty buffer (nb = 0), else nb = n1;
+//   2. the nd drafts are appended to slots nb .. nb+nd-1 (len stays nb);
+//   3. draft d's output from the (possibly folded) checkpoint and records
+//      0..nb+d, with no intermediate state:
+//        y_d = Lam_d (h C_d) + sum_i w_{d,i} (B_i . C_d) x_i + D x_d.
+// The stager (warp 9) reads the lengths and acceptance counts, loads the
+// small inputs, and bulk-copies the buffered prefix records and the draft
+// rows (x, B, C); warp 8 streams the heads' checkpoint tiles; warps 0-7 form
+// the fold weights, every draft's decay weights and B.C dots (fp64) and the
+// per-row terms z_d, then take one head at a time (8 warps, 8 rows each):
+// rows into registers, slot released, optional fold + write-back, and all
+// nd outputs from the same registers.
+// With nchunk > 1 the draft B and C rows (one copy per group) are appended
+// by m2_verify_append_bc_kernel after this kernel: a chunk that folds would
+// otherwise overwrite buffered B records that another chunk's CTA may not
+// have copied yet.
 
 constexpr int kMD = 4;  // most drafts per round
 
-struct VerifySmem {
-  float *Bb, *Bd, *Cd, *dtb, *dtd, *wdt, *lamf, *coef, *lam, *red;
-  double *bc;
-  void *xb, *xd;
-  // Bb [cap][N] | Bd [4][N] | Cd [4][N] | bc [4][cap+4] | dtb [hc][cap] | dtd [hc][4]
-  // | wdt [hc][cap] | lamf [pad4(hc)] | coef [hc][4][cap+4] | lam [hc][4] | red [8]
-  // | xb [hc][cap][P] | xd [hc][4][P] (input dtype)
-  __host__ __device__ static size_t bytes(int cap, int hc, int P, int N, int es) {
-    const int R = cap + kMD;
-    const size_t f = (size_t)cap * N + 2 * kMD * N + 2 * pad4(kMD * R) + pad4(hc * cap) +
-                     hc * kMD + pad4(hc * cap) + pad4(hc) + pad4(hc * kMD * R) + hc * kMD + 8;
-    return f * 4 + (size_t)hc * (cap + kMD) * P * es;
-  }
-  __device__ VerifySmem(unsigned char *base, int cap, int hc, int N, int P, int es) {
-    const int R = cap + kMD;
-    float *f = reinterpret_cast<float *>(base);
-    Bb = f;
-    Bd = Bb + cap * N;
-    Cd = Bd + kMD * N;
-    bc = reinterpret_cast<double *>(Cd + kMD * N);
-    dtb = Cd + kMD * N + 2 * pad4(kMD * R);
-    dtd = dtb + pad4(hc * cap);
-    wdt = dtd + hc * kMD;
-    lamf = wdt + pad4(hc * cap);
-    coef = lamf + pad4(hc);
-    lam = coef + pad4(hc * kMD * R);
-    red = lam + hc * kMD;
-    xb = red + 8;
-    xd = static_cast<unsigned char *>(xb) + (size_t)hc * cap * P * es;
+struct VerifyLayout {
+  int NS, NR, hc, nchunk, cap, L, tile_bytes, tile_stride;
+  int rec_floats, db_floats;  // stage floats per record buffer, scratch per item
+  int off_bars, off_recB, off_recX, off_dX, off_dB, off_dC, off_rec, off_db, off_single, off_ring,
+      total;
+  int recB_b, recX_b, dX_b, dBC_b;  // bytes per record buffer of each array
+  __host__ static int a128(int v) { return (v + 127) & ~127; }
+  __host__ static VerifyLayout make(int P, int N, int hpg, int nchunk, int cap, int L, int es,
+                                    int budget) {
+    VerifyLayout d;
+    d.nchunk = nchunk;
+    const int hc = d.hc = hpg / nchunk;
+    d.cap = cap;
+    d.L = L;
+    d.tile_bytes = P * N * 4;
+    d.tile_stride = a128(d.tile_bytes);
+    d.recB_b = a128(cap * N * es);
+    d.recX_b = a128(hc * cap * P * es);
+    d.dX_b = a128(kMD * hc * P * es);
+    d.dBC_b = a128(kMD * N * es);
+    // stage: dt prefix [hc][cap] | dt drafts [4][hc] | A [hc] | D [hc] | hdr [8]
+    d.rec_floats = pad4(hc * cap) + kMD * hc + pad4(hc) * 2 + 8;
+    // per item: Bf [cap][N] | wf [hc][cap] | lamf [hc] | lamd [4][hc] | Cf [4][N] | z [4][hc][P]
+    d.db_floats = cap * N + pad4(hc * cap) + pad4(hc) + kMD * hc + kMD * N + kMD * hc * P;
+    for (d.NR = 2; d.NR >= 1; --d.NR) {
+      int o = 0;
+      d.off_bars = o;
+      o += 256;
+      d.off_recB = o;
+      o += d.NR * d.recB_b;
+      d.off_recX = o;
+      o += d.NR * d.recX_b;
+      d.off_dX = o;
+      o += d.NR * d.dX_b;
+      d.off_dB = o;
+      o += d.NR * d.dBC_b;
+      d.off_dC = o;
+      o += d.NR * d.dBC_b;
+      d.off_rec = o;
+      o += a128(d.NR * d.rec_floats * 4);
+      d.off_db = o;  // one copy: every item starts at a barrier of all consumer warps
+      o += a128(d.db_floats * 4);
+      d.off_single = o;  // bc [4][cap+4] double | wd [4][hc][cap+4] float
+      o += a128(kMD * (cap + kMD) * 8 + kMD * hc * (cap + kMD) * 4);
+      d.off_ring = o;
+      d.NS = (budget - o) / d.tile_stride;
+      if (d.NS > 8) d.NS = 8;
+      if (d.NS >= 2) {
+        d.total = o + d.NS * d.tile_stride;
+        return d;
+      }
+    }
+    d.NS = 0;
+    return d;
   }
 };
 
 template <int P, int N, typename TI>
-__global__ void __launch_bounds__(kThreads, 2) m2_verify_kernel(const M2Params p) {
-  using T = Tile<P, N>;
-  constexpr int RPT = T::RPT, C4 = T::C4;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, rs = lane >> 3, c8 = lane & 7;
-  const int b = blockIdx.x / p.G, g = blockIdx.x - b * p.G;
-  const int hc = p.hpg, cap = p.cap, R = cap + kMD;
-  const int h_first = g * hc;
-  const size_t bh0 = (size_t)b * p.H + h_first;
-  const int nd = p.n_draft;
-  VerifySmem S(smem_raw, cap, hc, N, P, (int)sizeof(TI));
-  TI *s_xb = static_cast<TI *>(S.xb);
-  TI *s_xd = static_cast<TI *>(S.xd);
+__device__ __forceinline__ bool verify_stage(const M2Params &p, const VerifyLayout &lay,
+                                             unsigned char *smem, uint64_t *rfull,
+                                             uint64_t *rempty, int item, int it, int lane) {
+  constexpr int DPL = (8 * 20 + 31) / 32;  // prefix dt slots per lane (hc <= 8, cap <= 20)
+  const int hc = lay.hc, cap = lay.cap, L = lay.L, nd = p.n_draft;
+  const int rb = it % lay.NR;
+  const uint32_t rphase = (it / lay.NR) & 1;
+  bool ok = true;
+  if (lane == 0) ok = mbar_wait(&rempty[rb], rphase ^ 1);
+  if (!__shfl_sync(0xffffffffu, (int)ok, 0)) return false;
+  int b, g, chunk, h_first;
+  item_coords(p, item, lay.nchunk, hc, b, g, chunk, h_first);
+  const size_t bh0 = (size_t)b * p.H + h_first, bg = (size_t)b * p.G + g;
 
-  float4 cur[RPT][C4];
-  load_tile<P, N>(p.h0 + bh0 * (size_t)(P * N), warp, rs, c8, cur);
-
-  const int n0 = p.len[bh0];
-  const int a = p.acc ? p.acc[b] : 0;
+  // ---- loads
+  const int my_len = lane < hc ? __ldcg(&p.len[bh0 + lane]) : 0;
+  const int a = p.acc ? __ldcg(&p.acc[b]) : 0;
+  const float my_A = lane < hc ? p.A[h_first + lane] : 0.f;
+  const float my_D = lane < hc ? p.D[h_first + lane] : 0.f;
+  float dtv[DPL];
+#pragma unroll
+  for (int u = 0; u < DPL; ++u) {
+    const int e = lane + 32 * u, j = e / cap, i = e - j * cap;
+    dtv[u] = e < hc * cap ? __ldcg(&p.dtbuf[(bh0 + j) * cap + i]) : 0.f;
+  }
+  const int dd = lane / hc, dj = lane - (lane / hc) * hc;  // draft dt: lane -> (d, j)
+  const float my_dtd = lane < nd * hc ? ld_in<TI>(p.dt, b * p.bs_dt + (int64_t)dd * p.H + h_first + dj)
+                                      : 0.f;
+  // ---- lengths and checks
+  const int n0 = __shfl_sync(0xffffffffu, my_len, 0);
   const int n1 = n0 + a;
-  const bool fold = n1 >= p.L;
-  const int nb = fold ? 0 : n1;  // committed records the drafts follow
-  bool bad = tid == 0 && (n0 < 0 || n0 >= p.L || a < 0 || a > p.draft_max || n1 > cap ||
-                          nb + nd > cap);
-  if (tid > 0 && tid < hc) bad = p.len[bh0 + tid] != n0;
-  if (__syncthreads_or(bad)) {
-    if (tid == 0) report(p.status, RSSM_ERR_STATE);
+  const bool fold = n1 >= L;
+  const int nb = fold ? 0 : n1;
+  const bool bad = __any_sync(0xffffffffu, (lane < hc && my_len != n0)) || n0 < 0 || n0 >= L ||
+                   a < 0 || a > p.draft_max || n1 > cap || nb + nd > cap;
+  const int n1c = bad ? 0 : n1;  // copies stay in bounds for a bad item
+  // ---- shared-memory writes
+  float *st = reinterpret_cast<float *>(smem + lay.off_rec) + rb * lay.rec_floats;
+  float *dtb = st, *dtd = st + pad4(hc * cap), *As = dtd + kMD * hc, *Ds = As + pad4(hc);
+  int *hdr = reinterpret_cast<int *>(Ds + pad4(hc));
+#pragma unroll
+  for (int u = 0; u < DPL; ++u) {
+    const int e = lane + 32 * u;
+    if (e < hc * cap) dtb[e] = dtv[u];
+  }
+  if (lane < nd * hc) dtd[dd * hc + dj] = my_dtd;
+  if (lane < hc) {
+    As[lane] = my_A;
+    Ds[lane] = my_D;
+  }
+  if (lane == 0) {
+    hdr[0] = n0;
+    hdr[1] = n1;
+    hdr[2] = fold;
+    hdr[3] = nb;
+    hdr[4] = bad;
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    const uint32_t bB = n1c * N * sizeof(TI), bX = n1c * P * sizeof(TI);
+    const uint32_t bdX = hc * P * sizeof(TI), bdBC = N * sizeof(TI);
+    const uint32_t dcount = bad ? 0 : nd;
+    mbar_arrive_expect_tx(&rfull[rb], bB + hc * bX + dcount * (bdX + 2 * bdBC));
+    unsigned char *recB = smem + lay.off_recB + rb * lay.recB_b;
+    unsigned char *recX = smem + lay.off_recX + rb * lay.recX_b;
+    unsigned char *dX = smem + lay.off_dX + rb * lay.dX_b;
+    unsigned char *dB = smem + lay.off_dB + rb * lay.dBC_b;
+    unsigned char *dC = smem + lay.off_dC + rb * lay.dBC_b;
+    if (n1c > 0) {
+      bulk_g2s(recB, static_cast<const TI *>(p.Bbuf) + bg * cap * N, bB, &rfull[rb]);
+      for (int j = 0; j < hc; ++j)
+        bulk_g2s(recX + (size_t)j * cap * P * sizeof(TI),
+                 static_cast<const TI *>(p.xbuf) + (bh0 + j) * cap * P, bX, &rfull[rb]);
+    }
+    for (uint32_t d = 0; d < dcount; ++d) {
+      bulk_g2s(dX + d * bdX, static_cast<const TI *>(p.x) + b * p.bs_x + ((size_t)d * p.H + h_first) * P,
+               bdX, &rfull[rb]);
+      bulk_g2s(dB + d * bdBC, static_cast<const TI *>(p.Bm) + b * p.bs_B + ((size_t)d * p.G + g) * N,
+               bdBC, &rfull[rb]);
+      bulk_g2s(dC + d * bdBC, static_cast<const TI *>(p.Cm) + b * p.bs_C + ((size_t)d * p.G + g) * N,
+               bdBC, &rfull[rb]);
+    }
+  }
+  return true;
+}
+
+// Butterfly reduce-scatter of four per-lane partial sums over the 8 lanes of
+// a row group (lane bits 0-2): lane c8 ends with the full sum of value
+// c8 >> 1 (lanes c8 and c8 ^ 1 hold the same sum).  4 shuffles instead of 12.
+__device__ __forceinline__ float reduce4_over8(const float (&q)[4], int c8) {
+  const bool hi = c8 & 4;
+  float a0 = hi ? q[2] : q[0], a1 = hi ? q[3] : q[1];
+  const float s0 = hi ? q[0] : q[2], s1 = hi ? q[1] : q[3];
+  a0 += __shfl_xor_sync(0xffffffffu, s0, 4);
+  a1 += __shfl_xor_sync(0xffffffffu, s1, 4);
+  const bool mid = c8 & 2;
+  float k = mid ? a1 : a0;
+  k += __shfl_xor_sync(0xffffffffu, mid ? a0 : a1, 2);
+  return k + __shfl_xor_sync(0xffffffffu, k, 1);
+}
+
+constexpr int kVWarps = 16, kVThreads = 32 * kVWarps;  // verify consumer warps / threads
+
+template <int P, int N, typename TI>
+__global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyLayout lay) {
+  using T = Tile<P, N>;
+  constexpr int C4 = T::C4;
+  constexpr int RW = P / kVWarps, RG = RW / 4;  // one head at a time: 16 warps x RW rows
+  static_assert(RG >= 1, "headdim must be at least 64");
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int abort_word;
+  volatile int *abort_flag = &abort_word;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.off_bars);
+  uint64_t *empty = full + 8, *rfull = empty + 8, *rempty = rfull + 4;
+  unsigned char *ring = smem + lay.off_ring;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, rs = lane >> 3, c8 = lane & 7;
+  const int hc = lay.hc, cap = lay.cap, nd = p.n_draft, R = cap + kMD;
+  const int nitems = p.B * p.G * lay.nchunk;
+  const bool own_bc = lay.nchunk == 1;
+
+  if (tid == 0) {
+    for (int s = 0; s < 8; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kVWarps);
+    }
+    for (int r = 0; r < 4; ++r) {
+      mbar_init(&rfull[r], 1);
+      mbar_init(&rempty[r], kVWarps);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == kVWarps) {
+    if (lane == 0)
+      stream_tiles<P, N, 0>(p, full, empty, ring, lay.NS, lay.tile_stride, lay.tile_bytes, hc,
+                            abort_flag, nitems, lay.nchunk);
+    return;
+  }
+  if (warp == kVWarps + 1) {
+    int it = 0;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+      const bool abort_now = __any_sync(0xffffffffu, *abort_flag != 0);
+      if (abort_now || !verify_stage<P, N, TI>(p, lay, smem, rfull, rempty, item, it, lane)) {
+        if (lane == 0 && !abort_now) {
+          report(p.status, RSSM_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        return;
+      }
+    }
     return;
   }
 
-  // ---- stage buffered records 0..n1-1 and the drafts
-  const size_t bg = (size_t)b * p.G + g;
-  TI *Bb = static_cast<TI *>(p.Bbuf) + bg * cap * N;
-  TI *Cb = static_cast<TI *>(p.Cbuf) + bg * cap * N;
-  TI *xbuf = static_cast<TI *>(p.xbuf);
-  stage_f32<TI>(S.Bb, Bb, n1 * N, tid);
-  for (int j = 0; j < hc; ++j)
-    stage_raw(s_xb + j * cap * P, xbuf + (bh0 + j) * cap * P, n1 * P * (int)sizeof(TI), tid);
-  for (int e = tid; e < hc * n1; e += kThreads) {
-    const int j = e / n1, i = e - j * n1;
-    S.dtb[j * cap + i] = p.dtbuf[(bh0 + j) * cap + i];
+  double *bc = reinterpret_cast<double *>(smem + lay.off_single);  // [4][R]
+  float *cf = reinterpret_cast<float *>(bc + kMD * R);             // [4][hc][R] coefficients
+  int it = 0;
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+    const int rb = it % lay.NR;
+    const uint32_t rphase = (it / lay.NR) & 1;
+    int b, g, chunk, h_first;
+    item_coords(p, item, lay.nchunk, hc, b, g, chunk, h_first);
+    const size_t bh0 = (size_t)b * p.H + h_first, bg = (size_t)b * p.G + g;
+    const float *st = reinterpret_cast<const float *>(smem + lay.off_rec) + rb * lay.rec_floats;
+    const float *dtb = st, *dtd = st + pad4(hc * cap), *As = dtd + kMD * hc, *Ds = As + pad4(hc);
+    const int *hdr = reinterpret_cast<const int *>(Ds + pad4(hc));
+    const TI *recB = reinterpret_cast<const TI *>(smem + lay.off_recB + rb * lay.recB_b);
+    const TI *recX = reinterpret_cast<const TI *>(smem + lay.off_recX + rb * lay.recX_b);
+    const TI *dX = reinterpret_cast<const TI *>(smem + lay.off_dX + rb * lay.dX_b);
+    const TI *dB = reinterpret_cast<const TI *>(smem + lay.off_dB + rb * lay.dBC_b);
+    const TI *dC = reinterpret_cast<const TI *>(smem + lay.off_dC + rb * lay.dBC_b);
+    float *db = reinterpret_cast<float *>(smem + lay.off_db);
+    float *Bf = db, *wf = Bf + cap * N, *lamf = wf + pad4(hc * cap), *lamd = lamf + pad4(hc);
+    float *Cf = lamd + kMD * hc, *z = Cf + kMD * N;
+
+    const bool got = mbar_wait(&rfull[rb], rphase);
+    if (!got) {
+      report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    if (bar_or(1, kVThreads, !got || *abort_flag)) break;
+    if (hdr[4]) {
+      if (tid == 0) report(p.status, RSSM_ERR_STATE);
+      for (int j = 0; j < hc; ++j) {
+        const uint32_t pos = (uint32_t)it * hc + j;
+        if (!mbar_wait(&full[pos % lay.NS], (pos / lay.NS) & 1)) {
+          report(p.status, RSSM_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[pos % lay.NS]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rempty[rb]);
+      continue;
+    }
+    const int n1 = hdr[1], nb = hdr[3], K = nb + nd;
+    const bool fold = hdr[2];
+
+    // ---- S1: append the drafts; fp32 copies; B_i . C_d in fp64
+    for (int e = tid; e < nd * hc * P; e += kVThreads) {
+      const int d = e / (hc * P), rem = e - d * (hc * P), j = rem / P, q = rem - j * P;
+      static_cast<TI *>(p.xbuf)[((bh0 + j) * cap + nb + d) * P + q] = dX[(d * hc + j) * P + q];
+    }
+    for (int e = tid; e < nd * N; e += kVThreads) {
+      const int d = e / N, c = e - d * N;
+      if (own_bc) {
+        static_cast<TI *>(p.Bbuf)[(bg * cap + nb + d) * N + c] = dB[d * N + c];
+        static_cast<TI *>(p.Cbuf)[(bg * cap + nb + d) * N + c] = dC[d * N + c];
+      }
+      Cf[d * N + c] = to_f32(dC[d * N + c]);
+    }
+    if (tid < nd * hc) {
+      const int d = tid / hc, j = tid - (tid / hc) * hc;
+      p.dtbuf[(bh0 + j) * cap + nb + d] = dtd[d * hc + j];
+    }
+    if (fold)
+      for (int e = tid; e < n1 * N; e += kVThreads) Bf[e] = to_f32(recB[e]);
+    {
+      const int npair = nd * K;  // (d, i) with i <= nb + d are used
+      constexpr int PER = N / 16;
+      for (int base = 0; base < npair; base += kVThreads / 16) {
+        const int pr = base + (tid >> 4), c0 = (tid & 15) * PER;
+        const int d = pr / K, i = pr - d * K;
+        const bool use = pr < npair && i <= nb + d;
+        double acc = 0.0;
+        if (use) {
+          const TI *Bi = i < nb ? recB + i * N : dB + (i - nb) * N;
+#pragma unroll
+          for (int e = 0; e < PER; ++e)
+            acc = fma((double)to_f32(Bi[c0 + e]), (double)to_f32(dC[d * N + c0 + e]), acc);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+        if (use && (tid & 15) == 0) bc[d * R + i] = acc;
+      }
+    }
+    bar_sync(1, kVThreads);
+
+    // ---- S2 (one warp per head): decay weights from fp64 suffix sums.
+    // Draft sequence: the nb committed records, then the nd drafts; with
+    // S_l = sum_{m >= l} dt_m, draft d (records 0..nb+d) weighs record i by
+    // exp(A (S_{i+1} - S_{nb+d+1})) dt_i.  The fold sequence is the n1
+    // committed records.  Both scans run together.
+    for (int j = warp; j < hc; j += kVWarps) {
+      const double A = As[j];
+      const double dts = lane < nb ? (double)dtb[j * cap + lane]
+                                   : (lane < K ? (double)dtd[(lane - nb) * hc + j] : 0.0);
+      const double dtf = fold && lane < n1 ? (double)dtb[j * cap + lane] : 0.0;
+      double Ss = dts, Sf = dtf;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double ts = __shfl_down_sync(0xffffffffu, Ss, o);
+        const double tf = __shfl_down_sync(0xffffffffu, Sf, o);
+        if (lane + o < 32) {
+          Ss += ts;
+          Sf += tf;
+        }
+      }
+      const double Ss1 = __shfl_down_sync(0xffffffffu, Ss, 1);  // S_{l+1} (lane 31: unused)
+      const double Sf1 = __shfl_down_sync(0xffffffffu, Sf, 1);
+      const double Ss0 = __shfl_sync(0xffffffffu, Ss, 0);
+      double Se[kMD];
+#pragma unroll
+      for (int d = 0; d < kMD; ++d) Se[d] = __shfl_sync(0xffffffffu, Ss, (nb + d + 1) & 31);
+      if (fold) {
+        if (lane < n1) wf[j * cap + lane] = (float)(exp(A * (lane + 1 < n1 ? Sf1 : 0.0)) * dtf);
+        if (lane == 0) lamf[j] = (float)exp(A * Sf);
+      }
+#pragma unroll
+      for (int d = 0; d < kMD; ++d) {
+        if (d < nd) {
+          const int e = nb + d;  // last record of draft d
+          const double se = e + 1 < K ? Se[d] : 0.0;
+          if (lane <= e)
+            cf[(d * hc + j) * R + lane] =
+                (float)(exp(A * ((lane < e ? Ss1 : se) - se)) * dts * bc[d * R + lane]);
+          if (lane == 0) lamd[d * hc + j] = (float)exp(A * (Ss0 - se));
+        }
+      }
+    }
+    bar_sync(1, kVThreads);
+    // ---- S3: z[d][j][r] = sum_i cf[d][j][i] x_i[r] + D_j x_d[r]
+    for (int e = tid; e < nd * hc * P; e += kVThreads) {
+      const int d = e / (hc * P), rem = e - d * (hc * P), j = rem / P, r = rem - j * P;
+      const float *c = cf + (d * hc + j) * R;
+      float acc = 0.f;
+      int i = 0;
+      for (; i < nb; ++i) acc = fmaf(c[i], to_f32(recX[(j * cap + i) * P + r]), acc);
+      for (; i <= nb + d; ++i) acc = fmaf(c[i], to_f32(dX[((i - nb) * hc + j) * P + r]), acc);
+      z[e] = fmaf(Ds[j], to_f32(dX[(d * hc + j) * P + r]), acc);
+    }
+    bar_sync(1, kVThreads);
+
+    // ---- heads, one at a time: rows into registers, optional fold, outputs
+    const int dmine = c8 >> 1;  // the draft whose sum this lane ends with
+    for (int j = 0; j < hc; ++j) {
+      const int h = h_first + j;
+      const size_t bh = bh0 + j;
+      const uint32_t pos = (uint32_t)it * hc + j;
+      const int sl = pos % lay.NS;
+      if (!mbar_wait(&full[sl], (pos / lay.NS) & 1)) {
+        report(p.status, RSSM_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      float4 v[RG][C4];
+      int rows[RG];
+#pragma unroll
+      for (int u = 0; u < RG; ++u) {
+        rows[u] = warp * RW + 4 * u + rs;
+        view_row<P, N, 0>(ring + sl * lay.tile_stride, rows[u], c8, 1.0f, v[u]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[sl]);
+      if (fold) {
+        fold_rows<P, N, TI, RG>(v, lamf[j], n1, wf + j * cap, recX + j * cap * P, rows, Bf, c8);
+        float *tile = p.h0 + bh * (size_t)(P * N);
+#pragma unroll
+        for (int u = 0; u < RG; ++u) store_row<N>(tile, rows[u], c8, v[u]);
+      }
+      float q[RG][kMD];
+#pragma unroll
+      for (int d = 0; d < kMD; ++d) {
+        float4 cd[C4];
+#pragma unroll
+        for (int s = 0; s < C4; ++s) cd[s] = *reinterpret_cast<const float4 *>(&Cf[d * N + T::col(c8, s)]);
+#pragma unroll
+        for (int u = 0; u < RG; ++u) q[u][d] = tree_dot<C4>(v[u], cd);
+      }
+      float a[RG];
+#pragma unroll
+      for (int u = 0; u < RG; ++u) a[u] = reduce4_over8(q[u], c8);  // every lane shuffles
+      if (dmine < nd && (c8 & 1) == 0) {
+        const float ld = lamd[dmine * hc + j];
+        const float *zd = z + (dmine * hc + j) * P;
+        float *yd = p.y + b * p.bs_y + ((size_t)dmine * p.H + h) * P;
+#pragma unroll
+        for (int u = 0; u < RG; ++u) yd[rows[u]] = fmaf(ld, a[u], zd[rows[u]]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&rempty[rb]);
+    if (tid < hc) p.len[bh0 + tid] = nb;
   }
+}
+
+// Chunked verify only: append the draft B and C rows of group (b, g) at the
+// group's committed length, read back from the length the verify kernel just
+// wrote.  An item the verify kernel rejected (its status already reports it)
+// is skipped when the slots would not fit.
+template <typename TI>
+__global__ void __launch_bounds__(128) m2_verify_append_bc_kernel(const M2Params p) {
+  const int b = blockIdx.x / p.G, g = blockIdx.x - (blockIdx.x / p.G) * p.G;
+  const size_t bg = (size_t)b * p.G + g;
+  const int nb = p.len[(size_t)b * p.H + (size_t)g * p.hpg];
+  if (nb < 0 || nb + p.n_draft > p.cap) return;
   const TI *Bin = static_cast<const TI *>(p.Bm) + b * p.bs_B;
   const TI *Cin = static_cast<const TI *>(p.Cm) + b * p.bs_C;
-  for (int e = tid; e < nd * N; e += kThreads) {
-    const int d = e / N, c = e - d * N;
-    S.Bd[e] = to_f32(Bin[((size_t)d * p.G + g) * N + c]);
-    S.Cd[e] = to_f32(Cin[((size_t)d * p.G + g) * N + c]);
+  for (int e = threadIdx.x; e < p.n_draft * p.N; e += blockDim.x) {
+    const int d = e / p.N, c = e - d * p.N;
+    static_cast<TI *>(p.Bbuf)[(bg * p.cap + nb + d) * p.N + c] = Bin[((size_t)d * p.G + g) * p.N + c];
+    static_cast<TI *>(p.Cbuf)[(bg * p.cap + nb + d) * p.N + c] = Cin[((size_t)d * p.G + g) * p.N + c];
   }
-  const TI *xin = static_cast<const TI *>(p.x) + b * p.bs_x;
-  for (int e = tid; e < hc * nd * P; e += kThreads) {
-    const int j = e / (nd * P), rem = e - j * (nd * P), d = rem / P, q = rem - d * P;
-    s_xd[(j * kMD + d) * P + q] = xin[((size_t)d * p.H + h_first + j) * P + q];
-  }
-  for (int e = tid; e < hc * nd; e += kThreads) {
-    const int j = e / nd, d = e - j * nd;
-    S.dtd[j * kMD + d] = ld_in<TI>(p.dt, b * p.bs_dt + (int64_t)d * p.H + h_first + j);
-  }
-  __syncthreads();
-
-  // ---- drafts into their slots (after the reads above: with a fold they
-  // overwrite records just staged); B.C dots; decay weights and coefficients
-  for (int e = tid; e < nd * N; e += kThreads) {
-    const int d = e / N, c = e - d * N;
-    Bb[(size_t)(nb + d) * N + c] = Bin[((size_t)d * p.G + g) * N + c];
-    Cb[(size_t)(nb + d) * N + c] = Cin[((size_t)d * p.G + g) * N + c];
-  }
-  for (int e = tid; e < hc * nd * P; e += kThreads) {
-    const int j = e / (nd * P), rem = e - j * (nd * P), d = rem / P, q = rem - d * P;
-    xbuf[((bh0 + j) * cap + nb + d) * P + q] = s_xd[(j * kMD + d) * P + q];
-  }
-  for (int e = tid; e < hc * nd; e += kThreads) {
-    const int j = e / nd, d = e - j * nd;
-    p.dtbuf[(bh0 + j) * cap + nb + d] = S.dtd[j * kMD + d];
-  }
-  for (int pr = warp; pr < nd * (nb + nd); pr += 8) {
-    const int d = pr / (nb + nd), i = pr - d * (nb + nd);
-    if (i <= nb + d) {
-      const float *Bi = i < nb ? S.Bb + i * N : S.Bd + (i - nb) * N;
-      double acc = 0.0;
-      for (int c = lane; c < N; c += 32) acc = fma((double)Bi[c], (double)S.Cd[d * N + c], acc);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) S.bc[d * R + i] = acc;
-    }
-  }
-  __syncthreads();
-  for (int j = warp; j < hc; j += 8) {
-    const float A = p.A[h_first + j];
-    const float *dtb = S.dtb + j * cap, *dtd = S.dtd + j * kMD;
-    if (fold) decay_weights(dtb, n1, A, S.wdt + j * cap, S.lamf + j, lane);
-    for (int d = 0; d < nd; ++d) {
-      const int kd = nb + d + 1;
-      if (lane < kd) {
-        double s = 0.0;
-        for (int m = lane + 1; m < kd; ++m) s += m < nb ? dtb[m] : dtd[m - nb];
-        const double dti = lane < nb ? dtb[lane] : dtd[lane - nb];
-        S.coef[(j * kMD + d) * R + lane] = (float)(exp((double)A * s) * dti * S.bc[d * R + lane]);
-      }
-      if (lane == 0) {
-        double t = 0.0;
-        for (int m = 0; m < kd; ++m) t += m < nb ? dtb[m] : dtd[m - nb];
-        S.lam[j * kMD + d] = (float)exp((double)A * t);
-      }
-    }
-  }
-  __syncthreads();
-
-  // ---- head loop: optional fold, then the draft outputs from one tile read
-  for (int j = 0; j < hc; ++j) {
-    const int h = h_first + j;
-    const size_t bh = bh0 + j;
-    float4 nxt[RPT][C4];
-    if (j + 1 < hc) load_tile<P, N>(p.h0 + (bh + 1) * (size_t)(P * N), warp, rs, c8, nxt);
-    if (fold) {
-      fold_regs<P, N, TI>(cur, S.lamf[j], n1, S.wdt + j * cap, s_xb + j * cap * P, S.Bb, warp,
-                          rs, c8);
-      store_tile<P, N>(p.h0 + bh * (size_t)(P * N), warp, rs, c8, cur);
-    }
-    const float Dh = p.D[h];
-    const TI *xbj = s_xb + j * cap * P, *xdj = s_xd + j * kMD * P;
-#pragma unroll
-    for (int rho = 0; rho < RPT; ++rho) {
-      const int r = T::row(warp, rs, rho);
-      for (int d = 0; d < nd; ++d) {
-        float acc = 0.f;
-#pragma unroll
-        for (int s = 0; s < C4; ++s)
-          acc += dot4(cur[rho][s], *reinterpret_cast<const float4 *>(&S.Cd[d * N + T::col(c8, s)]));
-        acc *= S.lam[j * kMD + d];
-        const float *cf = S.coef + (j * kMD + d) * R;
-        for (int i = c8; i <= nb + d; i += 8) {
-          const float xi = i < nb ? to_f32(xbj[i * P + r]) : to_f32(xdj[(i - nb) * P + r]);
-          acc = fmaf(cf[i], xi, acc);
-        }
-        acc = sum8(acc);
-        if (c8 == 0)
-          p.y[b * p.bs_y + ((size_t)d * p.H + h) * P + r] = fmaf(Dh, to_f32(xdj[d * P + r]), acc);
-      }
-    }
-    if (j + 1 < hc) {
-#pragma unroll
-      for (int rho = 0; rho < RPT; ++rho)
-#pragma unroll
-        for (int s = 0; s < C4; ++s) cur[rho][s] = nxt[rho][s];
-    }
-  }
-  if (tid < hc) p.len[bh0 + tid] = nb;
 }
 
 // ================================================================= launchers
@@ -1473,10 +1744,6 @@ bool m2_supported(int P, int N) { return (P == 64 || P == 128) && (N == 64 || N 
 
 bool m2_heads_supported(int hpg) { return hpg <= 8 || hpg % 8 == 0; }
 
-size_t m2_verify_smem(int cap, int hpg, int P, int N, int es) {
-  return VerifySmem::bytes(cap, hpg, P, N, es);
-}
-
 cudaError_t m2_launch_decode(const M2Params &p, cudaStream_t s) {
   if (p.B * p.G == 0) return cudaSuccess;
   return dispatch_shape(p.P, p.N, p.in_bf16, [&](auto PP, auto NN, auto ti) {
@@ -1504,10 +1771,25 @@ cudaError_t m2_launch_verify(const M2Params &p, cudaStream_t s) {
   if (p.B * p.G == 0) return cudaSuccess;
   return dispatch_shape(p.P, p.N, p.in_bf16, [&](auto PP, auto NN, auto ti) {
     using TI = decltype(ti);
-    const size_t smem = VerifySmem::bytes(p.cap, p.hpg, decltype(PP)::value, decltype(NN)::value,
-                                          sizeof(TI));
-    return launch_dyn(m2_verify_kernel<decltype(PP)::value, decltype(NN)::value, TI>,
-                      (unsigned)(p.B * p.G), smem, s, p);
+    constexpr int P_ = decltype(PP)::value, N_ = decltype(NN)::value;
+    VerifyLayout lay;
+    lay.NS = 0;
+    for (int nc = 1; nc <= p.hpg && lay.NS < 2; ++nc)
+      if (p.hpg % nc == 0)
+        lay = VerifyLayout::make(P_, N_, p.hpg, nc, p.cap, p.L, (int)sizeof(TI), 220 * 1024);
+    if (lay.NS < 2) return cudaErrorInvalidConfiguration;
+    auto kernel = m2_verify_kernel<P_, N_, TI>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+    if (e != cudaSuccess) return e;
+    const int nitems = p.B * p.G * lay.nchunk;
+    const int grid = nitems < sm_count() ? nitems : sm_count();
+    kernel<<<grid, kVThreads + 64, lay.total, s>>>(p, lay);
+    if (lay.nchunk > 1) {
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      m2_verify_append_bc_kernel<TI><<<p.B * p.G, 128, 0, s>>>(p);
+    }
+    return cudaGetLastError();
   });
 }
 

@@ -61,6 +61,42 @@ def test_verify_rounds_match_oracle():
     assert rel_err(_gpu.f64(S_out), Ss) < TOL
 
 
+@pytest.mark.parametrize("P,N,dtype,H,G", [
+    (128, 128, torch.float32, 16, 2),   # 8 heads per group do not fit one CTA: head chunks
+    (64, 64, torch.float32, 12, 2),     # 6 heads per group
+    (128, 64, torch.bfloat16, 8, 8),    # one head per group
+    (64, 128, torch.bfloat16, 6, 2),    # 3 heads per group
+])
+def test_verify_shapes_match_oracle(P, N, dtype, H, G):
+    w, A, D, S0, rd = _draw(20, B=3, H=H, G=G, P=P, N=N, in_dtype=dtype)
+    layer, state, y, lens = _gpu_rounds(w, A, D, S0, rd)
+    orc = oracle.M2Replay(S0, G=w.G, L=w.L, cap=w.L + w.n_draft - 1)
+    yo, lt = orc.verify(rd["x"], rd["dt"], rd["Bm"], rd["Cm"], A, D, rd["acc"])
+    assert state.status() == 0
+    assert np.array_equal(lens[1:], lt)
+    assert per_step_rel_err(y.reshape(-1, *y.shape[3:]), yo.reshape(-1, *yo.shape[3:])) < TOL
+    assert rel_err(_gpu.f64(state.h0), orc.h0) < TOL
+    assert _gpu.m2_buffer_matches(state, orc, w.H // w.G)
+
+
+def test_verify_rejects_misaligned_draft_rows():
+    w, A, D, S0, rd = _draw(1, B=2, H=16, G=2)
+    layer = _gpu.layer_for(w)
+    state = rs.ReplayState(layer)
+    rs.replayssm_init(layer, state, S0.cuda())
+    dev = _gpu.to_dev(rd)
+    x = dev["x"][0]
+    raw = torch.empty(x.numel() + 1, dtype=x.dtype, device="cuda")
+    xm = raw[1:].view(x.shape)  # starts 2 bytes past an aligned address
+    xm.copy_(x)
+    y = torch.empty(w.B, w.n_draft, w.H, w.P, device="cuda")
+    drafts = dict(x=xm, dt=dev["dt"][0], Bm=dev["Bm"][0], Cm=dev["Cm"][0], A=A.cuda(),
+                  D=D.cuda())
+    with pytest.raises(rs.ReplayError, match="aligned"):
+        rs.replayssm_verify_commit(layer, state, None, drafts, y)
+    assert state.status() == 0 and int(state.len.sum()) == 0
+
+
 def test_verify_accept_none_keeps_checkpoint_bit_exact():
     w, A, D, S0, rd = _draw(6, B=2, H=16, G=2)
     acc0 = torch.zeros_like(rd["acc"])

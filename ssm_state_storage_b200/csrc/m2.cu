@@ -426,10 +426,25 @@ __device__ __forceinline__ void store_row(float *tile, int r, int c8, const floa
   for (int s = 0; s < N / 32; ++s) st_stream(tile + (size_t)r * N + 32 * s + 4 * c8, v[s]);
 }
 
+// v <- a * v and v <- x * b + v on a float4 as two paired fp32 operations
+// (Blackwell's f32x2 pipe: per component the same rounding as fmulf / fmaf).
+__device__ __forceinline__ float4 mul4x(float a, float4 v) {
+  const float2 a2 = make_float2(a, a);
+  const float2 lo = __fmul2_rn(a2, make_float2(v.x, v.y));
+  const float2 hi = __fmul2_rn(a2, make_float2(v.z, v.w));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+__device__ __forceinline__ float4 fma4x(float x, float4 b, float4 v) {
+  const float2 x2 = make_float2(x, x);
+  const float2 lo = __ffma2_rn(x2, make_float2(b.x, b.y), make_float2(v.x, v.y));
+  const float2 hi = __ffma2_rn(x2, make_float2(b.z, b.w), make_float2(v.z, v.w));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
 // The fold of RGC register-held rows of one head:
 //   v[u] <- lam v[u] + sum_{i<k} (w_i x_i[rows[u]]) B_i[cols],
 // record loop outermost so that each B_i fragment (fp32 in shared memory) is
-// loaded once and feeds 4 * RGC * (N/32) independent FMAs.
+// loaded once and feeds 4 * RGC * (N/32) independent FMAs (issued in pairs).
 template <int P, int N, typename TI, int RGC>
 __device__ __forceinline__ void fold_rows(float4 (&v)[RGC][N / 32], float lam, int k,
                                           const float *w, const TI *x, const int (&rows)[RGC],
@@ -437,8 +452,7 @@ __device__ __forceinline__ void fold_rows(float4 (&v)[RGC][N / 32], float lam, i
 #pragma unroll
   for (int u = 0; u < RGC; ++u)
 #pragma unroll
-    for (int s = 0; s < N / 32; ++s)
-      v[u][s] = make_float4(lam * v[u][s].x, lam * v[u][s].y, lam * v[u][s].z, lam * v[u][s].w);
+    for (int s = 0; s < N / 32; ++s) v[u][s] = mul4x(lam, v[u][s]);
   for (int i = 0; i < k; ++i) {
     float4 bb[N / 32];
 #pragma unroll
@@ -449,12 +463,7 @@ __device__ __forceinline__ void fold_rows(float4 (&v)[RGC][N / 32], float lam, i
     for (int u = 0; u < RGC; ++u) {
       const float xw = wi * to_f32(x[i * P + rows[u]]);
 #pragma unroll
-      for (int s = 0; s < N / 32; ++s) {
-        v[u][s].x = fmaf(xw, bb[s].x, v[u][s].x);
-        v[u][s].y = fmaf(xw, bb[s].y, v[u][s].y);
-        v[u][s].z = fmaf(xw, bb[s].z, v[u][s].z);
-        v[u][s].w = fmaf(xw, bb[s].w, v[u][s].w);
-      }
+      for (int s = 0; s < N / 32; ++s) v[u][s] = fma4x(xw, bb[s], v[u][s]);
     }
   }
 }
@@ -761,27 +770,57 @@ __device__ __forceinline__ void decode_stager(const M2Params &p, const DecodeLay
 // tiles into a ring of NS slots, hc heads per item, waiting only for free
 // slots.  On a failed wait it marks the CTA aborted and waits (bounded) for
 // the copies it has in flight before returning.
+// Tile producer (one thread): streams the checkpoint tiles (or their read
+// copies) of this CTA's items, in item order, into the NS-slot ring.  With
+// pf > 0 it also keeps an L2 prefetch pf tiles ahead of the ring, so HBM
+// keeps streaming while the consumers spend time on per-item work that does
+// not release ring slots.
 template <int P, int N, int QM>
 __device__ __forceinline__ void stream_tiles(const M2Params &p, uint64_t *full, uint64_t *empty,
                                              unsigned char *ring, int NS, int tile_stride,
                                              int tile_bytes, int hc, volatile int *abort_flag,
-                                             int nitems, int nchunk) {
+                                             int nitems, int nchunk, int pf) {
+  auto src_of = [&](int item, int j) -> size_t {
+    int b, g, chunk, h_first;
+    item_coords(p, item, nchunk, hc, b, g, chunk, h_first);
+    return (size_t)b * p.H + h_first + j;
+  };
+  auto prefetch = [&](size_t bh) {
+    if constexpr (QM == 1) {
+      bulk_prefetch_l2(p.rc + bh * (size_t)(P * N), P * N);
+    } else if constexpr (QM == 2) {
+      bulk_prefetch_l2(p.rc + bh * (size_t)(P * N / 2), P * N / 2);
+      bulk_prefetch_l2(p.rc_scale + bh * (size_t)(P * N / 16), P * N / 16);
+    } else {
+      bulk_prefetch_l2(p.h0 + bh * (size_t)(P * N), P * N * 4);
+    }
+  };
+  int pitem = blockIdx.x, pj = 0;  // next tile to prefetch
+  auto prefetch_next = [&]() {
+    if (pitem < nitems) {
+      prefetch(src_of(pitem, pj));
+      if (++pj == hc) {
+        pj = 0;
+        pitem += gridDim.x;
+      }
+    }
+  };
+  if (pf > 0)
+    for (int k = 0; k < pf + NS; ++k) prefetch_next();
   int slot = 0;
   uint32_t sphase = 0;
   uint32_t issued = 0, parity = 0;  // per slot: a copy was issued / its phase parity
   bool failed = false;
   for (int item = blockIdx.x; item < nitems && !failed; item += gridDim.x) {
-    int b, g, chunk, h_first;
-    item_coords(p, item, nchunk, hc, b, g, chunk, h_first);
-    const size_t bh0 = (size_t)b * p.H + h_first;
     for (int j = 0; j < hc; ++j) {
+      if (pf > 0) prefetch_next();
       if (*abort_flag || !mbar_wait(&empty[slot], sphase ^ 1)) {
         failed = true;
         break;
       }
       mbar_arrive_expect_tx(&full[slot], tile_bytes);
       unsigned char *dst = ring + slot * tile_stride;
-      const size_t bh = bh0 + j;
+      const size_t bh = src_of(item, j);
       if constexpr (QM == 1) {
         bulk_g2s(dst, p.rc + bh * (size_t)(P * N), P * N, &full[slot]);
       } else if constexpr (QM == 2) {
@@ -811,7 +850,7 @@ __device__ __forceinline__ void decode_tiles(const M2Params &p, const DecodeLayo
                                              const DecodeSmemPtrs &S, volatile int *abort_flag,
                                              int nitems, int nchunk) {
   stream_tiles<P, N, QM>(p, S.full, S.empty, S.ring, lay.NS, lay.tile_stride, lay.tile_bytes,
-                         lay.hc, abort_flag, nitems, nchunk);
+                         lay.hc, abort_flag, nitems, nchunk, 0);
 }
 
 constexpr int kDecodeThreads = kThreads + 64;  // 8 consumer warps, tile producer, stager
@@ -1207,12 +1246,17 @@ __global__ void __launch_bounds__(kThreads, 2) m2_full_kernel(const M2Params p) 
 // have copied yet.
 
 constexpr int kMD = 4;  // most drafts per round
+// Consumer warps form kVGroups groups that take alternate items (with two
+// groups one group's per-item setup overlaps the other's tile streaming; on
+// B200 that measured no faster than one group of 16 warps, which is used).
+constexpr int kVGroups = 1, kGWarps = 16, kGThreads = 32 * kGWarps;
+constexpr int kVWarps = kVGroups * kGWarps, kVThreads = 32 * kVWarps;
 
 struct VerifyLayout {
   int NS, NR, hc, nchunk, cap, L, tile_bytes, tile_stride;
   int rec_floats, db_floats;  // stage floats per record buffer, scratch per item
-  int off_bars, off_recB, off_recX, off_dX, off_dB, off_dC, off_rec, off_db, off_single, off_ring,
-      total;
+  int off_bars, off_recB, off_recX, off_dX, off_dB, off_dC, off_rec, off_scr, off_ring, total;
+  int db_b, scr_b;  // per consumer group: item scratch bytes, all scratch bytes
   int recB_b, recX_b, dX_b, dBC_b;  // bytes per record buffer of each array
   __host__ static int a128(int v) { return (v + 127) & ~127; }
   __host__ static VerifyLayout make(int P, int N, int hpg, int nchunk, int cap, int L, int es,
@@ -1230,8 +1274,8 @@ struct VerifyLayout {
     d.dBC_b = a128(kMD * N * es);
     // stage: dt prefix [hc][cap] | dt drafts [4][hc] | A [hc] | D [hc] | hdr [8]
     d.rec_floats = pad4(hc * cap) + kMD * hc + pad4(hc) * 2 + 8;
-    // per item: Bf [cap][N] | wf [hc][cap] | lamf [hc] | lamd [4][hc] | Cf [4][N] | z [4][hc][P]
-    d.db_floats = cap * N + pad4(hc * cap) + pad4(hc) + kMD * hc + kMD * N + kMD * hc * P;
+    // per item: Bf [cap][N] | wf [hc][cap] | lamf [hc] | lamd [4][hc] | z [4][hc][P]
+    d.db_floats = cap * N + pad4(hc * cap) + pad4(hc) + kMD * hc + kMD * hc * P;
     for (d.NR = 2; d.NR >= 1; --d.NR) {
       int o = 0;
       d.off_bars = o;
@@ -1248,10 +1292,11 @@ struct VerifyLayout {
       o += d.NR * d.dBC_b;
       d.off_rec = o;
       o += a128(d.NR * d.rec_floats * 4);
-      d.off_db = o;  // one copy: every item starts at a barrier of all consumer warps
-      o += a128(d.db_floats * 4);
-      d.off_single = o;  // bc [4][cap+4] double | wd [4][hc][cap+4] float
-      o += a128(kMD * (cap + kMD) * 8 + kMD * hc * (cap + kMD) * 4);
+      // per consumer group: item scratch | bc [4][cap+4] double | cf [4][hc][cap+4] float
+      d.off_scr = o;
+      d.db_b = a128(d.db_floats * 4);
+      d.scr_b = d.db_b + a128(kMD * (cap + kMD) * 8 + kMD * hc * (cap + kMD) * 4);
+      o += kVGroups * d.scr_b;
       d.off_ring = o;
       d.NS = (budget - o) / d.tile_stride;
       if (d.NS > 8) d.NS = 8;
@@ -1353,36 +1398,77 @@ __device__ __forceinline__ bool verify_stage(const M2Params &p, const VerifyLayo
   return true;
 }
 
-// Butterfly reduce-scatter of four per-lane partial sums over the 8 lanes of
-// a row group (lane bits 0-2): lane c8 ends with the full sum of value
-// c8 >> 1 (lanes c8 and c8 ^ 1 hold the same sum).  4 shuffles instead of 12.
-__device__ __forceinline__ float reduce4_over8(const float (&q)[4], int c8) {
-  const bool hi = c8 & 4;
-  float a0 = hi ? q[2] : q[0], a1 = hi ? q[3] : q[1];
-  const float s0 = hi ? q[0] : q[2], s1 = hi ? q[1] : q[3];
-  a0 += __shfl_xor_sync(0xffffffffu, s0, 4);
-  a1 += __shfl_xor_sync(0xffffffffu, s1, 4);
-  const bool mid = c8 & 2;
-  float k = mid ? a1 : a0;
-  k += __shfl_xor_sync(0xffffffffu, mid ? a0 : a1, 2);
-  return k + __shfl_xor_sync(0xffffffffu, k, 1);
+// Butterfly reduce-scatter over the 16 lanes of a half warp (lane bits 3..0):
+// every lane enters with V partial sums, and after log2(16) rounds lane c16
+// holds the complete sum of value c16 / (16 / V) (V = 4, 8 or 16).  Each
+// round sends half of the remaining values, so V sums cost V - 1 + (4 -
+// log2 V) shuffles instead of 4 V.
+template <int NV, int M>
+struct HalfWarpReduce {
+  static __device__ __forceinline__ void run(float *q, int c16) {
+    if constexpr (M > 0) {
+      if constexpr (NV == 1) {
+        q[0] += __shfl_xor_sync(0xffffffffu, q[0], M);
+        HalfWarpReduce<1, M / 2>::run(q, c16);
+      } else {
+        constexpr int H = NV / 2;
+        const bool up = c16 & M;
+#pragma unroll
+        for (int k = 0; k < H; ++k) {
+          const float keep = up ? q[H + k] : q[k], send = up ? q[k] : q[H + k];
+          q[k] = keep + __shfl_xor_sync(0xffffffffu, send, M);
+        }
+        HalfWarpReduce<H, M / 2>::run(q, c16);
+      }
+    }
+  }
+};
+
+// K consecutive input elements (bf16 or fp32) from shared memory as floats;
+// the address is aligned to K elements.
+template <typename TI, int K>
+__device__ __forceinline__ void ld_vec(const TI *src, float (&out)[K]) {
+  if constexpr (std::is_same<TI, float>::value) {
+    if constexpr (K == 4) {
+      const float4 v = *reinterpret_cast<const float4 *>(src);
+      out[0] = v.x, out[1] = v.y, out[2] = v.z, out[3] = v.w;
+    } else {
+      static_assert(K == 2, "2 or 4 elements");
+      const float2 v = *reinterpret_cast<const float2 *>(src);
+      out[0] = v.x, out[1] = v.y;
+    }
+  } else {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(src);
+    if constexpr (K == 4) {
+      const uint2 u = *reinterpret_cast<const uint2 *>(src);
+      const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+      const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+      out[0] = lo.x, out[1] = lo.y, out[2] = hi.x, out[3] = hi.y;
+    } else {
+      static_assert(K == 2, "2 or 4 elements");
+      const float2 v = __bfloat1622float2(h[0]);
+      out[0] = v.x, out[1] = v.y;
+    }
+  }
 }
 
-constexpr int kVWarps = 16, kVThreads = 32 * kVWarps;  // verify consumer warps / threads
+template <typename TI>
+__device__ __forceinline__ float4 ld_vec4(const TI *src) {
+  float t[4];
+  ld_vec<TI, 4>(src, t);
+  return make_float4(t[0], t[1], t[2], t[3]);
+}
+
 
 template <int P, int N, typename TI>
 __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyLayout lay) {
-  using T = Tile<P, N>;
-  constexpr int C4 = T::C4;
-  constexpr int RW = P / kVWarps, RG = RW / 4;  // one head at a time: 16 warps x RW rows
-  static_assert(RG >= 1, "headdim must be at least 64");
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int abort_word;
   volatile int *abort_flag = &abort_word;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.off_bars);
-  uint64_t *empty = full + 8, *rfull = empty + 8, *rempty = rfull + 4;
+  uint64_t *empty = full + 8, *rfull = empty + 8, *rempty = rfull + 4, *turn = rempty + 4;
   unsigned char *ring = smem + lay.off_ring;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, rs = lane >> 3, c8 = lane & 7;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int hc = lay.hc, cap = lay.cap, nd = p.n_draft, R = cap + kMD;
   const int nitems = p.B * p.G * lay.nchunk;
   const bool own_bc = lay.nchunk == 1;
@@ -1390,12 +1476,13 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
   if (tid == 0) {
     for (int s = 0; s < 8; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kVWarps);
+      mbar_init(&empty[s], kGWarps);  // each tile is read by one group
     }
     for (int r = 0; r < 4; ++r) {
       mbar_init(&rfull[r], 1);
-      mbar_init(&rempty[r], kVWarps);
+      mbar_init(&rempty[r], kGWarps);
     }
+    for (int g2 = 0; g2 < kVGroups; ++g2) mbar_init(&turn[g2], kGWarps);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -1403,7 +1490,7 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
   if (warp == kVWarps) {
     if (lane == 0)
       stream_tiles<P, N, 0>(p, full, empty, ring, lay.NS, lay.tile_stride, lay.tile_bytes, hc,
-                            abort_flag, nitems, lay.nchunk);
+                            abort_flag, nitems, lay.nchunk, hc);
     return;
   }
   if (warp == kVWarps + 1) {
@@ -1421,10 +1508,36 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
     return;
   }
 
-  double *bc = reinterpret_cast<double *>(smem + lay.off_single);  // [4][R]
-  float *cf = reinterpret_cast<float *>(bc + kMD * R);             // [4][hc][R] coefficients
-  int it = 0;
-  for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+  // Consumer group grp takes this CTA's items it = grp, grp + 2, ...
+  // Head-loop lane layout: a half warp covers one row, lane c16 holds the
+  // columns 64 s + 4 c16 .. +3 (s < N/64); a warp owns RW = P/8 rows of
+  // every head, taken four at a time (two per half warp).
+  constexpr int S4 = N / 64, RW = P / kGWarps, NSP = RW / 4, RZ = P / 32;
+  static_assert(NSP >= 1 && S4 >= 1, "headdim and d_state must be at least 64");
+  const int grp = warp / kGWarps, gw = warp - grp * kGWarps, gtid = tid - grp * kGThreads;
+  const uint32_t gbar = 1 + grp;  // the group's named barrier
+  const int h16 = lane >> 4, c16 = lane & 15;
+  unsigned char *scr = smem + lay.off_scr + grp * lay.scr_b;
+  double *bc = reinterpret_cast<double *>(scr + lay.db_b);  // [4][R]
+  float *cf = reinterpret_cast<float *>(bc + kMD * R);     // [4][hc][R] coefficients
+  // Ring hand-off: a group starts waiting for its item's first tile only after
+  // every warp of the other group has acquired the previous item's last
+  // tile (turn[grp]), so a slot is never awaited more than one phase ahead.
+  // With a single record buffer the hand-off also precedes the record wait.
+  auto take_turn = [&](int it_) -> bool {
+    if constexpr (kVGroups == 1) return true;
+    if (it_ == 0) return true;
+    return mbar_wait(&turn[grp], ((it_ - 1) >> 1) & 1);
+  };
+  auto pass_turn = [&]() {
+    if constexpr (kVGroups > 1) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&turn[grp ^ 1]);
+    }
+  };
+  int it = grp;
+  for (int item = blockIdx.x + grp * gridDim.x; item < nitems;
+       item += kVGroups * gridDim.x, it += kVGroups) {
     const int rb = it % lay.NR;
     const uint32_t rphase = (it / lay.NR) & 1;
     int b, g, chunk, h_first;
@@ -1438,18 +1551,22 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
     const TI *dX = reinterpret_cast<const TI *>(smem + lay.off_dX + rb * lay.dX_b);
     const TI *dB = reinterpret_cast<const TI *>(smem + lay.off_dB + rb * lay.dBC_b);
     const TI *dC = reinterpret_cast<const TI *>(smem + lay.off_dC + rb * lay.dBC_b);
-    float *db = reinterpret_cast<float *>(smem + lay.off_db);
+    float *db = reinterpret_cast<float *>(scr);
     float *Bf = db, *wf = Bf + cap * N, *lamf = wf + pad4(hc * cap), *lamd = lamf + pad4(hc);
-    float *Cf = lamd + kMD * hc, *z = Cf + kMD * N;
+    float *z = lamd + kMD * hc;
 
-    const bool got = mbar_wait(&rfull[rb], rphase);
+    const bool got = (lay.NR > 1 || take_turn(it)) && mbar_wait(&rfull[rb], rphase);
     if (!got) {
       report(p.status, RSSM_ERR_TIMEOUT);
       *abort_flag = 1;
     }
-    if (bar_or(1, kVThreads, !got || *abort_flag)) break;
+    if (bar_or(gbar, kGThreads, !got || *abort_flag)) break;
     if (hdr[4]) {
-      if (tid == 0) report(p.status, RSSM_ERR_STATE);
+      if (gtid == 0) report(p.status, RSSM_ERR_STATE);
+      if (lay.NR > 1 && !take_turn(it)) {
+        report(p.status, RSSM_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
       for (int j = 0; j < hc; ++j) {
         const uint32_t pos = (uint32_t)it * hc + j;
         if (!mbar_wait(&full[pos % lay.NS], (pos / lay.NS) & 1)) {
@@ -1459,6 +1576,7 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[pos % lay.NS]);
       }
+      pass_turn();
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&rempty[rb]);
@@ -1467,54 +1585,76 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
     const int n1 = hdr[1], nb = hdr[3], K = nb + nd;
     const bool fold = hdr[2];
 
-    // ---- S1: append the drafts; fp32 copies; B_i . C_d in fp64
-    for (int e = tid; e < nd * hc * P; e += kVThreads) {
-      const int d = e / (hc * P), rem = e - d * (hc * P), j = rem / P, q = rem - j * P;
-      static_cast<TI *>(p.xbuf)[((bh0 + j) * cap + nb + d) * P + q] = dX[(d * hc + j) * P + q];
-    }
-    for (int e = tid; e < nd * N; e += kVThreads) {
-      const int d = e / N, c = e - d * N;
-      if (own_bc) {
-        static_cast<TI *>(p.Bbuf)[(bg * cap + nb + d) * N + c] = dB[d * N + c];
-        static_cast<TI *>(p.Cbuf)[(bg * cap + nb + d) * N + c] = dC[d * N + c];
-      }
-      Cf[d * N + c] = to_f32(dC[d * N + c]);
-    }
-    if (tid < nd * hc) {
-      const int d = tid / hc, j = tid - (tid / hc) * hc;
-      p.dtbuf[(bh0 + j) * cap + nb + d] = dtd[d * hc + j];
-    }
-    if (fold)
-      for (int e = tid; e < n1 * N; e += kVThreads) Bf[e] = to_f32(recB[e]);
+    // ---- S1: append the drafts (16-byte chunks); fp32 B for the fold;
+    // B_i . C_d in fp64
     {
+      constexpr int XC = P * (int)sizeof(TI) / 16, BC = N * (int)sizeof(TI) / 16;
+      for (int c = gtid; c < nd * hc * XC; c += kGThreads) {
+        const int row = c / XC, k = c - row * XC, d = row / hc, j = row - d * hc;
+        reinterpret_cast<uint4 *>(static_cast<TI *>(p.xbuf) + ((bh0 + j) * cap + nb + d) * P)[k] =
+            reinterpret_cast<const uint4 *>(dX + (size_t)row * P)[k];
+      }
+      if (own_bc)
+        for (int c = gtid; c < 2 * nd * BC; c += kGThreads) {
+          const int which = c / (nd * BC), cc = c - which * (nd * BC), d = cc / BC, k = cc - d * BC;
+          TI *dst = static_cast<TI *>(which ? p.Cbuf : p.Bbuf) + (bg * cap + nb + d) * N;
+          reinterpret_cast<uint4 *>(dst)[k] =
+              reinterpret_cast<const uint4 *>((which ? dC : dB) + (size_t)d * N)[k];
+        }
+      if (gtid < nd * hc) {
+        const int d = gtid / hc, j = gtid - (gtid / hc) * hc;
+        p.dtbuf[(bh0 + j) * cap + nb + d] = dtd[d * hc + j];
+      }
+      if (fold)
+        for (int e = gtid; e < n1 * (N / 4); e += kGThreads)
+          reinterpret_cast<float4 *>(Bf)[e] = ld_vec4<TI>(recB + 4 * e);
       const int npair = nd * K;  // (d, i) with i <= nb + d are used
       constexpr int PER = N / 16;
-      for (int base = 0; base < npair; base += kVThreads / 16) {
-        const int pr = base + (tid >> 4), c0 = (tid & 15) * PER;
+      for (int base = 0; base < npair; base += kGThreads / 16) {
+        const int pr = base + (gtid >> 4), c0 = (gtid & 15) * PER;
         const int d = pr / K, i = pr - d * K;
         const bool use = pr < npair && i <= nb + d;
         double acc = 0.0;
         if (use) {
           const TI *Bi = i < nb ? recB + i * N : dB + (i - nb) * N;
 #pragma unroll
-          for (int e = 0; e < PER; ++e)
-            acc = fma((double)to_f32(Bi[c0 + e]), (double)to_f32(dC[d * N + c0 + e]), acc);
+          for (int e = 0; e < PER; e += 4) {
+            const float4 bv = ld_vec4<TI>(Bi + c0 + e), cv = ld_vec4<TI>(dC + d * N + c0 + e);
+            acc = fma((double)bv.x, (double)cv.x, acc);
+            acc = fma((double)bv.y, (double)cv.y, acc);
+            acc = fma((double)bv.z, (double)cv.z, acc);
+            acc = fma((double)bv.w, (double)cv.w, acc);
+          }
         }
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
         acc += __shfl_xor_sync(0xffffffffu, acc, 4);
         acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-        if (use && (tid & 15) == 0) bc[d * R + i] = acc;
+        if (use && (gtid & 15) == 0) bc[d * R + i] = acc;
       }
     }
-    bar_sync(1, kVThreads);
+    // draft C rows for this lane's columns, in registers for the whole item
+    float4 cr[kMD][S4];
+#pragma unroll
+    for (int d = 0; d < kMD; ++d)
+#pragma unroll
+      for (int s4 = 0; s4 < S4; ++s4) cr[d][s4] = ld_vec4<TI>(dC + d * N + 64 * s4 + 4 * c16);
+    bar_sync(gbar, kGThreads);
 
     // ---- S2 (one warp per head): decay weights from fp64 suffix sums.
     // Draft sequence: the nb committed records, then the nd drafts; with
-    // S_l = sum_{m >= l} dt_m, draft d (records 0..nb+d) weighs record i by
-    // exp(A (S_{i+1} - S_{nb+d+1})) dt_i.  The fold sequence is the n1
-    // committed records.  Both scans run together.
-    for (int j = warp; j < hc; j += kVWarps) {
+    // S_l = sum_{m >= l} dt_m, draft d (records 0..e, e = nb + d) weighs
+    // record i by exp(A (S_{i+1} - S_{e+1})) dt_i and the checkpoint by
+    // exp(A (S_0 - S_{e+1})).  Both factor through the reference point
+    // S_ref = S_{nb+1}:  exp(A (S_{i+1} - S_ref)) * exp(A (S_ref - S_{e+1})),
+    // so one exponential per lane serves every draft: lanes 0..K-1 take
+    // E_l = exp(A (S_{l+1} - S_ref)), lanes 27..30 take F_d = exp(A (S_ref -
+    // S_{e+1})) and lane 31 takes G = exp(A (S_0 - S_ref)).  No factor can
+    // overflow: S_ref - S_{e+1} and the S_{i+1} - S_ref of draft records span
+    // at most 4 dt, and every other argument is <= 0.  The fold sequence is
+    // the n1 committed records (weights exp(A S'_{l+1}) dt_l, decay
+    // exp(A S'_0)); both scans and both exponentials run side by side.
+    for (int j = gw; j < hc; j += kGWarps) {
       const double A = As[j];
       const double dts = lane < nb ? (double)dtb[j * cap + lane]
                                    : (lane < K ? (double)dtd[(lane - nb) * hc + j] : 0.0);
@@ -1529,43 +1669,65 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
           Sf += tf;
         }
       }
-      const double Ss1 = __shfl_down_sync(0xffffffffu, Ss, 1);  // S_{l+1} (lane 31: unused)
+      const double Ss1 = __shfl_down_sync(0xffffffffu, Ss, 1);  // S_{l+1}; lanes >= K: 0
       const double Sf1 = __shfl_down_sync(0xffffffffu, Sf, 1);
-      const double Ss0 = __shfl_sync(0xffffffffu, Ss, 0);
-      double Se[kMD];
-#pragma unroll
-      for (int d = 0; d < kMD; ++d) Se[d] = __shfl_sync(0xffffffffu, Ss, (nb + d + 1) & 31);
+      const double Sref = __shfl_sync(0xffffffffu, Ss, nb + 1);  // nb + 1 <= cap < 27
+      const double S0 = __shfl_sync(0xffffffffu, Ss, 0);
+      const double Sf0 = __shfl_sync(0xffffffffu, Sf, 0);
+      const double SeL = __shfl_sync(0xffffffffu, Ss, (nb + (lane - 27) + 1) & 31);  // lanes 27..30
+      double arg = 0.0;
+      if (lane < K) arg = A * (Ss1 - Sref);
+      else if (lane >= 27 && lane < 31) arg = lane - 27 < nd ? A * (Sref - SeL) : 0.0;
+      else if (lane == 31) arg = A * (S0 - Sref);
+      const double ex = exp(arg);
+      const double exf = exp(A * (lane + 1 < n1 ? Sf1 : (lane == 31 ? Sf0 : 0.0)));  // n1 <= 20
       if (fold) {
-        if (lane < n1) wf[j * cap + lane] = (float)(exp(A * (lane + 1 < n1 ? Sf1 : 0.0)) * dtf);
-        if (lane == 0) lamf[j] = (float)exp(A * Sf);
+        if (lane < n1) wf[j * cap + lane] = (float)(exf * dtf);
+        if (lane == 31) lamf[j] = (float)exf;
       }
+      const double G = __shfl_sync(0xffffffffu, ex, 31);
 #pragma unroll
       for (int d = 0; d < kMD; ++d) {
+        const double F = __shfl_sync(0xffffffffu, ex, 27 + d);
         if (d < nd) {
-          const int e = nb + d;  // last record of draft d
-          const double se = e + 1 < K ? Se[d] : 0.0;
-          if (lane <= e)
-            cf[(d * hc + j) * R + lane] =
-                (float)(exp(A * ((lane < e ? Ss1 : se) - se)) * dts * bc[d * R + lane]);
-          if (lane == 0) lamd[d * hc + j] = (float)exp(A * (Ss0 - se));
+          if (lane <= nb + d) cf[(d * hc + j) * R + lane] = (float)(ex * F * dts * bc[d * R + lane]);
+          if (lane == 0) lamd[d * hc + j] = (float)(G * F);
         }
       }
     }
-    bar_sync(1, kVThreads);
-    // ---- S3: z[d][j][r] = sum_i cf[d][j][i] x_i[r] + D_j x_d[r]
-    for (int e = tid; e < nd * hc * P; e += kVThreads) {
-      const int d = e / (hc * P), rem = e - d * (hc * P), j = rem / P, r = rem - j * P;
+    bar_sync(gbar, kGThreads);
+    // ---- S3 (one warp per (draft, head) row, RZ rows of the head per lane):
+    // z[d][j][r] = sum_i cf[d][j][i] x_i[r] + D_j x_d[r]
+    for (int row = gw; row < nd * hc; row += kGWarps) {
+      const int d = row / hc, j = row - d * hc;
       const float *c = cf + (d * hc + j) * R;
-      float acc = 0.f;
-      int i = 0;
-      for (; i < nb; ++i) acc = fmaf(c[i], to_f32(recX[(j * cap + i) * P + r]), acc);
-      for (; i <= nb + d; ++i) acc = fmaf(c[i], to_f32(dX[((i - nb) * hc + j) * P + r]), acc);
-      z[e] = fmaf(Ds[j], to_f32(dX[(d * hc + j) * P + r]), acc);
+      float acc[RZ], xv[RZ];
+#pragma unroll
+      for (int k = 0; k < RZ; ++k) acc[k] = 0.f;
+      for (int i = 0; i < nb; ++i) {
+        ld_vec<TI, RZ>(recX + (j * cap + i) * P + RZ * lane, xv);
+        const float ci = c[i];
+#pragma unroll
+        for (int k = 0; k < RZ; ++k) acc[k] = fmaf(ci, xv[k], acc[k]);
+      }
+      for (int i = nb; i <= nb + d; ++i) {
+        ld_vec<TI, RZ>(dX + ((i - nb) * hc + j) * P + RZ * lane, xv);
+        const float ci = c[i];
+#pragma unroll
+        for (int k = 0; k < RZ; ++k) acc[k] = fmaf(ci, xv[k], acc[k]);
+      }
+      ld_vec<TI, RZ>(dX + (d * hc + j) * P + RZ * lane, xv);
+      const float Dj = Ds[j];
+#pragma unroll
+      for (int k = 0; k < RZ; ++k) z[(d * hc + j) * P + RZ * lane + k] = fmaf(Dj, xv[k], acc[k]);
     }
-    bar_sync(1, kVThreads);
+    bar_sync(gbar, kGThreads);
 
     // ---- heads, one at a time: rows into registers, optional fold, outputs
-    const int dmine = c8 >> 1;  // the draft whose sum this lane ends with
+    if (lay.NR > 1 && !take_turn(it)) {
+      report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
     for (int j = 0; j < hc; ++j) {
       const int h = h_first + j;
       const size_t bh = bh0 + j;
@@ -1575,45 +1737,78 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
         report(p.status, RSSM_ERR_TIMEOUT);
         *abort_flag = 1;
       }
-      float4 v[RG][C4];
-      int rows[RG];
+      if (j == hc - 1) pass_turn();
+      const float *tl = reinterpret_cast<const float *>(ring + sl * lay.tile_stride);
+      const float lf = fold ? lamf[j] : 0.f;
 #pragma unroll
-      for (int u = 0; u < RG; ++u) {
-        rows[u] = warp * RW + 4 * u + rs;
-        view_row<P, N, 0>(ring + sl * lay.tile_stride, rows[u], c8, 1.0f, v[u]);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[sl]);
-      if (fold) {
-        fold_rows<P, N, TI, RG>(v, lamf[j], n1, wf + j * cap, recX + j * cap * P, rows, Bf, c8);
-        float *tile = p.h0 + bh * (size_t)(P * N);
+      for (int sp = 0; sp < NSP; ++sp) {
+        int rows[2];
+        float4 v[2][S4];
 #pragma unroll
-        for (int u = 0; u < RG; ++u) store_row<N>(tile, rows[u], c8, v[u]);
-      }
-      float q[RG][kMD];
+        for (int u = 0; u < 2; ++u) {
+          rows[u] = gw * RW + 4 * sp + 2 * u + h16;
 #pragma unroll
-      for (int d = 0; d < kMD; ++d) {
-        float4 cd[C4];
+          for (int s4 = 0; s4 < S4; ++s4)
+            v[u][s4] = *reinterpret_cast<const float4 *>(tl + rows[u] * N + 64 * s4 + 4 * c16);
+        }
+        if (sp == NSP - 1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[sl]);
+        }
+        if (fold) {  // v <- lam v + sum_i (w_i x_i[row]) B_i[cols], written back once
 #pragma unroll
-        for (int s = 0; s < C4; ++s) cd[s] = *reinterpret_cast<const float4 *>(&Cf[d * N + T::col(c8, s)]);
+          for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int u = 0; u < RG; ++u) q[u][d] = tree_dot<C4>(v[u], cd);
-      }
-      float a[RG];
+            for (int s4 = 0; s4 < S4; ++s4) v[u][s4] = mul4x(lf, v[u][s4]);
+          const float *wj = wf + j * cap;
+          const TI *xj = recX + j * cap * P;
+          for (int i = 0; i < n1; ++i) {
+            float4 bb[S4];
 #pragma unroll
-      for (int u = 0; u < RG; ++u) a[u] = reduce4_over8(q[u], c8);  // every lane shuffles
-      if (dmine < nd && (c8 & 1) == 0) {
-        const float ld = lamd[dmine * hc + j];
-        const float *zd = z + (dmine * hc + j) * P;
-        float *yd = p.y + b * p.bs_y + ((size_t)dmine * p.H + h) * P;
+            for (int s4 = 0; s4 < S4; ++s4)
+              bb[s4] = *reinterpret_cast<const float4 *>(&Bf[i * N + 64 * s4 + 4 * c16]);
+            const float wi = wj[i];
 #pragma unroll
-        for (int u = 0; u < RG; ++u) yd[rows[u]] = fmaf(ld, a[u], zd[rows[u]]);
+            for (int u = 0; u < 2; ++u) {
+              const float xw = wi * to_f32(xj[i * P + rows[u]]);
+#pragma unroll
+              for (int s4 = 0; s4 < S4; ++s4) v[u][s4] = fma4x(xw, bb[s4], v[u][s4]);
+            }
+          }
+          float *tile = p.h0 + bh * (size_t)(P * N);
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int s4 = 0; s4 < S4; ++s4)
+              st_stream(tile + (size_t)rows[u] * N + 64 * s4 + 4 * c16, v[u][s4]);
+        }
+        float q[2 * kMD];  // paired fp32 FMAs over this lane's 4 S4 columns
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int d = 0; d < kMD; ++d) {
+            float2 a = __fmul2_rn(make_float2(v[u][0].x, v[u][0].y), make_float2(cr[d][0].x, cr[d][0].y));
+            a = __ffma2_rn(make_float2(v[u][0].z, v[u][0].w), make_float2(cr[d][0].z, cr[d][0].w), a);
+#pragma unroll
+            for (int s4 = 1; s4 < S4; ++s4) {
+              a = __ffma2_rn(make_float2(v[u][s4].x, v[u][s4].y), make_float2(cr[d][s4].x, cr[d][s4].y), a);
+              a = __ffma2_rn(make_float2(v[u][s4].z, v[u][s4].w), make_float2(cr[d][s4].z, cr[d][s4].w), a);
+            }
+            q[u * kMD + d] = a.x + a.y;
+          }
+        HalfWarpReduce<2 * kMD, 8>::run(q, c16);  // every lane shuffles
+        const int idx = c16 >> 1, u = idx / kMD, d = idx - u * kMD;
+        if ((c16 & 1) == 0 && d < nd) {
+          const int r = rows[u];
+          p.y[b * p.bs_y + ((size_t)d * p.H + h) * P + r] =
+              fmaf(lamd[d * hc + j], q[0], z[(d * hc + j) * P + r]);
+        }
       }
     }
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&rempty[rb]);
-    if (tid < hc) p.len[bh0 + tid] = nb;
+    if (gtid < hc) p.len[bh0 + gtid] = nb;
   }
 }
 

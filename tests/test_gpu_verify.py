@@ -79,6 +79,23 @@ def test_verify_shapes_match_oracle(P, N, dtype, H, G):
     assert _gpu.m2_buffer_matches(state, orc, w.H // w.G)
 
 
+def test_verify_full_batch_sampled():
+    """m2_verify at its full batch of 512 (the benchmark's launch shape: many
+    items per CTA, both consumer groups busy) over 12 rounds; the oracle checks
+    4 sequences, all 128 heads."""
+    w, A, D, S0, rd = _draw(12)
+    layer, state, y, lens = _gpu_rounds(w, A, D, S0, rd)
+    assert state.status() == 0
+    seqs = [0, 203, 257, 511]
+    orc = oracle.M2Replay(S0[seqs], G=w.G, L=w.L, cap=w.L + w.n_draft - 1)
+    sub = {k: v[:, seqs] for k, v in rd.items()}
+    yo, lt = orc.verify(sub["x"], sub["dt"], sub["Bm"], sub["Cm"], A, D, sub["acc"])
+    ys = y[:, seqs]
+    assert np.array_equal(lens[1:][:, seqs], lt)
+    assert per_step_rel_err(ys.reshape(-1, *ys.shape[3:]), yo.reshape(-1, *yo.shape[3:])) < TOL
+    assert rel_err(_gpu.f64(state.h0[seqs]), orc.h0) < TOL
+
+
 def test_verify_rejects_misaligned_draft_rows():
     w, A, D, S0, rd = _draw(1, B=2, H=16, G=2)
     layer = _gpu.layer_for(w)

@@ -55,6 +55,39 @@ def parse():
     return ap.parse_args()
 
 
+# Sources of m2_decode_kernel: a DRAM-traffic figure recorded under profiles/
+# applies only while their content hash matches the one recorded with it.
+DECODE_SOURCES = ("m2.cu", "m2_device.cuh", "common.cuh", "pipeline.cuh", "codec.cuh",
+                  "internal.h")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "m2_decode_kernel_m2_serving_traffic.txt")
+
+
+def decode_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "ssm_state_storage_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(batch):
+    """DRAM bytes (read + write) per decode launch at batch 256 from the
+    committed ncu summary, or None when absent, for another batch, or taken on
+    different kernel sources."""
+    if batch != 256 or not os.path.exists(TRAFFIC_FILE):
+        return None
+    kv = {}
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 2 and not line.startswith("#"):
+                kv[parts[0]] = parts[1]
+    if kv.get("source_sha256") != decode_sources_sha256():
+        return None
+    return float(kv["traffic_bytes_per_launch"])
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -283,7 +316,8 @@ def run_ours(args, rank, world):
                    "step": "one 16-token window = 15 non-flush + 1 flush decode steps",
                    "l2": "inputs larger than L2 (1 GiB checkpoint streamed every step)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "kernel": "m2_decode_kernel",
+                     "frac": achieved / peak, "traffic": recorded_traffic(w.B),
+                     "kernel": "m2_decode_kernel",
                      "peak_source": peak_src,
                      "algorithmic_bytes_per_launch": win_bytes / L},
         "full_state": {"value": value_full, "unit": "tokens/s", "ms_per_step": ms_per_window_full,

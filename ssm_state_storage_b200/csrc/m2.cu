@@ -1,6 +1,7 @@
 // m2.cu -- Mamba-2 decode kernels for sm_100a: replay decode step with fused
-// flush fold, standalone fold (flush / commit / materialise), conventional
-// full-state step, and speculative verify with fused commit.
+// flush fold, standalone fold (flush / commit / materialise) and the
+// conventional full-state step.  The speculative verify round is in
+// m2_verify.cu; helpers shared by both are in m2_device.cuh.
 //
 // Method: every (sequence, head) keeps a checkpoint h0 and a buffer of the
 // latest input records; a non-flush step appends the current record and
@@ -24,502 +25,10 @@
 // registers with 128-bit loads: lane (rs = lane/8, c8 = lane%8) of warp w holds
 // rows w*P/8 + rs + 4*rho and columns 32*s + 4*c8, so each quarter-warp reads
 // one 128-byte line and the row sums need only 3 shuffle levels.
-#include <type_traits>
-
-#include "codec.cuh"
-#include "common.cuh"
-#include "internal.h"
-#include "pipeline.cuh"
+#include "m2_device.cuh"
 
 namespace rssm {
 namespace {
-
-__device__ __forceinline__ float sum8(float v) {  // over the 8 lanes of a quarter-warp
-  v += __shfl_xor_sync(0xffffffffu, v, 1);
-  v += __shfl_xor_sync(0xffffffffu, v, 2);
-  v += __shfl_xor_sync(0xffffffffu, v, 4);
-  return v;
-}
-
-// Dot product of C4 float4 pairs summed as a balanced tree.
-template <int C4>
-__device__ __forceinline__ float tree_dot(const float4 (&a)[C4], const float4 (&b)[C4]) {
-  float d[C4];
-#pragma unroll
-  for (int s = 0; s < C4; ++s) d[s] = (a[s].x * b[s].x + a[s].y * b[s].y) + (a[s].z * b[s].z + a[s].w * b[s].w);
-#pragma unroll
-  for (int w = 1; w < C4; w <<= 1)
-#pragma unroll
-    for (int s = 0; s + w < C4; s += 2 * w) d[s] += d[s + w];
-  return d[0];
-}
-
-template <int P, int N>
-struct Tile {
-  static constexpr int RPT = P / 32;  // rows per thread
-  static constexpr int C4 = N / 32;   // float4 column segments per thread
-  static __device__ __forceinline__ int row(int warp, int rs, int rho) {
-    return warp * (P / 8) + rs + 4 * rho;
-  }
-  static __device__ __forceinline__ int col(int c8, int s) { return 32 * s + 4 * c8; }
-};
-
-// ---------------------------------------------------------------- read copy
-
-// Load the read view of a head tile from its low-precision copy.
-template <int P, int N, int QM>
-__device__ __forceinline__ void load_read_view(const M2Params &p, size_t bh, int warp, int rs,
-                                               int c8, float4 (&v)[P / 32][N / 32]) {
-  using T = Tile<P, N>;
-  if constexpr (QM == 1) {
-    const uint8_t *rc = p.rc + bh * (size_t)(P * N);
-#pragma unroll
-    for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-      for (int s = 0; s < T::C4; ++s) {
-        const int r = T::row(warp, rs, rho), c = T::col(c8, s);
-        const uint32_t w = *reinterpret_cast<const uint32_t *>(rc + (size_t)r * N + c);
-        v[rho][s] = make_float4(e4m3_decode(w & 0xFF), e4m3_decode((w >> 8) & 0xFF),
-                                e4m3_decode((w >> 16) & 0xFF), e4m3_decode(w >> 24));
-      }
-  } else {
-    const uint8_t *rc = p.rc + bh * (size_t)(P * N / 2);
-    const uint8_t *sc = p.rc_scale + bh * (size_t)(P * N / 16);
-    const float sg = p.rc_gscale[bh];
-#pragma unroll
-    for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-      for (int s = 0; s < T::C4; ++s) {
-        const int r = T::row(warp, rs, rho), c = T::col(c8, s);
-        const uint32_t w = *reinterpret_cast<const uint16_t *>(rc + (size_t)r * (N / 2) + c / 2);
-        const float sb = e4m3_decode(sc[(size_t)r * (N / 16) + c / 16]);
-        v[rho][s] = make_float4(nvfp4_value(w & 0xF, sb, sg), nvfp4_value((w >> 4) & 0xF, sb, sg),
-                                nvfp4_value((w >> 8) & 0xF, sb, sg),
-                                nvfp4_value((w >> 12) & 0xF, sb, sg));
-      }
-  }
-}
-
-// Quantise a register tile after a fold.  fmt 1 = FP8, 2 = NVFP4.  With
-// roundtrip the values are replaced by deq(Q(v)) (quantised checkpoint);
-// otherwise the codes are written to the read copy.  Must be called by every
-// thread of the CTA (NVFP4 needs the tile maximum).
-template <int P, int N>
-__device__ __forceinline__ void quantize_tile(const M2Params &p, size_t bh, int fmt, bool roundtrip,
-                                              float4 (&v)[P / 32][N / 32], float *s_red, int warp,
-                                              int lane, int rs, int c8, int bar_threads = 0) {
-  using T = Tile<P, N>;
-  if (fmt == 1) {
-    uint8_t *rc = p.rc + bh * (size_t)(P * N);
-#pragma unroll
-    for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-      for (int s = 0; s < T::C4; ++s) {
-        const int r = T::row(warp, rs, rho), c = T::col(c8, s);
-        float4 &a = v[rho][s];
-        const uint32_t b0 = e4m3_encode(a.x), b1 = e4m3_encode(a.y), b2 = e4m3_encode(a.z),
-                       b3 = e4m3_encode(a.w);
-        if (roundtrip) {
-          a = make_float4(e4m3_decode(b0), e4m3_decode(b1), e4m3_decode(b2), e4m3_decode(b3));
-        } else {
-          *reinterpret_cast<uint32_t *>(rc + (size_t)r * N + c) = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-        }
-      }
-    return;
-  }
-  // NVFP4: tile maximum first
-  float m = 0.f;
-#pragma unroll
-  for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s) {
-      const float4 a = v[rho][s];
-      m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
-    }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) s_red[warp] = m;
-  if (bar_threads) bar_sync(2, bar_threads);  // the consumer warps only
-  else __syncthreads();
-  float amax = s_red[0];
-#pragma unroll
-  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, s_red[w]);
-  const float sg = nvfp4_tile_scale(amax);
-  uint8_t *rc = p.rc + bh * (size_t)(P * N / 2);
-  uint8_t *sc = p.rc_scale + bh * (size_t)(P * N / 16);
-#pragma unroll
-  for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s) {
-      const int r = T::row(warp, rs, rho), c = T::col(c8, s);
-      float4 &a = v[rho][s];
-      float bm = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-      const uint32_t scode = nvfp4_block_code(bm, sg);
-      const float d = nvfp4_step(scode, sg);
-      const uint32_t lo = nvfp4_pack2(a.x, a.y, d), hi = nvfp4_pack2(a.z, a.w, d);
-      if (roundtrip) {
-        const float sb = e4m3_decode(scode);
-        a = make_float4(nvfp4_value(lo & 0xF, sb, sg), nvfp4_value(lo >> 4, sb, sg),
-                        nvfp4_value(hi & 0xF, sb, sg), nvfp4_value(hi >> 4, sb, sg));
-      } else {
-        *reinterpret_cast<uint16_t *>(rc + (size_t)r * (N / 2) + c / 2) = (uint16_t)(lo | (hi << 8));
-        if ((c8 & 3) == 0) sc[(size_t)r * (N / 16) + c / 16] = (uint8_t)scode;
-      }
-    }
-  if (!roundtrip && warp == 0 && lane == 0) p.rc_gscale[bh] = sg;
-}
-
-template <int P, int N>
-__device__ __forceinline__ void load_tile(const float *tile, int warp, int rs, int c8,
-                                          float4 (&v)[P / 32][N / 32]) {
-  using T = Tile<P, N>;
-#pragma unroll
-  for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s)
-      v[rho][s] = ld_stream(tile + (size_t)T::row(warp, rs, rho) * N + T::col(c8, s));
-}
-
-template <int P, int N>
-__device__ __forceinline__ void store_tile(float *tile, int warp, int rs, int c8,
-                                           const float4 (&v)[P / 32][N / 32]) {
-  using T = Tile<P, N>;
-#pragma unroll
-  for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s)
-      st_stream(tile + (size_t)T::row(warp, rs, rho) * N + T::col(c8, s), v[rho][s]);
-}
-
-// Decay weights of k records for one head, by one warp (lane i owns record i):
-//   wdt[i] = exp(A * sum_{i<m<k} dt_m) * dt_i,   *lam = exp(A * sum_{m<k} dt_m).
-// The suffix sums come from a shuffle scan (fixed association order, so the
-// result does not depend on timing); every dt term is non-negative, so no
-// cancellation occurs.  Sums, products and exponentials are taken in fp64 (a
-// handful per head; B200 runs fp64 at half the fp32 rate): an fp32 exp(A s)
-// would carry a relative error of about |A s| * 2^-24 into every weight.
-__device__ __forceinline__ void decay_weights_scan(const float *dt, int k, float A, float *wdt,
-                                                   float *lam, int lane) {
-  const double mine = lane < k ? (double)dt[lane] : 0.0;
-  double s = lane + 1 < k ? (double)dt[lane + 1] : 0.0;  // suffix of the records after this one
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double t = __shfl_down_sync(0xffffffffu, s, o);
-    if (lane + o < 32) s += t;
-  }
-  const double a = A;
-  if (lane < k) wdt[lane] = (float)(exp(a * s) * mine);
-  if (lane == 0) *lam = (float)exp(a * (s + mine));
-}
-
-__device__ __forceinline__ void decay_weights(const float *dt, int k, float A, float *wdt,
-                                              float *lam, int lane) {
-  const double a = A;
-  if (lane < k) {
-    double s = 0.0;
-    for (int m = lane + 1; m < k; ++m) s += dt[m];
-    wdt[lane] = (float)(exp(a * s) * (double)dt[lane]);
-  }
-  if (lane == 0) {
-    double t = 0.0;
-    for (int m = 0; m < k; ++m) t += dt[m];
-    *lam = (float)exp(a * t);
-  }
-}
-
-// h <- lam * h + sum_{i<k} (wdt_i x_i[r]) B_i[cols]  -- the fold, in registers.
-// x: the head's records [k][P] (input dtype); B: the group's records [k][N] fp32.
-template <typename TB>
-__device__ __forceinline__ float4 ld4_smem(const TB *p) {
-  if constexpr (sizeof(TB) == 4) {
-    return *reinterpret_cast<const float4 *>(p);
-  } else {
-    const uint2 raw = *reinterpret_cast<const uint2 *>(p);
-    const TB *e = reinterpret_cast<const TB *>(&raw);
-    return make_float4(to_f32(e[0]), to_f32(e[1]), to_f32(e[2]), to_f32(e[3]));
-  }
-}
-
-template <int P, int N, typename TI, typename TB = float>
-__device__ __forceinline__ void fold_regs(float4 (&hv)[P / 32][N / 32], float lam, int k,
-                                          const float *wdt, const TI *x, const TB *Bs,
-                                          int warp, int rs, int c8) {
-  using T = Tile<P, N>;
-#pragma unroll
-  for (int rho = 0; rho < T::RPT; ++rho) {
-    const int r = T::row(warp, rs, rho);
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s) {
-      hv[rho][s].x *= lam;
-      hv[rho][s].y *= lam;
-      hv[rho][s].z *= lam;
-      hv[rho][s].w *= lam;
-    }
-    for (int i = 0; i < k; ++i) {
-      const float xw = wdt[i] * to_f32(x[i * P + r]);
-#pragma unroll
-      for (int s = 0; s < T::C4; ++s) {
-        const float4 bb = ld4_smem<TB>(&Bs[i * N + T::col(c8, s)]);
-        hv[rho][s].x = fmaf(xw, bb.x, hv[rho][s].x);
-        hv[rho][s].y = fmaf(xw, bb.y, hv[rho][s].y);
-        hv[rho][s].z = fmaf(xw, bb.z, hv[rho][s].z);
-        hv[rho][s].w = fmaf(xw, bb.w, hv[rho][s].w);
-      }
-    }
-  }
-}
-
-// The fold with the record loop outermost: each B_i fragment (fp32 in shared
-// memory) is loaded once and used for all of the thread's rows.
-template <int P, int N, typename TI>
-__device__ __forceinline__ void fold_regs_hoisted(float4 (&hv)[P / 32][N / 32], float lam, int k,
-                                                  const float *wdt, const TI *x, const float *Bf,
-                                                  int warp, int rs, int c8) {
-  using T = Tile<P, N>;
-#pragma unroll
-  for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s) {
-      hv[rho][s].x *= lam;
-      hv[rho][s].y *= lam;
-      hv[rho][s].z *= lam;
-      hv[rho][s].w *= lam;
-    }
-  // two accumulation chains (even / odd records): shorter rounding chains and
-  // independent FMA streams
-  float4 acc[T::RPT][T::C4];
-#pragma unroll
-  for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s) acc[rho][s] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i = 0; i < k; ++i) {
-    float4 bb[T::C4];
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s)
-      bb[s] = *reinterpret_cast<const float4 *>(&Bf[i * N + T::col(c8, s)]);
-    const float w = wdt[i];
-    const bool odd = i & 1;
-#pragma unroll
-    for (int rho = 0; rho < T::RPT; ++rho) {
-      const float xw = w * to_f32(x[i * P + T::row(warp, rs, rho)]);
-#pragma unroll
-      for (int s = 0; s < T::C4; ++s) {
-        float4 &d = odd ? acc[rho][s] : hv[rho][s];
-        d.x = fmaf(xw, bb[s].x, d.x);
-        d.y = fmaf(xw, bb[s].y, d.y);
-        d.z = fmaf(xw, bb[s].z, d.z);
-        d.w = fmaf(xw, bb[s].w, d.w);
-      }
-    }
-  }
-#pragma unroll
-  for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s) {
-      hv[rho][s].x += acc[rho][s].x;
-      hv[rho][s].y += acc[rho][s].y;
-      hv[rho][s].z += acc[rho][s].z;
-      hv[rho][s].w += acc[rho][s].w;
-    }
-}
-
-// After a fold: round the checkpoint (qmode 3/4), store it, refresh the read
-// copy (qmode 1/2).  NVFP4 variants synchronise the CTA.
-template <int P, int N, int QM>
-__device__ __forceinline__ void commit_checkpoint(const M2Params &p, size_t bh, float *dst,
-                                                  float4 (&hv)[P / 32][N / 32], float *s_red,
-                                                  int warp, int lane, int rs, int c8,
-                                                  int bar_threads = 0) {
-  if constexpr (QM >= 3)
-    quantize_tile<P, N>(p, bh, QM - 2, true, hv, s_red, warp, lane, rs, c8, bar_threads);
-  store_tile<P, N>(dst, warp, rs, c8, hv);
-  if constexpr (QM == 1 || QM == 2)
-    quantize_tile<P, N>(p, bh, QM, false, hv, s_red, warp, lane, rs, c8, bar_threads);
-}
-
-// Heads handled by one CTA: the whole group when it has at most 8 heads,
-// otherwise chunks of 8 (the host requires H/G <= 8 or a multiple of 8).
-__host__ __device__ __forceinline__ int head_chunk(int hpg) { return hpg <= 8 ? hpg : 8; }
-
-// Copy `count` elements of T from global to shared memory as fp32, 16 bytes
-// per load (both ends 16-byte aligned, count a multiple of 16 / sizeof(T)).
-template <typename T>
-__device__ __forceinline__ void stage_f32(float *dst, const T *src, int count, int tid) {
-  constexpr int V = 16 / sizeof(T);
-  const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
-  for (int v = tid; v < count / V; v += kThreads) {
-    const uint4 raw = s4[v];
-    const T *e = reinterpret_cast<const T *>(&raw);
-#pragma unroll
-    for (int j = 0; j < V; ++j) dst[v * V + j] = to_f32(e[j]);
-  }
-}
-
-// Copy `bytes` (multiple of 16) from global to shared memory unchanged.
-__device__ __forceinline__ void stage_raw(void *dst, const void *src, int bytes, int tid) {
-  const uint4 *s4 = static_cast<const uint4 *>(src);
-  uint4 *d4 = static_cast<uint4 *>(dst);
-  for (int v = tid; v < bytes / 16; v += kThreads) d4[v] = s4[v];
-}
-
-__host__ __device__ __forceinline__ int pad4(int n) { return (n + 3) & ~3; }
-
-// Shared-memory layout of the decode / fold kernels (floats unless noted):
-//   B [L][N] | C [N] | bc [pad4(L)] | dt [hc][L] | wdt [hc][L] | lam [pad4(hc)]
-//   | red [2][8] (tile maxima, alternating between consecutive heads) | x [hc][L][P] (input dtype)
-struct DecodeSmem {
-  float *B, *C, *bc, *dt, *wdt, *lam, *red;
-  void *x;
-  __host__ __device__ static size_t bytes(int L, int hc, int P, int N, int es) {
-    const size_t f = (size_t)L * N + N + pad4(L) + 2 * pad4(hc * L) + pad4(hc) + 16;
-    return f * 4 + (size_t)hc * L * P * es;
-  }
-  __device__ DecodeSmem(unsigned char *base, int L, int hc, int N) {
-    float *f = reinterpret_cast<float *>(base);
-    B = f;
-    C = B + L * N;
-    bc = C + N;
-    dt = bc + pad4(L);
-    wdt = dt + pad4(hc * L);
-    lam = wdt + pad4(hc * L);
-    red = lam + pad4(hc);
-    x = red + 16;
-  }
-};
-
-// ------------------------------------------------------------- row helpers
-// One row of a P x N head tile as seen by one lane of the decode kernel:
-// columns 32 s + 4 c8 (s < N/32), four values each.
-
-template <int P, int N, int QM>
-__device__ __forceinline__ void view_row(const unsigned char *t, int r, int c8, float sg,
-                                         float4 (&v)[N / 32]) {
-#pragma unroll
-  for (int s = 0; s < N / 32; ++s) {
-    const int c = 32 * s + 4 * c8;
-    if constexpr (QM == 1) {
-      const uint32_t w = *reinterpret_cast<const uint32_t *>(t + r * N + c);
-      v[s] = make_float4(e4m3_decode(w & 0xFF), e4m3_decode((w >> 8) & 0xFF),
-                         e4m3_decode((w >> 16) & 0xFF), e4m3_decode(w >> 24));
-    } else if constexpr (QM == 2) {
-      const uint32_t w = *reinterpret_cast<const uint16_t *>(t + r * (N / 2) + c / 2);
-      const float sb = e4m3_decode(t[P * N / 2 + r * (N / 16) + c / 16]);
-      v[s] = make_float4(nvfp4_value(w & 0xF, sb, sg), nvfp4_value((w >> 4) & 0xF, sb, sg),
-                         nvfp4_value((w >> 8) & 0xF, sb, sg), nvfp4_value((w >> 12) & 0xF, sb, sg));
-    } else {
-      v[s] = *reinterpret_cast<const float4 *>(t + (r * N + c) * 4);
-    }
-  }
-}
-
-template <int N>
-__device__ __forceinline__ void load_row(const float *tile, int r, int c8, float4 (&v)[N / 32]) {
-#pragma unroll
-  for (int s = 0; s < N / 32; ++s) v[s] = ld_stream(tile + (size_t)r * N + 32 * s + 4 * c8);
-}
-
-template <int N>
-__device__ __forceinline__ void store_row(float *tile, int r, int c8, const float4 (&v)[N / 32]) {
-#pragma unroll
-  for (int s = 0; s < N / 32; ++s) st_stream(tile + (size_t)r * N + 32 * s + 4 * c8, v[s]);
-}
-
-// v <- a * v and v <- x * b + v on a float4 as two paired fp32 operations
-// (Blackwell's f32x2 pipe: per component the same rounding as fmulf / fmaf).
-__device__ __forceinline__ float4 mul4x(float a, float4 v) {
-  const float2 a2 = make_float2(a, a);
-  const float2 lo = __fmul2_rn(a2, make_float2(v.x, v.y));
-  const float2 hi = __fmul2_rn(a2, make_float2(v.z, v.w));
-  return make_float4(lo.x, lo.y, hi.x, hi.y);
-}
-__device__ __forceinline__ float4 fma4x(float x, float4 b, float4 v) {
-  const float2 x2 = make_float2(x, x);
-  const float2 lo = __ffma2_rn(x2, make_float2(b.x, b.y), make_float2(v.x, v.y));
-  const float2 hi = __ffma2_rn(x2, make_float2(b.z, b.w), make_float2(v.z, v.w));
-  return make_float4(lo.x, lo.y, hi.x, hi.y);
-}
-
-// The fold of RGC register-held rows of one head:
-//   v[u] <- lam v[u] + sum_{i<k} (w_i x_i[rows[u]]) B_i[cols],
-// record loop outermost so that each B_i fragment (fp32 in shared memory) is
-// loaded once and feeds 4 * RGC * (N/32) independent FMAs (issued in pairs).
-template <int P, int N, typename TI, int RGC>
-__device__ __forceinline__ void fold_rows(float4 (&v)[RGC][N / 32], float lam, int k,
-                                          const float *w, const TI *x, const int (&rows)[RGC],
-                                          const float *Bf, int c8) {
-#pragma unroll
-  for (int u = 0; u < RGC; ++u)
-#pragma unroll
-    for (int s = 0; s < N / 32; ++s) v[u][s] = mul4x(lam, v[u][s]);
-  for (int i = 0; i < k; ++i) {
-    float4 bb[N / 32];
-#pragma unroll
-    for (int s = 0; s < N / 32; ++s)
-      bb[s] = *reinterpret_cast<const float4 *>(&Bf[i * N + 32 * s + 4 * c8]);
-    const float wi = w[i];
-#pragma unroll
-    for (int u = 0; u < RGC; ++u) {
-      const float xw = wi * to_f32(x[i * P + rows[u]]);
-#pragma unroll
-      for (int s = 0; s < N / 32; ++s) v[u][s] = fma4x(xw, bb[s], v[u][s]);
-    }
-  }
-}
-
-template <int N>
-__device__ __forceinline__ void fp8_roundtrip_row(float4 (&v)[N / 32]) {
-#pragma unroll
-  for (int s = 0; s < N / 32; ++s)
-    v[s] = make_float4(e4m3_decode(e4m3_encode(v[s].x)), e4m3_decode(e4m3_encode(v[s].y)),
-                       e4m3_decode(e4m3_encode(v[s].z)), e4m3_decode(e4m3_encode(v[s].w)));
-}
-
-template <int N>
-__device__ __forceinline__ void fp8_codes_row(uint8_t *rc_tile, int r, int c8,
-                                              const float4 (&v)[N / 32]) {
-#pragma unroll
-  for (int s = 0; s < N / 32; ++s) {
-    const uint32_t w = e4m3_encode(v[s].x) | (e4m3_encode(v[s].y) << 8) |
-                       (e4m3_encode(v[s].z) << 16) | (e4m3_encode(v[s].w) << 24);
-    *reinterpret_cast<uint32_t *>(rc_tile + (size_t)r * N + 32 * s + 4 * c8) = w;
-  }
-}
-
-template <int N>
-__device__ __forceinline__ float absmax_row(const float4 (&v)[N / 32]) {
-  float m = 0.f;
-#pragma unroll
-  for (int s = 0; s < N / 32; ++s)
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(v[s].x), fabsf(v[s].y)), fmaxf(fabsf(v[s].z), fabsf(v[s].w))));
-  return m;
-}
-
-// NVFP4 of one row given the tile scale: block maxima over the 4 lanes that
-// share a 16-column block, then codes (written) or deq(Q(v)) (roundtrip).
-template <int P, int N>
-__device__ __forceinline__ void nvfp4_row(float4 (&v)[N / 32], float sg, bool roundtrip,
-                                          uint8_t *rc_tile, uint8_t *sc_tile, int r, int c8) {
-#pragma unroll
-  for (int s = 0; s < N / 32; ++s) {
-    const int c = 32 * s + 4 * c8;
-    float bm = fmaxf(fmaxf(fabsf(v[s].x), fabsf(v[s].y)), fmaxf(fabsf(v[s].z), fabsf(v[s].w)));
-    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-    const uint32_t scode = nvfp4_block_code(bm, sg);
-    const float d = nvfp4_step(scode, sg);
-    const uint32_t lo = nvfp4_pack2(v[s].x, v[s].y, d), hi = nvfp4_pack2(v[s].z, v[s].w, d);
-    if (roundtrip) {
-      const float sb = e4m3_decode(scode);
-      v[s] = make_float4(nvfp4_value(lo & 0xF, sb, sg), nvfp4_value(lo >> 4, sb, sg),
-                         nvfp4_value(hi & 0xF, sb, sg), nvfp4_value(hi >> 4, sb, sg));
-    } else {
-      *reinterpret_cast<uint16_t *>(rc_tile + (size_t)r * (N / 2) + c / 2) = (uint16_t)(lo | (hi << 8));
-      if ((c8 & 3) == 0) sc_tile[(size_t)r * (N / 16) + c / 16] = (uint8_t)scode;
-    }
-  }
-}
 
 // =============================================================== decode step
 // Persistent, warp-specialised kernel: one CTA per SM walks work items
@@ -641,14 +150,6 @@ struct Stage {
   }
 };
 
-__device__ __forceinline__ void item_coords(const M2Params &p, int item, int nchunk, int hc, int &b,
-                                            int &g, int &chunk, int &h_first) {
-  const int bg_i = item / nchunk;
-  chunk = item - bg_i * nchunk;
-  b = bg_i / p.G;
-  g = bg_i - b * p.G;
-  h_first = g * p.hpg + chunk * hc;
-}
 
 // Stager warp: for item `it` wait until its record buffer is free, then stage
 // the small per-item inputs.  Every global load of the item is issued first
@@ -770,81 +271,6 @@ __device__ __forceinline__ void decode_stager(const M2Params &p, const DecodeLay
 // tiles into a ring of NS slots, hc heads per item, waiting only for free
 // slots.  On a failed wait it marks the CTA aborted and waits (bounded) for
 // the copies it has in flight before returning.
-// Tile producer (one thread): streams the checkpoint tiles (or their read
-// copies) of this CTA's items, in item order, into the NS-slot ring.  With
-// pf > 0 it also keeps an L2 prefetch pf tiles ahead of the ring, so HBM
-// keeps streaming while the consumers spend time on per-item work that does
-// not release ring slots.
-template <int P, int N, int QM>
-__device__ __forceinline__ void stream_tiles(const M2Params &p, uint64_t *full, uint64_t *empty,
-                                             unsigned char *ring, int NS, int tile_stride,
-                                             int tile_bytes, int hc, volatile int *abort_flag,
-                                             int nitems, int nchunk, int pf) {
-  auto src_of = [&](int item, int j) -> size_t {
-    int b, g, chunk, h_first;
-    item_coords(p, item, nchunk, hc, b, g, chunk, h_first);
-    return (size_t)b * p.H + h_first + j;
-  };
-  auto prefetch = [&](size_t bh) {
-    if constexpr (QM == 1) {
-      bulk_prefetch_l2(p.rc + bh * (size_t)(P * N), P * N);
-    } else if constexpr (QM == 2) {
-      bulk_prefetch_l2(p.rc + bh * (size_t)(P * N / 2), P * N / 2);
-      bulk_prefetch_l2(p.rc_scale + bh * (size_t)(P * N / 16), P * N / 16);
-    } else {
-      bulk_prefetch_l2(p.h0 + bh * (size_t)(P * N), P * N * 4);
-    }
-  };
-  int pitem = blockIdx.x, pj = 0;  // next tile to prefetch
-  auto prefetch_next = [&]() {
-    if (pitem < nitems) {
-      prefetch(src_of(pitem, pj));
-      if (++pj == hc) {
-        pj = 0;
-        pitem += gridDim.x;
-      }
-    }
-  };
-  if (pf > 0)
-    for (int k = 0; k < pf + NS; ++k) prefetch_next();
-  int slot = 0;
-  uint32_t sphase = 0;
-  uint32_t issued = 0, parity = 0;  // per slot: a copy was issued / its phase parity
-  bool failed = false;
-  for (int item = blockIdx.x; item < nitems && !failed; item += gridDim.x) {
-    for (int j = 0; j < hc; ++j) {
-      if (pf > 0) prefetch_next();
-      if (*abort_flag || !mbar_wait(&empty[slot], sphase ^ 1)) {
-        failed = true;
-        break;
-      }
-      mbar_arrive_expect_tx(&full[slot], tile_bytes);
-      unsigned char *dst = ring + slot * tile_stride;
-      const size_t bh = src_of(item, j);
-      if constexpr (QM == 1) {
-        bulk_g2s(dst, p.rc + bh * (size_t)(P * N), P * N, &full[slot]);
-      } else if constexpr (QM == 2) {
-        bulk_g2s(dst, p.rc + bh * (size_t)(P * N / 2), P * N / 2, &full[slot]);
-        bulk_g2s(dst + P * N / 2, p.rc_scale + bh * (size_t)(P * N / 16), P * N / 16, &full[slot]);
-      } else {
-        bulk_g2s(dst, p.h0 + bh * (size_t)(P * N), P * N * 4, &full[slot]);
-      }
-      issued |= 1u << slot;
-      parity = (parity & ~(1u << slot)) | (sphase << slot);
-      if (++slot == NS) {
-        slot = 0;
-        sphase ^= 1;
-      }
-    }
-  }
-  if (failed) {
-    if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
-    *abort_flag = 1;
-    for (int s = 0; s < NS; ++s)
-      if (issued & (1u << s)) mbar_wait(&full[s], (parity >> s) & 1u);
-  }
-}
-
 template <int P, int N, int QM>
 __device__ __forceinline__ void decode_tiles(const M2Params &p, const DecodeLayout &lay,
                                              const DecodeSmemPtrs &S, volatile int *abort_flag,
@@ -1221,616 +647,6 @@ __global__ void __launch_bounds__(kThreads, 2) m2_full_kernel(const M2Params p) 
   }
 }
 
-// ============================================================ verify round
-// Persistent speculative-verify kernel, structured like the decode kernel.
-// Work item = (sequence, group, chunk) with hc = (H/G)/nchunk heads; nchunk
-// is 1 unless the staged records of all the group's heads do not fit in
-// shared memory beside the tile ring.  Per item:
-//   1. commit of the previous round: n1 = len + accepted; when n1 >= window
-//      the n1 buffered records are folded into h0 (written once) and the
-//      drafts follow an empty buffer (nb = 0), else nb = n1;
-//   2. the nd drafts are appended to slots nb .. nb+nd-1 (len stays nb);
-//   3. draft d's output from the (possibly folded) checkpoint and records
-//      0..nb+d, with no intermediate state:
-//        y_d = Lam_d (h C_d) + sum_i w_{d,i} (B_i . C_d) x_i + D x_d.
-// The stager (warp 9) reads the lengths and acceptance counts, loads the
-// small inputs, and bulk-copies the buffered prefix records and the draft
-// rows (x, B, C); warp 8 streams the heads' checkpoint tiles; warps 0-7 form
-// the fold weights, every draft's decay weights and B.C dots (fp64) and the
-// per-row terms z_d, then take one head at a time (8 warps, 8 rows each):
-// rows into registers, slot released, optional fold + write-back, and all
-// nd outputs from the same registers.
-// With nchunk > 1 the draft B and C rows (one copy per group) are appended
-// by m2_verify_append_bc_kernel after this kernel: a chunk that folds would
-// otherwise overwrite buffered B records that another chunk's CTA may not
-// have copied yet.
-
-constexpr int kMD = 4;  // most drafts per round
-// Consumer warps form kVGroups groups that take alternate items (with two
-// groups one group's per-item setup overlaps the other's tile streaming; on
-// B200 that measured no faster than one group of 16 warps, which is used).
-constexpr int kVGroups = 1, kGWarps = 16, kGThreads = 32 * kGWarps;
-constexpr int kVWarps = kVGroups * kGWarps, kVThreads = 32 * kVWarps;
-
-struct VerifyLayout {
-  int NS, NR, hc, nchunk, cap, L, tile_bytes, tile_stride;
-  int rec_floats, db_floats;  // stage floats per record buffer, scratch per item
-  int off_bars, off_recB, off_recX, off_dX, off_dB, off_dC, off_rec, off_scr, off_ring, total;
-  int db_b, scr_b;  // per consumer group: item scratch bytes, all scratch bytes
-  int recB_b, recX_b, dX_b, dBC_b;  // bytes per record buffer of each array
-  __host__ static int a128(int v) { return (v + 127) & ~127; }
-  __host__ static VerifyLayout make(int P, int N, int hpg, int nchunk, int cap, int L, int es,
-                                    int budget) {
-    VerifyLayout d;
-    d.nchunk = nchunk;
-    const int hc = d.hc = hpg / nchunk;
-    d.cap = cap;
-    d.L = L;
-    d.tile_bytes = P * N * 4;
-    d.tile_stride = a128(d.tile_bytes);
-    d.recB_b = a128(cap * N * es);
-    d.recX_b = a128(hc * cap * P * es);
-    d.dX_b = a128(kMD * hc * P * es);
-    d.dBC_b = a128(kMD * N * es);
-    // stage: dt prefix [hc][cap] | dt drafts [4][hc] | A [hc] | D [hc] | hdr [8]
-    d.rec_floats = pad4(hc * cap) + kMD * hc + pad4(hc) * 2 + 8;
-    // per item: Bf [cap][N] | wf [hc][cap] | lamf [hc] | lamd [4][hc] | z [4][hc][P]
-    d.db_floats = cap * N + pad4(hc * cap) + pad4(hc) + kMD * hc + kMD * hc * P;
-    for (d.NR = 2; d.NR >= 1; --d.NR) {
-      int o = 0;
-      d.off_bars = o;
-      o += 256;
-      d.off_recB = o;
-      o += d.NR * d.recB_b;
-      d.off_recX = o;
-      o += d.NR * d.recX_b;
-      d.off_dX = o;
-      o += d.NR * d.dX_b;
-      d.off_dB = o;
-      o += d.NR * d.dBC_b;
-      d.off_dC = o;
-      o += d.NR * d.dBC_b;
-      d.off_rec = o;
-      o += a128(d.NR * d.rec_floats * 4);
-      // per consumer group: item scratch | bc [4][cap+4] double | cf [4][hc][cap+4] float
-      d.off_scr = o;
-      d.db_b = a128(d.db_floats * 4);
-      d.scr_b = d.db_b + a128(kMD * (cap + kMD) * 8 + kMD * hc * (cap + kMD) * 4);
-      o += kVGroups * d.scr_b;
-      d.off_ring = o;
-      d.NS = (budget - o) / d.tile_stride;
-      if (d.NS > 8) d.NS = 8;
-      if (d.NS >= 2) {
-        d.total = o + d.NS * d.tile_stride;
-        return d;
-      }
-    }
-    d.NS = 0;
-    return d;
-  }
-};
-
-template <int P, int N, typename TI>
-__device__ __forceinline__ bool verify_stage(const M2Params &p, const VerifyLayout &lay,
-                                             unsigned char *smem, uint64_t *rfull,
-                                             uint64_t *rempty, int item, int it, int lane) {
-  constexpr int DPL = (8 * 20 + 31) / 32;  // prefix dt slots per lane (hc <= 8, cap <= 20)
-  const int hc = lay.hc, cap = lay.cap, L = lay.L, nd = p.n_draft;
-  const int rb = it % lay.NR;
-  const uint32_t rphase = (it / lay.NR) & 1;
-  bool ok = true;
-  if (lane == 0) ok = mbar_wait(&rempty[rb], rphase ^ 1);
-  if (!__shfl_sync(0xffffffffu, (int)ok, 0)) return false;
-  int b, g, chunk, h_first;
-  item_coords(p, item, lay.nchunk, hc, b, g, chunk, h_first);
-  const size_t bh0 = (size_t)b * p.H + h_first, bg = (size_t)b * p.G + g;
-
-  // ---- loads
-  const int my_len = lane < hc ? __ldcg(&p.len[bh0 + lane]) : 0;
-  const int a = p.acc ? __ldcg(&p.acc[b]) : 0;
-  const float my_A = lane < hc ? p.A[h_first + lane] : 0.f;
-  const float my_D = lane < hc ? p.D[h_first + lane] : 0.f;
-  float dtv[DPL];
-#pragma unroll
-  for (int u = 0; u < DPL; ++u) {
-    const int e = lane + 32 * u, j = e / cap, i = e - j * cap;
-    dtv[u] = e < hc * cap ? __ldcg(&p.dtbuf[(bh0 + j) * cap + i]) : 0.f;
-  }
-  const int dd = lane / hc, dj = lane - (lane / hc) * hc;  // draft dt: lane -> (d, j)
-  const float my_dtd = lane < nd * hc ? ld_in<TI>(p.dt, b * p.bs_dt + (int64_t)dd * p.H + h_first + dj)
-                                      : 0.f;
-  // ---- lengths and checks
-  const int n0 = __shfl_sync(0xffffffffu, my_len, 0);
-  const int n1 = n0 + a;
-  const bool fold = n1 >= L;
-  const int nb = fold ? 0 : n1;
-  const bool bad = __any_sync(0xffffffffu, (lane < hc && my_len != n0)) || n0 < 0 || n0 >= L ||
-                   a < 0 || a > p.draft_max || n1 > cap || nb + nd > cap;
-  const int n1c = bad ? 0 : n1;  // copies stay in bounds for a bad item
-  // ---- shared-memory writes
-  float *st = reinterpret_cast<float *>(smem + lay.off_rec) + rb * lay.rec_floats;
-  float *dtb = st, *dtd = st + pad4(hc * cap), *As = dtd + kMD * hc, *Ds = As + pad4(hc);
-  int *hdr = reinterpret_cast<int *>(Ds + pad4(hc));
-#pragma unroll
-  for (int u = 0; u < DPL; ++u) {
-    const int e = lane + 32 * u;
-    if (e < hc * cap) dtb[e] = dtv[u];
-  }
-  if (lane < nd * hc) dtd[dd * hc + dj] = my_dtd;
-  if (lane < hc) {
-    As[lane] = my_A;
-    Ds[lane] = my_D;
-  }
-  if (lane == 0) {
-    hdr[0] = n0;
-    hdr[1] = n1;
-    hdr[2] = fold;
-    hdr[3] = nb;
-    hdr[4] = bad;
-  }
-  fence_proxy_async_smem();
-  __syncwarp();
-  if (lane == 0) {
-    const uint32_t bB = n1c * N * sizeof(TI), bX = n1c * P * sizeof(TI);
-    const uint32_t bdX = hc * P * sizeof(TI), bdBC = N * sizeof(TI);
-    const uint32_t dcount = bad ? 0 : nd;
-    mbar_arrive_expect_tx(&rfull[rb], bB + hc * bX + dcount * (bdX + 2 * bdBC));
-    unsigned char *recB = smem + lay.off_recB + rb * lay.recB_b;
-    unsigned char *recX = smem + lay.off_recX + rb * lay.recX_b;
-    unsigned char *dX = smem + lay.off_dX + rb * lay.dX_b;
-    unsigned char *dB = smem + lay.off_dB + rb * lay.dBC_b;
-    unsigned char *dC = smem + lay.off_dC + rb * lay.dBC_b;
-    if (n1c > 0) {
-      bulk_g2s(recB, static_cast<const TI *>(p.Bbuf) + bg * cap * N, bB, &rfull[rb]);
-      for (int j = 0; j < hc; ++j)
-        bulk_g2s(recX + (size_t)j * cap * P * sizeof(TI),
-                 static_cast<const TI *>(p.xbuf) + (bh0 + j) * cap * P, bX, &rfull[rb]);
-    }
-    for (uint32_t d = 0; d < dcount; ++d) {
-      bulk_g2s(dX + d * bdX, static_cast<const TI *>(p.x) + b * p.bs_x + ((size_t)d * p.H + h_first) * P,
-               bdX, &rfull[rb]);
-      bulk_g2s(dB + d * bdBC, static_cast<const TI *>(p.Bm) + b * p.bs_B + ((size_t)d * p.G + g) * N,
-               bdBC, &rfull[rb]);
-      bulk_g2s(dC + d * bdBC, static_cast<const TI *>(p.Cm) + b * p.bs_C + ((size_t)d * p.G + g) * N,
-               bdBC, &rfull[rb]);
-    }
-  }
-  return true;
-}
-
-// Butterfly reduce-scatter over the 16 lanes of a half warp (lane bits 3..0):
-// every lane enters with V partial sums, and after log2(16) rounds lane c16
-// holds the complete sum of value c16 / (16 / V) (V = 4, 8 or 16).  Each
-// round sends half of the remaining values, so V sums cost V - 1 + (4 -
-// log2 V) shuffles instead of 4 V.
-template <int NV, int M>
-struct HalfWarpReduce {
-  static __device__ __forceinline__ void run(float *q, int c16) {
-    if constexpr (M > 0) {
-      if constexpr (NV == 1) {
-        q[0] += __shfl_xor_sync(0xffffffffu, q[0], M);
-        HalfWarpReduce<1, M / 2>::run(q, c16);
-      } else {
-        constexpr int H = NV / 2;
-        const bool up = c16 & M;
-#pragma unroll
-        for (int k = 0; k < H; ++k) {
-          const float keep = up ? q[H + k] : q[k], send = up ? q[k] : q[H + k];
-          q[k] = keep + __shfl_xor_sync(0xffffffffu, send, M);
-        }
-        HalfWarpReduce<H, M / 2>::run(q, c16);
-      }
-    }
-  }
-};
-
-// K consecutive input elements (bf16 or fp32) from shared memory as floats;
-// the address is aligned to K elements.
-template <typename TI, int K>
-__device__ __forceinline__ void ld_vec(const TI *src, float (&out)[K]) {
-  if constexpr (std::is_same<TI, float>::value) {
-    if constexpr (K == 4) {
-      const float4 v = *reinterpret_cast<const float4 *>(src);
-      out[0] = v.x, out[1] = v.y, out[2] = v.z, out[3] = v.w;
-    } else {
-      static_assert(K == 2, "2 or 4 elements");
-      const float2 v = *reinterpret_cast<const float2 *>(src);
-      out[0] = v.x, out[1] = v.y;
-    }
-  } else {
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(src);
-    if constexpr (K == 4) {
-      const uint2 u = *reinterpret_cast<const uint2 *>(src);
-      const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-      const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-      out[0] = lo.x, out[1] = lo.y, out[2] = hi.x, out[3] = hi.y;
-    } else {
-      static_assert(K == 2, "2 or 4 elements");
-      const float2 v = __bfloat1622float2(h[0]);
-      out[0] = v.x, out[1] = v.y;
-    }
-  }
-}
-
-template <typename TI>
-__device__ __forceinline__ float4 ld_vec4(const TI *src) {
-  float t[4];
-  ld_vec<TI, 4>(src, t);
-  return make_float4(t[0], t[1], t[2], t[3]);
-}
-
-
-template <int P, int N, typename TI>
-__global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyLayout lay) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int abort_word;
-  volatile int *abort_flag = &abort_word;
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.off_bars);
-  uint64_t *empty = full + 8, *rfull = empty + 8, *rempty = rfull + 4, *turn = rempty + 4;
-  unsigned char *ring = smem + lay.off_ring;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int hc = lay.hc, cap = lay.cap, nd = p.n_draft, R = cap + kMD;
-  const int nitems = p.B * p.G * lay.nchunk;
-  const bool own_bc = lay.nchunk == 1;
-
-  if (tid == 0) {
-    for (int s = 0; s < 8; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kGWarps);  // each tile is read by one group
-    }
-    for (int r = 0; r < 4; ++r) {
-      mbar_init(&rfull[r], 1);
-      mbar_init(&rempty[r], kGWarps);
-    }
-    for (int g2 = 0; g2 < kVGroups; ++g2) mbar_init(&turn[g2], kGWarps);
-    *abort_flag = 0;
-    mbar_fence_init();
-  }
-  __syncthreads();
-  if (warp == kVWarps) {
-    if (lane == 0)
-      stream_tiles<P, N, 0>(p, full, empty, ring, lay.NS, lay.tile_stride, lay.tile_bytes, hc,
-                            abort_flag, nitems, lay.nchunk, hc);
-    return;
-  }
-  if (warp == kVWarps + 1) {
-    int it = 0;
-    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
-      const bool abort_now = __any_sync(0xffffffffu, *abort_flag != 0);
-      if (abort_now || !verify_stage<P, N, TI>(p, lay, smem, rfull, rempty, item, it, lane)) {
-        if (lane == 0 && !abort_now) {
-          report(p.status, RSSM_ERR_TIMEOUT);
-          *abort_flag = 1;
-        }
-        return;
-      }
-    }
-    return;
-  }
-
-  // Consumer group grp takes this CTA's items it = grp, grp + 2, ...
-  // Head-loop lane layout: a half warp covers one row, lane c16 holds the
-  // columns 64 s + 4 c16 .. +3 (s < N/64); a warp owns RW = P/8 rows of
-  // every head, taken four at a time (two per half warp).
-  constexpr int S4 = N / 64, RW = P / kGWarps, NSP = RW / 4, RZ = P / 32;
-  static_assert(NSP >= 1 && S4 >= 1, "headdim and d_state must be at least 64");
-  const int grp = warp / kGWarps, gw = warp - grp * kGWarps, gtid = tid - grp * kGThreads;
-  const uint32_t gbar = 1 + grp;  // the group's named barrier
-  const int h16 = lane >> 4, c16 = lane & 15;
-  unsigned char *scr = smem + lay.off_scr + grp * lay.scr_b;
-  double *bc = reinterpret_cast<double *>(scr + lay.db_b);  // [4][R]
-  float *cf = reinterpret_cast<float *>(bc + kMD * R);     // [4][hc][R] coefficients
-  // Ring hand-off: a group starts waiting for its item's first tile only after
-  // every warp of the other group has acquired the previous item's last
-  // tile (turn[grp]), so a slot is never awaited more than one phase ahead.
-  // With a single record buffer the hand-off also precedes the record wait.
-  auto take_turn = [&](int it_) -> bool {
-    if constexpr (kVGroups == 1) return true;
-    if (it_ == 0) return true;
-    return mbar_wait(&turn[grp], ((it_ - 1) >> 1) & 1);
-  };
-  auto pass_turn = [&]() {
-    if constexpr (kVGroups > 1) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&turn[grp ^ 1]);
-    }
-  };
-  int it = grp;
-  for (int item = blockIdx.x + grp * gridDim.x; item < nitems;
-       item += kVGroups * gridDim.x, it += kVGroups) {
-    const int rb = it % lay.NR;
-    const uint32_t rphase = (it / lay.NR) & 1;
-    int b, g, chunk, h_first;
-    item_coords(p, item, lay.nchunk, hc, b, g, chunk, h_first);
-    const size_t bh0 = (size_t)b * p.H + h_first, bg = (size_t)b * p.G + g;
-    const float *st = reinterpret_cast<const float *>(smem + lay.off_rec) + rb * lay.rec_floats;
-    const float *dtb = st, *dtd = st + pad4(hc * cap), *As = dtd + kMD * hc, *Ds = As + pad4(hc);
-    const int *hdr = reinterpret_cast<const int *>(Ds + pad4(hc));
-    const TI *recB = reinterpret_cast<const TI *>(smem + lay.off_recB + rb * lay.recB_b);
-    const TI *recX = reinterpret_cast<const TI *>(smem + lay.off_recX + rb * lay.recX_b);
-    const TI *dX = reinterpret_cast<const TI *>(smem + lay.off_dX + rb * lay.dX_b);
-    const TI *dB = reinterpret_cast<const TI *>(smem + lay.off_dB + rb * lay.dBC_b);
-    const TI *dC = reinterpret_cast<const TI *>(smem + lay.off_dC + rb * lay.dBC_b);
-    float *db = reinterpret_cast<float *>(scr);
-    float *Bf = db, *wf = Bf + cap * N, *lamf = wf + pad4(hc * cap), *lamd = lamf + pad4(hc);
-    float *z = lamd + kMD * hc;
-
-    const bool got = (lay.NR > 1 || take_turn(it)) && mbar_wait(&rfull[rb], rphase);
-    if (!got) {
-      report(p.status, RSSM_ERR_TIMEOUT);
-      *abort_flag = 1;
-    }
-    if (bar_or(gbar, kGThreads, !got || *abort_flag)) break;
-    if (hdr[4]) {
-      if (gtid == 0) report(p.status, RSSM_ERR_STATE);
-      if (lay.NR > 1 && !take_turn(it)) {
-        report(p.status, RSSM_ERR_TIMEOUT);
-        *abort_flag = 1;
-      }
-      for (int j = 0; j < hc; ++j) {
-        const uint32_t pos = (uint32_t)it * hc + j;
-        if (!mbar_wait(&full[pos % lay.NS], (pos / lay.NS) & 1)) {
-          report(p.status, RSSM_ERR_TIMEOUT);
-          *abort_flag = 1;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[pos % lay.NS]);
-      }
-      pass_turn();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&rempty[rb]);
-      continue;
-    }
-    const int n1 = hdr[1], nb = hdr[3], K = nb + nd;
-    const bool fold = hdr[2];
-
-    // ---- S1: append the drafts (16-byte chunks); fp32 B for the fold;
-    // B_i . C_d in fp64
-    {
-      constexpr int XC = P * (int)sizeof(TI) / 16, BC = N * (int)sizeof(TI) / 16;
-      for (int c = gtid; c < nd * hc * XC; c += kGThreads) {
-        const int row = c / XC, k = c - row * XC, d = row / hc, j = row - d * hc;
-        reinterpret_cast<uint4 *>(static_cast<TI *>(p.xbuf) + ((bh0 + j) * cap + nb + d) * P)[k] =
-            reinterpret_cast<const uint4 *>(dX + (size_t)row * P)[k];
-      }
-      if (own_bc)
-        for (int c = gtid; c < 2 * nd * BC; c += kGThreads) {
-          const int which = c / (nd * BC), cc = c - which * (nd * BC), d = cc / BC, k = cc - d * BC;
-          TI *dst = static_cast<TI *>(which ? p.Cbuf : p.Bbuf) + (bg * cap + nb + d) * N;
-          reinterpret_cast<uint4 *>(dst)[k] =
-              reinterpret_cast<const uint4 *>((which ? dC : dB) + (size_t)d * N)[k];
-        }
-      if (gtid < nd * hc) {
-        const int d = gtid / hc, j = gtid - (gtid / hc) * hc;
-        p.dtbuf[(bh0 + j) * cap + nb + d] = dtd[d * hc + j];
-      }
-      if (fold)
-        for (int e = gtid; e < n1 * (N / 4); e += kGThreads)
-          reinterpret_cast<float4 *>(Bf)[e] = ld_vec4<TI>(recB + 4 * e);
-      const int npair = nd * K;  // (d, i) with i <= nb + d are used
-      constexpr int PER = N / 16;
-      for (int base = 0; base < npair; base += kGThreads / 16) {
-        const int pr = base + (gtid >> 4), c0 = (gtid & 15) * PER;
-        const int d = pr / K, i = pr - d * K;
-        const bool use = pr < npair && i <= nb + d;
-        double acc = 0.0;
-        if (use) {
-          const TI *Bi = i < nb ? recB + i * N : dB + (i - nb) * N;
-#pragma unroll
-          for (int e = 0; e < PER; e += 4) {
-            const float4 bv = ld_vec4<TI>(Bi + c0 + e), cv = ld_vec4<TI>(dC + d * N + c0 + e);
-            acc = fma((double)bv.x, (double)cv.x, acc);
-            acc = fma((double)bv.y, (double)cv.y, acc);
-            acc = fma((double)bv.z, (double)cv.z, acc);
-            acc = fma((double)bv.w, (double)cv.w, acc);
-          }
-        }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-        if (use && (gtid & 15) == 0) bc[d * R + i] = acc;
-      }
-    }
-    // draft C rows for this lane's columns, in registers for the whole item
-    float4 cr[kMD][S4];
-#pragma unroll
-    for (int d = 0; d < kMD; ++d)
-#pragma unroll
-      for (int s4 = 0; s4 < S4; ++s4) cr[d][s4] = ld_vec4<TI>(dC + d * N + 64 * s4 + 4 * c16);
-    bar_sync(gbar, kGThreads);
-
-    // ---- S2 (one warp per head): decay weights from fp64 suffix sums.
-    // Draft sequence: the nb committed records, then the nd drafts; with
-    // S_l = sum_{m >= l} dt_m, draft d (records 0..e, e = nb + d) weighs
-    // record i by exp(A (S_{i+1} - S_{e+1})) dt_i and the checkpoint by
-    // exp(A (S_0 - S_{e+1})).  Both factor through the reference point
-    // S_ref = S_{nb+1}:  exp(A (S_{i+1} - S_ref)) * exp(A (S_ref - S_{e+1})),
-    // so one exponential per lane serves every draft: lanes 0..K-1 take
-    // E_l = exp(A (S_{l+1} - S_ref)), lanes 27..30 take F_d = exp(A (S_ref -
-    // S_{e+1})) and lane 31 takes G = exp(A (S_0 - S_ref)).  No factor can
-    // overflow: S_ref - S_{e+1} and the S_{i+1} - S_ref of draft records span
-    // at most 4 dt, and every other argument is <= 0.  The fold sequence is
-    // the n1 committed records (weights exp(A S'_{l+1}) dt_l, decay
-    // exp(A S'_0)); both scans and both exponentials run side by side.
-    for (int j = gw; j < hc; j += kGWarps) {
-      const double A = As[j];
-      const double dts = lane < nb ? (double)dtb[j * cap + lane]
-                                   : (lane < K ? (double)dtd[(lane - nb) * hc + j] : 0.0);
-      const double dtf = fold && lane < n1 ? (double)dtb[j * cap + lane] : 0.0;
-      double Ss = dts, Sf = dtf;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const double ts = __shfl_down_sync(0xffffffffu, Ss, o);
-        const double tf = __shfl_down_sync(0xffffffffu, Sf, o);
-        if (lane + o < 32) {
-          Ss += ts;
-          Sf += tf;
-        }
-      }
-      const double Ss1 = __shfl_down_sync(0xffffffffu, Ss, 1);  // S_{l+1}; lanes >= K: 0
-      const double Sf1 = __shfl_down_sync(0xffffffffu, Sf, 1);
-      const double Sref = __shfl_sync(0xffffffffu, Ss, nb + 1);  // nb + 1 <= cap < 27
-      const double S0 = __shfl_sync(0xffffffffu, Ss, 0);
-      const double Sf0 = __shfl_sync(0xffffffffu, Sf, 0);
-      const double SeL = __shfl_sync(0xffffffffu, Ss, (nb + (lane - 27) + 1) & 31);  // lanes 27..30
-      double arg = 0.0;
-      if (lane < K) arg = A * (Ss1 - Sref);
-      else if (lane >= 27 && lane < 31) arg = lane - 27 < nd ? A * (Sref - SeL) : 0.0;
-      else if (lane == 31) arg = A * (S0 - Sref);
-      const double ex = exp(arg);
-      const double exf = exp(A * (lane + 1 < n1 ? Sf1 : (lane == 31 ? Sf0 : 0.0)));  // n1 <= 20
-      if (fold) {
-        if (lane < n1) wf[j * cap + lane] = (float)(exf * dtf);
-        if (lane == 31) lamf[j] = (float)exf;
-      }
-      const double G = __shfl_sync(0xffffffffu, ex, 31);
-#pragma unroll
-      for (int d = 0; d < kMD; ++d) {
-        const double F = __shfl_sync(0xffffffffu, ex, 27 + d);
-        if (d < nd) {
-          if (lane <= nb + d) cf[(d * hc + j) * R + lane] = (float)(ex * F * dts * bc[d * R + lane]);
-          if (lane == 0) lamd[d * hc + j] = (float)(G * F);
-        }
-      }
-    }
-    bar_sync(gbar, kGThreads);
-    // ---- S3 (one warp per (draft, head) row, RZ rows of the head per lane):
-    // z[d][j][r] = sum_i cf[d][j][i] x_i[r] + D_j x_d[r]
-    for (int row = gw; row < nd * hc; row += kGWarps) {
-      const int d = row / hc, j = row - d * hc;
-      const float *c = cf + (d * hc + j) * R;
-      float acc[RZ], xv[RZ];
-#pragma unroll
-      for (int k = 0; k < RZ; ++k) acc[k] = 0.f;
-      for (int i = 0; i < nb; ++i) {
-        ld_vec<TI, RZ>(recX + (j * cap + i) * P + RZ * lane, xv);
-        const float ci = c[i];
-#pragma unroll
-        for (int k = 0; k < RZ; ++k) acc[k] = fmaf(ci, xv[k], acc[k]);
-      }
-      for (int i = nb; i <= nb + d; ++i) {
-        ld_vec<TI, RZ>(dX + ((i - nb) * hc + j) * P + RZ * lane, xv);
-        const float ci = c[i];
-#pragma unroll
-        for (int k = 0; k < RZ; ++k) acc[k] = fmaf(ci, xv[k], acc[k]);
-      }
-      ld_vec<TI, RZ>(dX + (d * hc + j) * P + RZ * lane, xv);
-      const float Dj = Ds[j];
-#pragma unroll
-      for (int k = 0; k < RZ; ++k) z[(d * hc + j) * P + RZ * lane + k] = fmaf(Dj, xv[k], acc[k]);
-    }
-    bar_sync(gbar, kGThreads);
-
-    // ---- heads, one at a time: rows into registers, optional fold, outputs
-    if (lay.NR > 1 && !take_turn(it)) {
-      report(p.status, RSSM_ERR_TIMEOUT);
-      *abort_flag = 1;
-    }
-    for (int j = 0; j < hc; ++j) {
-      const int h = h_first + j;
-      const size_t bh = bh0 + j;
-      const uint32_t pos = (uint32_t)it * hc + j;
-      const int sl = pos % lay.NS;
-      if (!mbar_wait(&full[sl], (pos / lay.NS) & 1)) {
-        report(p.status, RSSM_ERR_TIMEOUT);
-        *abort_flag = 1;
-      }
-      if (j == hc - 1) pass_turn();
-      const float *tl = reinterpret_cast<const float *>(ring + sl * lay.tile_stride);
-      const float lf = fold ? lamf[j] : 0.f;
-#pragma unroll
-      for (int sp = 0; sp < NSP; ++sp) {
-        int rows[2];
-        float4 v[2][S4];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          rows[u] = gw * RW + 4 * sp + 2 * u + h16;
-#pragma unroll
-          for (int s4 = 0; s4 < S4; ++s4)
-            v[u][s4] = *reinterpret_cast<const float4 *>(tl + rows[u] * N + 64 * s4 + 4 * c16);
-        }
-        if (sp == NSP - 1) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[sl]);
-        }
-        if (fold) {  // v <- lam v + sum_i (w_i x_i[row]) B_i[cols], written back once
-#pragma unroll
-          for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int s4 = 0; s4 < S4; ++s4) v[u][s4] = mul4x(lf, v[u][s4]);
-          const float *wj = wf + j * cap;
-          const TI *xj = recX + j * cap * P;
-          for (int i = 0; i < n1; ++i) {
-            float4 bb[S4];
-#pragma unroll
-            for (int s4 = 0; s4 < S4; ++s4)
-              bb[s4] = *reinterpret_cast<const float4 *>(&Bf[i * N + 64 * s4 + 4 * c16]);
-            const float wi = wj[i];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const float xw = wi * to_f32(xj[i * P + rows[u]]);
-#pragma unroll
-              for (int s4 = 0; s4 < S4; ++s4) v[u][s4] = fma4x(xw, bb[s4], v[u][s4]);
-            }
-          }
-          float *tile = p.h0 + bh * (size_t)(P * N);
-#pragma unroll
-          for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int s4 = 0; s4 < S4; ++s4)
-              st_stream(tile + (size_t)rows[u] * N + 64 * s4 + 4 * c16, v[u][s4]);
-        }
-        float q[2 * kMD];  // paired fp32 FMAs over this lane's 4 S4 columns
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-          for (int d = 0; d < kMD; ++d) {
-            float2 a = __fmul2_rn(make_float2(v[u][0].x, v[u][0].y), make_float2(cr[d][0].x, cr[d][0].y));
-            a = __ffma2_rn(make_float2(v[u][0].z, v[u][0].w), make_float2(cr[d][0].z, cr[d][0].w), a);
-#pragma unroll
-            for (int s4 = 1; s4 < S4; ++s4) {
-              a = __ffma2_rn(make_float2(v[u][s4].x, v[u][s4].y), make_float2(cr[d][s4].x, cr[d][s4].y), a);
-              a = __ffma2_rn(make_float2(v[u][s4].z, v[u][s4].w), make_float2(cr[d][s4].z, cr[d][s4].w), a);
-            }
-            q[u * kMD + d] = a.x + a.y;
-          }
-        HalfWarpReduce<2 * kMD, 8>::run(q, c16);  // every lane shuffles
-        const int idx = c16 >> 1, u = idx / kMD, d = idx - u * kMD;
-        if ((c16 & 1) == 0 && d < nd) {
-          const int r = rows[u];
-          p.y[b * p.bs_y + ((size_t)d * p.H + h) * P + r] =
-              fmaf(lamd[d * hc + j], q[0], z[(d * hc + j) * P + r]);
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&rempty[rb]);
-    if (gtid < hc) p.len[bh0 + gtid] = nb;
-  }
-}
-
-// Chunked verify only: append the draft B and C rows of group (b, g) at the
-// group's committed length, read back from the length the verify kernel just
-// wrote.  An item the verify kernel rejected (its status already reports it)
-// is skipped when the slots would not fit.
-template <typename TI>
-__global__ void __launch_bounds__(128) m2_verify_append_bc_kernel(const M2Params p) {
-  const int b = blockIdx.x / p.G, g = blockIdx.x - (blockIdx.x / p.G) * p.G;
-  const size_t bg = (size_t)b * p.G + g;
-  const int nb = p.len[(size_t)b * p.H + (size_t)g * p.hpg];
-  if (nb < 0 || nb + p.n_draft > p.cap) return;
-  const TI *Bin = static_cast<const TI *>(p.Bm) + b * p.bs_B;
-  const TI *Cin = static_cast<const TI *>(p.Cm) + b * p.bs_C;
-  for (int e = threadIdx.x; e < p.n_draft * p.N; e += blockDim.x) {
-    const int d = e / p.N, c = e - d * p.N;
-    static_cast<TI *>(p.Bbuf)[(bg * p.cap + nb + d) * p.N + c] = Bin[((size_t)d * p.G + g) * p.N + c];
-    static_cast<TI *>(p.Cbuf)[(bg * p.cap + nb + d) * p.N + c] = Cin[((size_t)d * p.G + g) * p.N + c];
-  }
-}
-
 // ================================================================= launchers
 
 template <typename K>
@@ -1844,12 +660,6 @@ cudaError_t launch_dyn(K kernel, unsigned grid, size_t smem, cudaStream_t s, con
   return cudaGetLastError();
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
-  return n > 0 ? n : 148;
-}
 
 // Heads per decode work item: the whole group up to 8 heads, else chunks of 8
 // (per-item setup is amortised over as many heads as the ring allows).
@@ -1918,21 +728,6 @@ cudaError_t fold_mode(const M2Params &p, int mode, cudaStream_t s) {
   }
 }
 
-template <typename F>
-cudaError_t dispatch_shape(int P, int N, int bf16, F &&f) {
-#define RSSM_M2_CASE(PP, NN)                                                                    \
-  if (P == PP && N == NN)                                                                       \
-    return bf16 ? f(std::integral_constant<int, PP>{}, std::integral_constant<int, NN>{},       \
-                    __nv_bfloat16{})                                                            \
-                : f(std::integral_constant<int, PP>{}, std::integral_constant<int, NN>{}, 0.0f);
-  RSSM_M2_CASE(64, 64)
-  RSSM_M2_CASE(64, 128)
-  RSSM_M2_CASE(128, 64)
-  RSSM_M2_CASE(128, 128)
-#undef RSSM_M2_CASE
-  return cudaErrorInvalidValue;
-}
-
 }  // namespace
 
 bool m2_supported(int P, int N) { return (P == 64 || P == 128) && (N == 64 || N == 128); }
@@ -1962,30 +757,5 @@ cudaError_t m2_launch_full(const M2Params &p, cudaStream_t s) {
   });
 }
 
-cudaError_t m2_launch_verify(const M2Params &p, cudaStream_t s) {
-  if (p.B * p.G == 0) return cudaSuccess;
-  return dispatch_shape(p.P, p.N, p.in_bf16, [&](auto PP, auto NN, auto ti) {
-    using TI = decltype(ti);
-    constexpr int P_ = decltype(PP)::value, N_ = decltype(NN)::value;
-    VerifyLayout lay;
-    lay.NS = 0;
-    for (int nc = 1; nc <= p.hpg && lay.NS < 2; ++nc)
-      if (p.hpg % nc == 0)
-        lay = VerifyLayout::make(P_, N_, p.hpg, nc, p.cap, p.L, (int)sizeof(TI), 220 * 1024);
-    if (lay.NS < 2) return cudaErrorInvalidConfiguration;
-    auto kernel = m2_verify_kernel<P_, N_, TI>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
-    if (e != cudaSuccess) return e;
-    const int nitems = p.B * p.G * lay.nchunk;
-    const int grid = nitems < sm_count() ? nitems : sm_count();
-    kernel<<<grid, kVThreads + 64, lay.total, s>>>(p, lay);
-    if (lay.nchunk > 1) {
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      m2_verify_append_bc_kernel<TI><<<p.B * p.G, 128, 0, s>>>(p);
-    }
-    return cudaGetLastError();
-  });
-}
 
 }  // namespace rssm

@@ -52,6 +52,10 @@ def parse():
                     help="sequences of m2_serving (profiling captures use a smaller batch)")
     ap.add_argument("--sub-steps", type=int, default=60,
                     help="timed windows / rounds of the secondary measurements")
+    ap.add_argument("--drift", action="store_true",
+                    help="instead of timing: output-error drift of the low-precision read copy "
+                         "and of a quantised checkpoint over m2_readcopy (batch 64, 8192 steps)")
+    ap.add_argument("--drift-steps", type=int, default=8192)
     return ap.parse_args()
 
 
@@ -571,9 +575,103 @@ def bench_verify(args, dev, peak, rs, bm, wl, torch):
             "gpu_launches": rounds}
 
 
+def run_drift(args, rank):
+    """m2_readcopy: batch 64 of the m2_serving heads decoded for 8192 steps by
+    five replay variants on the same inputs -- fp32 checkpoint (the
+    reference), FP8 / NVFP4 read copy over an fp32 checkpoint, and FP8 / NVFP4
+    quantised checkpoint -- plus the conventional fp32 full-state decode.  Per
+    step, each variant's output error against the fp32 replay output:
+    max_i |y - y_ref| / max(|y_ref|, 1e-2 rms(y_ref)) and the normwise
+    ||y - y_ref|| / ||y_ref||.  Prints one JSON line (errors at t = 16, 128,
+    1024, 8192 as the max over the preceding half-decade, and the fitted
+    growth exponent of the normwise error in t)."""
+    if rank != 0:
+        return
+    import math
+
+    import torch
+
+    from ssm_state_storage_b200 import replayssm as rs
+    from ssm_state_storage_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = wl.make("m2_readcopy")
+    T = args.drift_steps
+    g = wl.Generator(w)
+    A, D = (t.to(dev) for t in g.params())
+    S0 = g.initial_state().to(dev)
+    variants = [("fp32", {}), ("read_fp8", {"read_fmt": "fp8"}), ("read_nvfp4", {"read_fmt": "nvfp4"}),
+                ("ckpt_fp8", {"ckpt_fmt": "fp8"}), ("ckpt_nvfp4", {"ckpt_fmt": "nvfp4"})]
+    runs = []
+    for name, kw in variants:
+        layer = rs.Layer("m2", w.B, w.H, w.P, w.N, ngroups=w.G, window=w.L, in_dtype=w.in_dtype, **kw)
+        st = rs.ReplayState(layer, device=dev)
+        rs.replayssm_init(layer, st, S0)
+        runs.append((name, layer, st))
+    full_layer = rs.Layer("m2", w.B, w.H, w.P, w.N, ngroups=w.G, window=w.L, in_dtype=w.in_dtype)
+    S_full = S0.clone()
+    names = [v[0] for v in variants[1:]] + ["full_state_fp32"]
+    maxrel = {n: torch.zeros(T, dtype=torch.float64) for n in names}
+    normw = {n: torch.zeros(T, dtype=torch.float64) for n in names}
+    y = {n: torch.empty(w.B, w.H, w.P, device=dev) for n, _ in variants}
+    y["full_state_fp32"] = torch.empty(w.B, w.H, w.P, device=dev)
+    chunk = 256
+    t0 = time.time()
+    for c0 in range(0, T, chunk):
+        n = min(chunk, T - c0)
+        stp = {k: v.to(dev) for k, v in g.steps(n).items()}
+        mr = {k: torch.empty(n, device=dev) for k in names}
+        nw = {k: torch.empty(n, device=dev) for k in names}
+        for t in range(n):
+            inp = dict(x=stp["x"][t], dt=stp["dt"][t], Bm=stp["Bm"][t], Cm=stp["Cm"][t], A=A, D=D)
+            for name, layer, st in runs:
+                rs.replayssm_decode_step(layer, st, inp, y[name])
+            rs.replayssm_full_decode_step(full_layer, S_full, inp, y["full_state_fp32"])
+            ref = y["fp32"]
+            rms = ref.square().mean().sqrt()
+            den = torch.maximum(ref.abs(), 1e-2 * rms)
+            for k in names:
+                diff = y[k] - ref
+                mr[k][t] = (diff.abs() / den).max()
+                nw[k][t] = diff.norm() / ref.norm()
+        for k in names:
+            maxrel[k][c0:c0 + n] = mr[k].double().cpu()
+            normw[k][c0:c0 + n] = nw[k].double().cpu()
+    for name, _, st in runs:
+        if st.status() != 0:
+            raise RuntimeError(f"device status {st.status()} in variant {name}")
+    marks = [m for m in (16, 128, 1024, 8192) if m <= T]
+
+    def at(series, m):  # max over (m / sqrt(8), m]
+        lo = max(int(m / math.sqrt(8)), 1)
+        return float(series[lo - 1:m].max())
+
+    def growth(series):  # least-squares slope of log(err) in log(t), t >= 16
+        ts = torch.arange(16, T + 1, dtype=torch.float64)
+        e = series[15:T].clamp_min(1e-30)
+        lx, ly = ts.log(), e.log()
+        lx, ly = lx - lx.mean(), ly - ly.mean()
+        return float((lx * ly).sum() / (lx * lx).sum())
+
+    out = {"metric": "output error vs the fp32 replay output over a long decode", "workload":
+           "m2_readcopy", "config": {"batch": w.B, "heads": w.H, "headdim": w.P, "d_state": w.N,
+                                      "groups": w.G, "window": w.L, "steps": T, "inputs": "bf16"},
+           "data": "synthetic", "seconds": time.time() - t0, "variants": {}}
+    for k in names:
+        out["variants"][k] = {
+            "max_rel": {str(m): at(maxrel[k], m) for m in marks},
+            "normwise": {str(m): at(normw[k], m) for m in marks},
+            "normwise_growth_exponent": growth(normw[k]),
+        }
+    print(json.dumps(out), flush=True)
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
+    if args.drift:
+        run_drift(args, rank)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.impl == "reference":
         run_reference(args, rank)

@@ -579,8 +579,10 @@ def run_drift(args, rank):
     """m2_readcopy: batch 64 of the m2_serving heads decoded for 8192 steps by
     five replay variants on the same inputs -- fp32 checkpoint (the
     reference), FP8 / NVFP4 read copy over an fp32 checkpoint, and FP8 / NVFP4
-    quantised checkpoint -- plus the conventional fp32 full-state decode.  Per
-    step, each variant's output error against the fp32 replay output:
+    quantised checkpoint -- plus the conventional fp32 full-state decode, for
+    two decay settings: the workload's A_h = -exp(U(0, ln 16)) (the state
+    forgets a window in ~e^-8) and a long-memory A_h / 100.  Per step, each
+    variant's output error against the fp32 replay output of its setting:
     max_i |y - y_ref| / max(|y_ref|, 1e-2 rms(y_ref)) and the normwise
     ||y - y_ref|| / ||y_ref||.  Prints one JSON line (errors at t = 16, 128,
     1024, 8192 as the max over the preceding half-decade, and the fitted
@@ -598,48 +600,54 @@ def run_drift(args, rank):
     w = wl.make("m2_readcopy")
     T = args.drift_steps
     g = wl.Generator(w)
-    A, D = (t.to(dev) for t in g.params())
+    A0, D = (t.to(dev) for t in g.params())
     S0 = g.initial_state().to(dev)
-    variants = [("fp32", {}), ("read_fp8", {"read_fmt": "fp8"}), ("read_nvfp4", {"read_fmt": "nvfp4"}),
-                ("ckpt_fp8", {"ckpt_fmt": "fp8"}), ("ckpt_nvfp4", {"ckpt_fmt": "nvfp4"})]
-    runs = []
-    for name, kw in variants:
-        layer = rs.Layer("m2", w.B, w.H, w.P, w.N, ngroups=w.G, window=w.L, in_dtype=w.in_dtype, **kw)
-        st = rs.ReplayState(layer, device=dev)
-        rs.replayssm_init(layer, st, S0)
-        runs.append((name, layer, st))
+    settings = {"workload_A": A0, "long_memory_A/100": A0 / 100.0}
+    fmts = [("fp32", {}), ("read_fp8", {"read_fmt": "fp8"}), ("read_nvfp4", {"read_fmt": "nvfp4"}),
+            ("ckpt_fp8", {"ckpt_fmt": "fp8"}), ("ckpt_nvfp4", {"ckpt_fmt": "nvfp4"})]
+    runs = {}
+    for sname in settings:
+        for name, kw in fmts:
+            layer = rs.Layer("m2", w.B, w.H, w.P, w.N, ngroups=w.G, window=w.L,
+                             in_dtype=w.in_dtype, **kw)
+            st = rs.ReplayState(layer, device=dev)
+            rs.replayssm_init(layer, st, S0)
+            runs[(sname, name)] = (layer, st, torch.empty(w.B, w.H, w.P, device=dev))
     full_layer = rs.Layer("m2", w.B, w.H, w.P, w.N, ngroups=w.G, window=w.L, in_dtype=w.in_dtype)
-    S_full = S0.clone()
-    names = [v[0] for v in variants[1:]] + ["full_state_fp32"]
-    maxrel = {n: torch.zeros(T, dtype=torch.float64) for n in names}
-    normw = {n: torch.zeros(T, dtype=torch.float64) for n in names}
-    y = {n: torch.empty(w.B, w.H, w.P, device=dev) for n, _ in variants}
-    y["full_state_fp32"] = torch.empty(w.B, w.H, w.P, device=dev)
+    S_full = {sname: S0.clone() for sname in settings}
+    y_full = {sname: torch.empty(w.B, w.H, w.P, device=dev) for sname in settings}
+    names = [n for n, _ in fmts[1:]] + ["full_state_fp32"]
+    keys = [(sn, n) for sn in settings for n in names]
+    maxrel = {k: torch.zeros(T, dtype=torch.float64) for k in keys}
+    normw = {k: torch.zeros(T, dtype=torch.float64) for k in keys}
     chunk = 256
     t0 = time.time()
     for c0 in range(0, T, chunk):
         n = min(chunk, T - c0)
         stp = {k: v.to(dev) for k, v in g.steps(n).items()}
-        mr = {k: torch.empty(n, device=dev) for k in names}
-        nw = {k: torch.empty(n, device=dev) for k in names}
+        mr = {k: torch.empty(n, device=dev) for k in keys}
+        nw = {k: torch.empty(n, device=dev) for k in keys}
         for t in range(n):
-            inp = dict(x=stp["x"][t], dt=stp["dt"][t], Bm=stp["Bm"][t], Cm=stp["Cm"][t], A=A, D=D)
-            for name, layer, st in runs:
-                rs.replayssm_decode_step(layer, st, inp, y[name])
-            rs.replayssm_full_decode_step(full_layer, S_full, inp, y["full_state_fp32"])
-            ref = y["fp32"]
-            rms = ref.square().mean().sqrt()
-            den = torch.maximum(ref.abs(), 1e-2 * rms)
-            for k in names:
-                diff = y[k] - ref
-                mr[k][t] = (diff.abs() / den).max()
-                nw[k][t] = diff.norm() / ref.norm()
-        for k in names:
+            for sname, A in settings.items():
+                inp = dict(x=stp["x"][t], dt=stp["dt"][t], Bm=stp["Bm"][t], Cm=stp["Cm"][t], A=A, D=D)
+                for name, _ in fmts:
+                    layer, st, yv = runs[(sname, name)]
+                    rs.replayssm_decode_step(layer, st, inp, yv)
+                rs.replayssm_full_decode_step(full_layer, S_full[sname], inp, y_full[sname])
+                ref = runs[(sname, "fp32")][2]
+                rms = ref.square().mean().sqrt()
+                den = torch.maximum(ref.abs(), 1e-2 * rms)
+                for name in names:
+                    yv = y_full[sname] if name == "full_state_fp32" else runs[(sname, name)][2]
+                    diff = yv - ref
+                    mr[(sname, name)][t] = (diff.abs() / den).max()
+                    nw[(sname, name)][t] = diff.norm() / ref.norm()
+        for k in keys:
             maxrel[k][c0:c0 + n] = mr[k].double().cpu()
             normw[k][c0:c0 + n] = nw[k].double().cpu()
-    for name, _, st in runs:
+    for (sname, name), (_, st, _) in runs.items():
         if st.status() != 0:
-            raise RuntimeError(f"device status {st.status()} in variant {name}")
+            raise RuntimeError(f"device status {st.status()} in variant {sname}/{name}")
     marks = [m for m in (16, 128, 1024, 8192) if m <= T]
 
     def at(series, m):  # max over (m / sqrt(8), m]
@@ -656,13 +664,13 @@ def run_drift(args, rank):
     out = {"metric": "output error vs the fp32 replay output over a long decode", "workload":
            "m2_readcopy", "config": {"batch": w.B, "heads": w.H, "headdim": w.P, "d_state": w.N,
                                       "groups": w.G, "window": w.L, "steps": T, "inputs": "bf16"},
-           "data": "synthetic", "seconds": time.time() - t0, "variants": {}}
-    for k in names:
-        out["variants"][k] = {
-            "max_rel": {str(m): at(maxrel[k], m) for m in marks},
-            "normwise": {str(m): at(normw[k], m) for m in marks},
-            "normwise_growth_exponent": growth(normw[k]),
-        }
+           "data": "synthetic", "seconds": time.time() - t0, "settings": {}}
+    for sname in settings:
+        out["settings"][sname] = {
+            name: {"max_rel": {str(m): at(maxrel[(sname, name)], m) for m in marks},
+                   "normwise": {str(m): at(normw[(sname, name)], m) for m in marks},
+                   "normwise_growth_exponent": growth(normw[(sname, name)])}
+            for name in names}
     print(json.dumps(out), flush=True)
 
 

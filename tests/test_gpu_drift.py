@@ -3,10 +3,8 @@ oracle over many flushes, and the error ordering of the low-precision
 variants (read copy over an fp32 checkpoint vs a quantised checkpoint)."""
 import numpy as np
 import pytest
-import torch
 
 import oracle
-from ssm_state_storage_b200 import replayssm as rs
 from ssm_state_storage_b200 import workloads as wl
 from tests import _gpu
 from tests._util import norm_err, rel_err
@@ -21,45 +19,47 @@ def _decode(w, A, D, S0, st, **kw):
 
 
 @pytest.fixture(scope="module")
-def runs():
+def draw():
     w = wl.make("m2_readcopy", B=2, H=16, G=2)
     g = wl.Generator(w)
     A, D = g.params()
-    S0 = g.initial_state()
-    st = g.steps(T)
-    out = {"fp32": _decode(w, A, D, S0, st)}
-    for kind in ("read_fmt", "ckpt_fmt"):
-        for fmt in ("fp8", "nvfp4"):
-            out[f"{kind}:{fmt}"] = _decode(w, A, D, S0, st, **{kind: fmt})
-    yc, _, _, _ = oracle.m2_conventional(S0, st["x"], st["dt"], st["Bm"], st["Cm"], A, D)
-    return w, out, yc
+    return w, A, D, g.initial_state(), g.steps(T)
 
 
-def test_fp32_replay_matches_oracle_over_64_flushes(runs):
+def test_fp32_replay_matches_oracle_over_64_flushes(draw):
     """1024 steps = 64 windows: per-step error against the fp64 conventional
     recurrence stays within the fp32 tolerance (no accumulation over folds)."""
-    w, out, yc = runs
-    got = out["fp32"]
+    w, A, D, S0, st = draw
+    got = _decode(w, A, D, S0, st)
+    yc, _, _, _ = oracle.m2_conventional(S0, st["x"], st["dt"], st["Bm"], st["Cm"], A, D)
     errs = [rel_err(a, b) for a, b in zip(got["y"], yc)]
     assert max(errs) < 1e-4, max(errs)
     assert got["state"].status() == 0
 
 
-def _curve(out, key):
-    ref = out["fp32"]["y"]
-    return np.array([norm_err(a, b) for a, b in zip(out[key]["y"], ref)])
-
-
 @pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
-def test_read_copy_error_stays_bounded_quantised_checkpoint_drifts(runs, fmt):
+@pytest.mark.parametrize("decay", [1.0, 0.01])
+def test_read_copy_error_stays_bounded_quantised_checkpoint_drifts(draw, fmt, decay):
     """[sitech §Bounding quantisation error]: the read copy's error enters the
     output only, so it does not grow with the horizon; quantising the
-    checkpoint itself feeds the error back into the recurrence."""
-    w, out, _ = runs
-    rc = _curve(out, f"read_fmt:{fmt}")
-    ck = _curve(out, f"ckpt_fmt:{fmt}")
-    early, late = slice(16, 144), slice(T - 128, T)
-    print(fmt, "read copy early/late", rc[early].mean(), rc[late].mean(),
-          "checkpoint early/late", ck[early].mean(), ck[late].mean())
-    assert rc[late].mean() < 3.0 * rc[early].mean()
-    assert ck[late].mean() > rc[late].mean()
+    checkpoint itself feeds the error back into the recurrence.  With the
+    workload's decay rates (decay = 1) a window forgets the checkpoint by
+    ~e^-8 and both errors stay flat; with a long memory (A / 100) the
+    quantised checkpoint's error accumulates over the folds."""
+    w, A, D, S0, st = draw
+    A = A * decay
+    ref = _decode(w, A, D, S0, st)["y"]
+    rc = np.array([norm_err(a, b) for a, b in zip(_decode(w, A, D, S0, st, read_fmt=fmt)["y"], ref)])
+    ck = np.array([norm_err(a, b) for a, b in zip(_decode(w, A, D, S0, st, ckpt_fmt=fmt)["y"], ref)])
+    early, late = slice(32, 160), slice(T - 128, T)
+    print(f"\n{fmt} decay {decay}: read copy early/late {rc[early].mean():.3e} {rc[late].mean():.3e}"
+          f"  checkpoint early/late {ck[early].mean():.3e} {ck[late].mean():.3e}")
+    # measured on B200 (this test's draw): read copy late/early 1.05-1.21 in all four
+    # cases; checkpoint late/early 1.2 (decay 1) and 2.0-2.2 (decay 0.01), where it
+    # ends 3.2-3.5x above the read copy
+    assert rc[late].mean() < 1.5 * rc[early].mean()
+    if decay < 1.0:
+        assert ck[late].mean() > 1.5 * ck[early].mean()
+        assert ck[late].mean() > 2.0 * rc[late].mean()
+    else:
+        assert ck[late].mean() < 1.5 * ck[early].mean()

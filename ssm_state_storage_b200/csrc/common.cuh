@@ -51,6 +51,21 @@ __device__ __forceinline__ float dot4(float4 a, float4 b) {
   return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
 }
 
+// v <- a * v and v <- x * b + v on a float4 as two paired fp32 operations
+// (Blackwell's f32x2 pipe: per component the same rounding as fmulf / fmaf).
+__device__ __forceinline__ float4 mul4x(float a, float4 v) {
+  const float2 a2 = make_float2(a, a);
+  const float2 lo = __fmul2_rn(a2, make_float2(v.x, v.y));
+  const float2 hi = __fmul2_rn(a2, make_float2(v.z, v.w));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+__device__ __forceinline__ float4 fma4x(float x, float4 b, float4 v) {
+  const float2 x2 = make_float2(x, x);
+  const float2 lo = __ffma2_rn(x2, make_float2(b.x, b.y), make_float2(v.x, v.y));
+  const float2 hi = __ffma2_rn(x2, make_float2(b.z, b.w), make_float2(v.z, v.w));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
 // Load element i of a step input stored as T.
 template <typename T>
 __device__ __forceinline__ float ld_in(const void *base, int64_t i) {

@@ -323,8 +323,8 @@ struct GdnLayout {
       o += a128(d.NR * d.stage_floats * 4);
       d.off_db = o;
       o += a128(2 * d.db_floats * 4);
-      d.off_single = o;  // part [8][2][128] | z [2][128] | ucur [128]
-      o += a128((8 * 2 * 128 + 2 * 128 + 128) * 4);
+      d.off_single = o;  // part [8][2][128] | z [2][128] | ucur [128] | opart [128]
+      o += a128((8 * 2 * 128 + 2 * 128 + 2 * 128) * 4);
       d.off_ring = o;
       d.NS = (budget - o) / kHalfBytes;
       if (d.NS > 8) d.NS = 8;
@@ -341,7 +341,7 @@ struct GdnLayout {
 struct GdnPtrs {
   uint64_t *full, *empty, *rfull, *rempty;
   unsigned char *recK, *ring;
-  float *recU, *stage, *db, *part, *z, *ucur;
+  float *recU, *stage, *db, *part, *z, *ucur, *opart;
   __device__ GdnPtrs(unsigned char *smem, const GdnLayout &l) {
     full = reinterpret_cast<uint64_t *>(smem + l.off_bars);
     empty = full + 8;
@@ -354,6 +354,7 @@ struct GdnPtrs {
     part = reinterpret_cast<float *>(smem + l.off_single);
     z = part + 8 * 2 * 128;
     ucur = z + 2 * 128;
+    opart = ucur + 128;
     ring = smem + l.off_ring;
   }
 };
@@ -550,11 +551,16 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
         p.bbuf[bh * p.cap + k - 1] = beta;
       }
     }
-    if (warp == 0) {  // R_i = prod_{i<m<k} alpha_m (lane i), gamma, in fp64
-      double r = 1.0;
-      for (int m = lane + 1; m < k; ++m) r *= alpha[m];
-      if (lane < k) R[lane] = (float)r;
-      if (lane == 0) gam[0] = (float)(r * alpha[0]);
+    if (warp == 7) {  // R_i = prod_{i<m<k} alpha_m (lane i), gamma: fp64 suffix-product scan
+      double pr = lane < k ? (double)alpha[lane] : 1.0;  // inclusive: prod_{m >= lane}
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_down_sync(0xffffffffu, pr, o);
+        if (lane + o < 32) pr *= t;
+      }
+      const double nxt = __shfl_down_sync(0xffffffffu, pr, 1);  // prod_{m > lane}
+      if (lane < k) R[lane] = (float)(lane + 1 < 32 ? nxt : 1.0);
+      if (lane == 0) gam[0] = (float)pr;
     }
     {
       // 2k-1 dot products of 128: k_j.k_{k-1} (j < k-1) then k_i.q (i < k);
@@ -562,13 +568,16 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
       const int ndot = 2 * k - 1;
       for (int base = 0; base < ndot; base += kThreads / 16) {
         const int d = base + (tid >> 4), c0 = (tid & 15) * 8;
-        double acc = 0.0;
+        double acc = 0.0, acc1 = 0.0;  // two independent fp64 chains
         if (d < ndot) {
           const int i = d < k - 1 ? d : d - (k - 1);
           const float *other = d < k - 1 ? ks : qs;
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
+          for (int e = 0; e < 8; e += 2) {
             acc = fma((double)to_f32(rK[i * DKc + c0 + e]), (double)other[c0 + e], acc);
+            acc1 = fma((double)to_f32(rK[i * DKc + c0 + e + 1]), (double)other[c0 + e + 1], acc1);
+          }
+          acc += acc1;
         }
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
@@ -629,31 +638,45 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
       S.z[vsel * 128 + c] = acc;
     }
     bar_sync(1, kThreads);
-    // ---- P4: u of this record, the output (one column per thread)
-    if (tid < 128) {
-      const int c = tid;
+    // ---- P4: threads 0-127 form u of this record (column c), threads 128-255
+    // the output's terms over the older records; then the output's last term
+    // needs u, exchanged through shared memory.
+    {
+      const int c = tid & 127;
       const float g = gam[0];
-      float acc = vs[c] - g * S.z[c];
-      for (int j = 0; j < k - 1; ++j) acc = fmaf(-R[j] * kk[j], rU[j * DVc + c], acc);
-      const float u = beta * acc;
-      float o = g * S.z[128 + c];
-      for (int i = 0; i < k - 1; ++i) o = fmaf(R[i] * kq[i], rU[i * DVc + c], o);
-      o = fmaf(kq[k - 1], u, o);  // R_{k-1} = 1
+      if (tid < 128) {
+        float a0 = vs[c] - g * S.z[c], a1 = 0.f;
+        int j = 0;
+        for (; j + 1 < k - 1; j += 2) {
+          a0 = fmaf(-R[j] * kk[j], rU[j * DVc + c], a0);
+          a1 = fmaf(-R[j + 1] * kk[j + 1], rU[(j + 1) * DVc + c], a1);
+        }
+        if (j < k - 1) a0 = fmaf(-R[j] * kk[j], rU[j * DVc + c], a0);
+        const float u = beta * (a0 + a1);
+        if (!flush) p.ubuf[(bh * p.cap + k - 1) * DVc + c] = u;
+        S.ucur[c] = u;
+      } else {
+        float o0 = g * S.z[128 + c], o1 = 0.f;
+        int i = 0;
+        for (; i + 1 < k - 1; i += 2) {
+          o0 = fmaf(R[i] * kq[i], rU[i * DVc + c], o0);
+          o1 = fmaf(R[i + 1] * kq[i + 1], rU[(i + 1) * DVc + c], o1);
+        }
+        if (i < k - 1) o0 = fmaf(R[i] * kq[i], rU[i * DVc + c], o0);
+        S.opart[c] = o0 + o1;
+      }
+    }
+    bar_sync(1, kThreads);
+    if (tid >= 128) {
+      const int c = tid - 128;
+      const float o = fmaf(kq[k - 1], S.ucur[c], S.opart[c]);  // R_{k-1} = 1
       p.y[b * p.bs_y + (size_t)h * DVc + c] = p.scale * o;
-      if (!flush) p.ubuf[(bh * p.cap + k - 1) * DVc + c] = u;
-      S.ucur[c] = u;
     }
     // ---- P5 (flush): h0 <- gamma h0 + sum_i R_i k_i u_i^T, written once
     if (flush) {
-      bar_sync(1, kThreads);
       const float g = gam[0];
 #pragma unroll
-      for (int rho = 0; rho < 16; ++rho) {
-        hv[rho].x *= g;
-        hv[rho].y *= g;
-        hv[rho].z *= g;
-        hv[rho].w *= g;
-      }
+      for (int rho = 0; rho < 16; ++rho) hv[rho] = mul4x(g, hv[rho]);
       for (int i = 0; i < k; ++i) {
         const float4 ui = *reinterpret_cast<const float4 *>(
             i < k - 1 ? &rU[i * DVc + 4 * lane] : &S.ucur[4 * lane]);
@@ -663,13 +686,7 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
           const float4 k4 = *reinterpret_cast<const float4 *>(&Kf[i * DKc + row0 + 4 * t]);
           const float kr[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float w = ri * kr[e];
-            hv[4 * t + e].x = fmaf(w, ui.x, hv[4 * t + e].x);
-            hv[4 * t + e].y = fmaf(w, ui.y, hv[4 * t + e].y);
-            hv[4 * t + e].z = fmaf(w, ui.z, hv[4 * t + e].z);
-            hv[4 * t + e].w = fmaf(w, ui.w, hv[4 * t + e].w);
-          }
+          for (int e = 0; e < 4; ++e) hv[4 * t + e] = fma4x(ri * kr[e], ui, hv[4 * t + e]);
         }
       }
       float *dst = p.h0 + bh * (DKc * DVc);

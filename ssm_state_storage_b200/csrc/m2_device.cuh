@@ -407,21 +407,6 @@ __device__ __forceinline__ void store_row(float *tile, int r, int c8, const floa
   for (int s = 0; s < N / 32; ++s) st_stream(tile + (size_t)r * N + 32 * s + 4 * c8, v[s]);
 }
 
-// v <- a * v and v <- x * b + v on a float4 as two paired fp32 operations
-// (Blackwell's f32x2 pipe: per component the same rounding as fmulf / fmaf).
-__device__ __forceinline__ float4 mul4x(float a, float4 v) {
-  const float2 a2 = make_float2(a, a);
-  const float2 lo = __fmul2_rn(a2, make_float2(v.x, v.y));
-  const float2 hi = __fmul2_rn(a2, make_float2(v.z, v.w));
-  return make_float4(lo.x, lo.y, hi.x, hi.y);
-}
-__device__ __forceinline__ float4 fma4x(float x, float4 b, float4 v) {
-  const float2 x2 = make_float2(x, x);
-  const float2 lo = __ffma2_rn(x2, make_float2(b.x, b.y), make_float2(v.x, v.y));
-  const float2 hi = __ffma2_rn(x2, make_float2(b.z, b.w), make_float2(v.z, v.w));
-  return make_float4(lo.x, lo.y, hi.x, hi.y);
-}
-
 // The fold of RGC register-held rows of one head:
 //   v[u] <- lam v[u] + sum_{i<k} (w_i x_i[rows[u]]) B_i[cols],
 // record loop outermost so that each B_i fragment (fp32 in shared memory) is

@@ -81,10 +81,10 @@ struct VerifyLayout {
       o += d.NR * d.dBC_b;
       d.off_rec = o;
       o += a128(d.NR * d.rec_floats * 4);
-      // per consumer group: item scratch | bc [4][cap+4] double | cf [4][hc][cap+4] float
+      // per consumer group: item scratch | bc [4][cap+4] double | wd [4][hc][cap+4] double
       d.off_scr = o;
       d.db_b = a128(d.db_floats * 4);
-      d.scr_b = d.db_b + a128(kMD * (cap + kMD) * 8 + kMD * hc * (cap + kMD) * 4);
+      d.scr_b = d.db_b + a128(kMD * (cap + kMD) * 8 + kMD * hc * (cap + kMD) * 8);
       o += kVGroups * d.scr_b;
       d.off_ring = o;
       d.NS = (budget - o) / d.tile_stride;
@@ -308,7 +308,7 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
   const int h16 = lane >> 4, c16 = lane & 15;
   unsigned char *scr = smem + lay.off_scr + grp * lay.scr_b;
   double *bc = reinterpret_cast<double *>(scr + lay.db_b);  // [4][R]
-  float *cf = reinterpret_cast<float *>(bc + kMD * R);     // [4][hc][R] coefficients
+  double *wd = bc + kMD * R;                                // [4][hc][R] decay weights
   // Ring hand-off: a group starts waiting for its item's first tile only after
   // every warp of the other group has acquired the previous item's last
   // tile (turn[grp]), so a slot is never awaited more than one phase ahead.
@@ -374,33 +374,17 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
     const int n1 = hdr[1], nb = hdr[3], K = nb + nd;
     const bool fold = hdr[2];
 
-    // ---- S1: append the drafts (16-byte chunks); fp32 B for the fold;
-    // B_i . C_d in fp64
-    {
-      constexpr int XC = P * (int)sizeof(TI) / 16, BC = N * (int)sizeof(TI) / 16;
-      for (int c = gtid; c < nd * hc * XC; c += kGThreads) {
-        const int row = c / XC, k = c - row * XC, d = row / hc, j = row - d * hc;
-        reinterpret_cast<uint4 *>(static_cast<TI *>(p.xbuf) + ((bh0 + j) * cap + nb + d) * P)[k] =
-            reinterpret_cast<const uint4 *>(dX + (size_t)row * P)[k];
-      }
-      if (own_bc)
-        for (int c = gtid; c < 2 * nd * BC; c += kGThreads) {
-          const int which = c / (nd * BC), cc = c - which * (nd * BC), d = cc / BC, k = cc - d * BC;
-          TI *dst = static_cast<TI *>(which ? p.Cbuf : p.Bbuf) + (bg * cap + nb + d) * N;
-          reinterpret_cast<uint4 *>(dst)[k] =
-              reinterpret_cast<const uint4 *>((which ? dC : dB) + (size_t)d * N)[k];
-        }
-      if (gtid < nd * hc) {
-        const int d = gtid / hc, j = gtid - (gtid / hc) * hc;
-        p.dtbuf[(bh0 + j) * cap + nb + d] = dtd[d * hc + j];
-      }
+    // ---- S1 (warps 8-15): fp32 B for the fold, B_i . C_d in fp64; alongside,
+    // S2 (warps 0-7): the decay weights, then the draft appends.
+    if (gw >= kGWarps / 2) {
+      const int t2 = gtid - kGThreads / 2;
       if (fold)
-        for (int e = gtid; e < n1 * (N / 4); e += kGThreads)
+        for (int e = t2; e < n1 * (N / 4); e += kGThreads / 2)
           reinterpret_cast<float4 *>(Bf)[e] = ld_vec4<TI>(recB + 4 * e);
       const int npair = nd * K;  // (d, i) with i <= nb + d are used
       constexpr int PER = N / 16;
-      for (int base = 0; base < npair; base += kGThreads / 16) {
-        const int pr = base + (gtid >> 4), c0 = (gtid & 15) * PER;
+      for (int base = 0; base < npair; base += kGThreads / 32) {
+        const int pr = base + (t2 >> 4), c0 = (t2 & 15) * PER;
         const int d = pr / K, i = pr - d * K;
         const bool use = pr < npair && i <= nb + d;
         double acc = 0.0;
@@ -419,7 +403,81 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
         acc += __shfl_xor_sync(0xffffffffu, acc, 4);
         acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-        if (use && (gtid & 15) == 0) bc[d * R + i] = acc;
+        if (use && (t2 & 15) == 0) bc[d * R + i] = acc;
+      }
+    } else {
+      // ---- S2 (one warp per head): decay weights from fp64 suffix sums.
+      // Draft sequence: the nb committed records, then the nd drafts; with
+      // S_l = sum_{m >= l} dt_m, draft d (records 0..e, e = nb + d) weighs
+      // record i by exp(A (S_{i+1} - S_{e+1})) dt_i and the checkpoint by
+      // exp(A (S_0 - S_{e+1})).  Both factor through the reference point
+      // S_ref = S_{nb+1}:  exp(A (S_{i+1} - S_ref)) * exp(A (S_ref - S_{e+1})),
+      // so one exponential per lane serves every draft: lanes 0..K-1 take
+      // E_l = exp(A (S_{l+1} - S_ref)), lanes 27..30 take F_d = exp(A (S_ref -
+      // S_{e+1})) and lane 31 takes G = exp(A (S_0 - S_ref)).  No factor can
+      // overflow: S_ref - S_{e+1} and the S_{i+1} - S_ref of draft records span
+      // at most 4 dt, and every other argument is <= 0.  The fold sequence is
+      // the n1 committed records (weights exp(A S'_{l+1}) dt_l, decay
+      // exp(A S'_0)); both scans and both exponentials run side by side.
+      for (int j = gw; j < hc; j += kGWarps / 2) {
+        const double A = As[j];
+        const double dts = lane < nb ? (double)dtb[j * cap + lane]
+                                     : (lane < K ? (double)dtd[(lane - nb) * hc + j] : 0.0);
+        const double dtf = fold && lane < n1 ? (double)dtb[j * cap + lane] : 0.0;
+        double Ss = dts, Sf = dtf;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const double ts = __shfl_down_sync(0xffffffffu, Ss, o);
+          const double tf = __shfl_down_sync(0xffffffffu, Sf, o);
+          if (lane + o < 32) {
+            Ss += ts;
+            Sf += tf;
+          }
+        }
+        const double Ss1 = __shfl_down_sync(0xffffffffu, Ss, 1);  // S_{l+1}; lanes >= K: 0
+        const double Sf1 = __shfl_down_sync(0xffffffffu, Sf, 1);
+        const double Sref = __shfl_sync(0xffffffffu, Ss, nb + 1);  // nb + 1 <= cap < 27
+        const double S0 = __shfl_sync(0xffffffffu, Ss, 0);
+        const double Sf0 = __shfl_sync(0xffffffffu, Sf, 0);
+        const double SeL = __shfl_sync(0xffffffffu, Ss, (nb + (lane - 27) + 1) & 31);  // lanes 27..30
+        double arg = 0.0;
+        if (lane < K) arg = A * (Ss1 - Sref);
+        else if (lane >= 27 && lane < 31) arg = lane - 27 < nd ? A * (Sref - SeL) : 0.0;
+        else if (lane == 31) arg = A * (S0 - Sref);
+        const double ex = exp(arg);
+        const double exf = exp(A * (lane + 1 < n1 ? Sf1 : (lane == 31 ? Sf0 : 0.0)));  // n1 <= 20
+        if (fold) {
+          if (lane < n1) wf[j * cap + lane] = (float)(exf * dtf);
+          if (lane == 31) lamf[j] = (float)exf;
+        }
+        const double G = __shfl_sync(0xffffffffu, ex, 31);
+#pragma unroll
+        for (int d = 0; d < kMD; ++d) {
+          const double F = __shfl_sync(0xffffffffu, ex, 27 + d);
+          if (d < nd) {
+            if (lane <= nb + d) wd[(d * hc + j) * R + lane] = ex * F * dts;
+            if (lane == 0) lamd[d * hc + j] = (float)(G * F);
+          }
+        }
+      }
+      {
+        constexpr int XC = P * (int)sizeof(TI) / 16, BC = N * (int)sizeof(TI) / 16;
+        for (int c = gtid; c < nd * hc * XC; c += kGThreads / 2) {
+          const int row = c / XC, k = c - row * XC, d = row / hc, j = row - d * hc;
+          reinterpret_cast<uint4 *>(static_cast<TI *>(p.xbuf) + ((bh0 + j) * cap + nb + d) * P)[k] =
+              reinterpret_cast<const uint4 *>(dX + (size_t)row * P)[k];
+        }
+        if (own_bc)
+          for (int c = gtid; c < 2 * nd * BC; c += kGThreads / 2) {
+            const int which = c / (nd * BC), cc = c - which * (nd * BC), d = cc / BC, k = cc - d * BC;
+            TI *dst = static_cast<TI *>(which ? p.Cbuf : p.Bbuf) + (bg * cap + nb + d) * N;
+            reinterpret_cast<uint4 *>(dst)[k] =
+                reinterpret_cast<const uint4 *>((which ? dC : dB) + (size_t)d * N)[k];
+          }
+        if (gtid < nd * hc) {
+          const int d = gtid / hc, j = gtid - (gtid / hc) * hc;
+          p.dtbuf[(bh0 + j) * cap + nb + d] = dtd[d * hc + j];
+        }
       }
     }
     // draft C rows for this lane's columns, in registers for the whole item
@@ -429,79 +487,24 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
 #pragma unroll
       for (int s4 = 0; s4 < S4; ++s4) cr[d][s4] = ld_vec4<TI>(dC + d * N + 64 * s4 + 4 * c16);
     bar_sync(gbar, kGThreads);
-
-    // ---- S2 (one warp per head): decay weights from fp64 suffix sums.
-    // Draft sequence: the nb committed records, then the nd drafts; with
-    // S_l = sum_{m >= l} dt_m, draft d (records 0..e, e = nb + d) weighs
-    // record i by exp(A (S_{i+1} - S_{e+1})) dt_i and the checkpoint by
-    // exp(A (S_0 - S_{e+1})).  Both factor through the reference point
-    // S_ref = S_{nb+1}:  exp(A (S_{i+1} - S_ref)) * exp(A (S_ref - S_{e+1})),
-    // so one exponential per lane serves every draft: lanes 0..K-1 take
-    // E_l = exp(A (S_{l+1} - S_ref)), lanes 27..30 take F_d = exp(A (S_ref -
-    // S_{e+1})) and lane 31 takes G = exp(A (S_0 - S_ref)).  No factor can
-    // overflow: S_ref - S_{e+1} and the S_{i+1} - S_ref of draft records span
-    // at most 4 dt, and every other argument is <= 0.  The fold sequence is
-    // the n1 committed records (weights exp(A S'_{l+1}) dt_l, decay
-    // exp(A S'_0)); both scans and both exponentials run side by side.
-    for (int j = gw; j < hc; j += kGWarps) {
-      const double A = As[j];
-      const double dts = lane < nb ? (double)dtb[j * cap + lane]
-                                   : (lane < K ? (double)dtd[(lane - nb) * hc + j] : 0.0);
-      const double dtf = fold && lane < n1 ? (double)dtb[j * cap + lane] : 0.0;
-      double Ss = dts, Sf = dtf;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const double ts = __shfl_down_sync(0xffffffffu, Ss, o);
-        const double tf = __shfl_down_sync(0xffffffffu, Sf, o);
-        if (lane + o < 32) {
-          Ss += ts;
-          Sf += tf;
-        }
-      }
-      const double Ss1 = __shfl_down_sync(0xffffffffu, Ss, 1);  // S_{l+1}; lanes >= K: 0
-      const double Sf1 = __shfl_down_sync(0xffffffffu, Sf, 1);
-      const double Sref = __shfl_sync(0xffffffffu, Ss, nb + 1);  // nb + 1 <= cap < 27
-      const double S0 = __shfl_sync(0xffffffffu, Ss, 0);
-      const double Sf0 = __shfl_sync(0xffffffffu, Sf, 0);
-      const double SeL = __shfl_sync(0xffffffffu, Ss, (nb + (lane - 27) + 1) & 31);  // lanes 27..30
-      double arg = 0.0;
-      if (lane < K) arg = A * (Ss1 - Sref);
-      else if (lane >= 27 && lane < 31) arg = lane - 27 < nd ? A * (Sref - SeL) : 0.0;
-      else if (lane == 31) arg = A * (S0 - Sref);
-      const double ex = exp(arg);
-      const double exf = exp(A * (lane + 1 < n1 ? Sf1 : (lane == 31 ? Sf0 : 0.0)));  // n1 <= 20
-      if (fold) {
-        if (lane < n1) wf[j * cap + lane] = (float)(exf * dtf);
-        if (lane == 31) lamf[j] = (float)exf;
-      }
-      const double G = __shfl_sync(0xffffffffu, ex, 31);
-#pragma unroll
-      for (int d = 0; d < kMD; ++d) {
-        const double F = __shfl_sync(0xffffffffu, ex, 27 + d);
-        if (d < nd) {
-          if (lane <= nb + d) cf[(d * hc + j) * R + lane] = (float)(ex * F * dts * bc[d * R + lane]);
-          if (lane == 0) lamd[d * hc + j] = (float)(G * F);
-        }
-      }
-    }
-    bar_sync(gbar, kGThreads);
     // ---- S3 (one warp per (draft, head) row, RZ rows of the head per lane):
-    // z[d][j][r] = sum_i cf[d][j][i] x_i[r] + D_j x_d[r]
+    // z[d][j][r] = sum_i c_i x_i[r] + D_j x_d[r], with the coefficient
+    // c_i = w_{d,i} (B_i . C_d) rounded once by lane i and broadcast
     for (int row = gw; row < nd * hc; row += kGWarps) {
       const int d = row / hc, j = row - d * hc;
-      const float *c = cf + (d * hc + j) * R;
+      const float cl = lane <= nb + d ? (float)(wd[(d * hc + j) * R + lane] * bc[d * R + lane]) : 0.f;
       float acc[RZ], xv[RZ];
 #pragma unroll
       for (int k = 0; k < RZ; ++k) acc[k] = 0.f;
       for (int i = 0; i < nb; ++i) {
         ld_vec<TI, RZ>(recX + (j * cap + i) * P + RZ * lane, xv);
-        const float ci = c[i];
+        const float ci = __shfl_sync(0xffffffffu, cl, i);
 #pragma unroll
         for (int k = 0; k < RZ; ++k) acc[k] = fmaf(ci, xv[k], acc[k]);
       }
       for (int i = nb; i <= nb + d; ++i) {
         ld_vec<TI, RZ>(dX + ((i - nb) * hc + j) * P + RZ * lane, xv);
-        const float ci = c[i];
+        const float ci = __shfl_sync(0xffffffffu, cl, i);
 #pragma unroll
         for (int k = 0; k < RZ; ++k) acc[k] = fmaf(ci, xv[k], acc[k]);
       }

@@ -276,7 +276,7 @@ __device__ __forceinline__ void decode_tiles(const M2Params &p, const DecodeLayo
                                              const DecodeSmemPtrs &S, volatile int *abort_flag,
                                              int nitems, int nchunk) {
   stream_tiles<P, N, QM>(p, S.full, S.empty, S.ring, lay.NS, lay.tile_stride, lay.tile_bytes,
-                         lay.hc, abort_flag, nitems, nchunk, 0);
+                         lay.hc, abort_flag, nitems, nchunk);
 }
 
 constexpr int kDecodeThreads = kThreads + 64;  // 8 consumer warps, tile producer, stager

@@ -497,49 +497,25 @@ __device__ __forceinline__ void item_coords(const M2Params &p, int item, int nch
 }
 
 // Tile producer (one thread): streams the checkpoint tiles (or their read
-// copies) of this CTA's items, in item order, into the NS-slot ring.  With
-// pf > 0 it also keeps an L2 prefetch pf tiles ahead of the ring, so HBM
-// keeps streaming while the consumers spend time on per-item work that does
-// not release ring slots.
+// copies) of this CTA's items, in item order, into the NS-slot ring.  (An L2
+// bulk prefetch running one or two items ahead of the ring made the verify
+// round 4-8% slower on B200, so there is none.)
 template <int P, int N, int QM>
 __device__ __forceinline__ void stream_tiles(const M2Params &p, uint64_t *full, uint64_t *empty,
                                              unsigned char *ring, int NS, int tile_stride,
                                              int tile_bytes, int hc, volatile int *abort_flag,
-                                             int nitems, int nchunk, int pf) {
+                                             int nitems, int nchunk) {
   auto src_of = [&](int item, int j) -> size_t {
     int b, g, chunk, h_first;
     item_coords(p, item, nchunk, hc, b, g, chunk, h_first);
     return (size_t)b * p.H + h_first + j;
   };
-  auto prefetch = [&](size_t bh) {
-    if constexpr (QM == 1) {
-      bulk_prefetch_l2(p.rc + bh * (size_t)(P * N), P * N);
-    } else if constexpr (QM == 2) {
-      bulk_prefetch_l2(p.rc + bh * (size_t)(P * N / 2), P * N / 2);
-      bulk_prefetch_l2(p.rc_scale + bh * (size_t)(P * N / 16), P * N / 16);
-    } else {
-      bulk_prefetch_l2(p.h0 + bh * (size_t)(P * N), P * N * 4);
-    }
-  };
-  int pitem = blockIdx.x, pj = 0;  // next tile to prefetch
-  auto prefetch_next = [&]() {
-    if (pitem < nitems) {
-      prefetch(src_of(pitem, pj));
-      if (++pj == hc) {
-        pj = 0;
-        pitem += gridDim.x;
-      }
-    }
-  };
-  if (pf > 0)
-    for (int k = 0; k < pf + NS; ++k) prefetch_next();
   int slot = 0;
   uint32_t sphase = 0;
   uint32_t issued = 0, parity = 0;  // per slot: a copy was issued / its phase parity
   bool failed = false;
   for (int item = blockIdx.x; item < nitems && !failed; item += gridDim.x) {
     for (int j = 0; j < hc; ++j) {
-      if (pf > 0) prefetch_next();
       if (*abort_flag || !mbar_wait(&empty[slot], sphase ^ 1)) {
         failed = true;
         break;

@@ -279,7 +279,7 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
   if (warp == kVWarps) {
     if (lane == 0)
       stream_tiles<P, N, 0>(p, full, empty, ring, lay.NS, lay.tile_stride, lay.tile_bytes, hc,
-                            abort_flag, nitems, lay.nchunk, hc);
+                            abort_flag, nitems, lay.nchunk);
     return;
   }
   if (warp == kVWarps + 1) {

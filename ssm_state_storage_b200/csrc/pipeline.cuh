@@ -73,12 +73,6 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
-// Hint that `bytes` of global memory at `src` will be read soon: a bulk
-// prefetch into L2 (no completion to wait for; 16-byte aligned, bytes % 16 == 0).
-__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
 // Order this thread's generic-proxy shared-memory accesses before later
 // async-proxy (bulk copy) writes to the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -85,7 +85,7 @@ typedef enum { RSSM_FMT_NONE = 0, RSSM_FMT_FP8 = 1, RSSM_FMT_NVFP4 = 2 } rssm_fm
 /* Static description of one SSM layer's decode state. */
 typedef struct {
   int32_t kind;      /* rssm_kind                                               */
-  int32_t batch;     /* B, sequences (>= 0)                                      */
+  int32_t batch;     /* B, sequences (>= 0; 0: every call returns RSSM_OK at once) */
   int32_t nheads;    /* H                                                        */
   int32_t headdim;   /* Mamba-2 P (64 or 128); GDN DV (128)                      */
   int32_t dstate;    /* Mamba-2 N (64 or 128); GDN DK (128)                      */

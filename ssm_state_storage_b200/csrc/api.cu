@@ -227,6 +227,7 @@ const char *replayssm_last_cuda_error(void) { return cudaGetErrorString(g_last_c
 rssm_status replayssm_init(const rssm_desc *d, rssm_state *s, const float *S0, void *stream) {
   rssm_status st = check_desc(d);
   if (st != RSSM_OK) return st;
+  if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
   if ((st = check_state(d, s)) != RSSM_OK) return st;
   if (!S0) return RSSM_ERR_INVALID_ARG;
   cudaStream_t cs = to_stream(stream);
@@ -249,6 +250,7 @@ rssm_status replayssm_decode_step(const rssm_desc *d, rssm_state *s, const rssm_
                                   float *y, void *stream) {
   rssm_status st = check_desc(d);
   if (st != RSSM_OK) return st;
+  if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
   if ((st = check_state(d, s)) != RSSM_OK) return st;
   if (!y) return RSSM_ERR_INVALID_ARG;
   if (d->kind == RSSM_MAMBA2) {
@@ -268,6 +270,7 @@ rssm_status replayssm_flush(const rssm_desc *d, rssm_state *s, const float *A, i
                             void *stream) {
   rssm_status st = check_desc(d);
   if (st != RSSM_OK) return st;
+  if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
   if ((st = check_state(d, s)) != RSSM_OK) return st;
   if (d->kind == RSSM_MAMBA2) {
     if (!A) return RSSM_ERR_INVALID_ARG;
@@ -288,6 +291,7 @@ rssm_status replayssm_verify_commit(const rssm_desc *d, rssm_state *s,
   if (st != RSSM_OK) return st;
   if (d->kind != RSSM_MAMBA2) return RSSM_ERR_UNSUPPORTED;
   if (d->read_fmt != RSSM_FMT_NONE || d->ckpt_fmt != RSSM_FMT_NONE) return RSSM_ERR_UNSUPPORTED;
+  if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
   if ((st = check_state(d, s)) != RSSM_OK) return st;
   if (n_draft < 1 || n_draft > d->draft_max) return RSSM_ERR_CAPACITY;
   if (d->nheads / d->ngroups > 8) return RSSM_ERR_UNSUPPORTED;  // one CTA per group
@@ -312,6 +316,7 @@ rssm_status replayssm_commit(const rssm_desc *d, rssm_state *s, const int32_t *a
   rssm_status st = check_desc(d);
   if (st != RSSM_OK) return st;
   if (d->kind != RSSM_MAMBA2) return RSSM_ERR_UNSUPPORTED;
+  if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
   if ((st = check_state(d, s)) != RSSM_OK) return st;
   if (!accepted || !A) return RSSM_ERR_INVALID_ARG;
   M2Params p = m2_params(d, s);
@@ -325,6 +330,7 @@ rssm_status replayssm_full_decode_step(const rssm_desc *d, float *S, const rssm_
                                        void *stream) {
   rssm_status st = check_desc(d);
   if (st != RSSM_OK) return st;
+  if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
   if (!S || !y) return RSSM_ERR_INVALID_ARG;
   if (!aligned16(S)) return RSSM_ERR_ALIGNMENT;
   if (d->kind == RSSM_MAMBA2) {
@@ -350,6 +356,7 @@ rssm_status replayssm_materialize(const rssm_desc *d, const rssm_state *s, const
                                   float *S_out, void *stream) {
   rssm_status st = check_desc(d);
   if (st != RSSM_OK) return st;
+  if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
   if ((st = check_state(d, s)) != RSSM_OK) return st;
   if (!S_out) return RSSM_ERR_INVALID_ARG;
   if (!aligned16(S_out)) return RSSM_ERR_ALIGNMENT;

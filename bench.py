@@ -342,6 +342,8 @@ def run_ours(args, rank, world):
         torch.cuda.empty_cache()
         line["verify"] = bench_verify(args, dev, peak, rs, bm, wl, torch)
         torch.cuda.empty_cache()
+        line["read_copy"] = bench_readcopy(args, dev, peak, rs, bm, wl, torch, ms_per_window)
+        torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample()
     if rank == 0:
@@ -463,7 +465,7 @@ def bench_gdn(args, dev, peak, rs, bm, wl, torch):
     return {"workload": "gdn_serving", "value": tok / (ms_r * 1e-3), "unit": "tokens/s",
             "ms_per_window": ms_r / n,
             "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
-                         "frac": ach_r / peak, "kernel": "gdn_kernel<decode>"},
+                         "frac": ach_r / peak, "kernel": "gdn_decode_kernel"},
             "full_state": {"value": tok / (ms_f * 1e-3), "unit": "tokens/s",
                            "achieved_gbs": ach_f, "frac": ach_f / peak,
                            "kernel": "gdn_kernel<full>"},
@@ -471,6 +473,49 @@ def bench_gdn(args, dev, peak, rs, bm, wl, torch):
             "bytes_per_head_token": {"replay": wb / (w.B * w.H * L),
                                      "full_state": fb / (w.B * w.H * L)},
             "gpu_launches": n * L}
+
+
+def bench_readcopy(args, dev, peak, rs, bm, wl, torch, ms_fp32):
+    """m2_serving (batch 256) decoded with a low-precision read copy of the
+    checkpoint: every output reads the FP8 / NVFP4 copy instead of the fp32
+    checkpoint (which the flush fold still reads and writes)."""
+    w = wl.make(WORKLOAD)
+    L, pool = w.L, 4 * w.L
+    g = wl.Generator(w)
+    A, D = (t.to(dev) for t in g.params())
+    S0 = g.initial_state().to(dev)
+    st = {k: v.to(dev) for k, v in g.steps(pool).items()}
+    step_in = [dict(x=st["x"][t], dt=st["dt"][t], Bm=st["Bm"][t], Cm=st["Cm"][t], A=A, D=D)
+               for t in range(pool)]
+    y = torch.empty(w.B, w.H, w.P, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    n = args.sub_steps
+    out = {"workload": WORKLOAD, "note": "outputs read the copy; the fold keeps the fp32 checkpoint"}
+    for fmt in ("fp8", "nvfp4"):
+        layer = rs.Layer("m2", w.B, w.H, w.P, w.N, ngroups=w.G, window=L, in_dtype=w.in_dtype,
+                         read_fmt=fmt)
+        state = rs.ReplayState(layer, device=dev)
+        rs.replayssm_init(layer, state, S0)
+
+        def window(wi):
+            for j in range(L):
+                rs.replayssm_decode_step(layer, state, step_in[(wi * L + j) % pool], y, stream)
+
+        for i in range(3):
+            window(i)
+        ms = _events_ms(window, n, stream, torch, dev)
+        if state.status() != 0:
+            raise RuntimeError(f"device status {state.status()} after the {fmt} read-copy run")
+        wb = bm.m2_replay_window_bytes_rc(L, w.P, w.N, w.H // w.G, 2, fmt) * w.B * w.H
+        ach = wb / (ms / n * 1e-3) / 1e9
+        out[fmt] = {"value": w.B * L * n / (ms * 1e-3), "unit": "tokens/s", "ms_per_window": ms / n,
+                    "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                                 "frac": ach / peak, "kernel": "m2_decode_kernel (read copy)"},
+                    "bytes_per_head_token": wb / (w.B * w.H * L),
+                    "over_fp32_replay": ms_fp32 / (ms / n), "gpu_launches": n * L}
+        del state
+        torch.cuda.empty_cache()
+    return out
 
 
 def bench_verify(args, dev, peak, rs, bm, wl, torch):

@@ -46,6 +46,31 @@ def m2_replay_window_bytes(L, P, N, hpg, in_bytes):
     return sum(m2_replay_bytes(k, L, P, N, hpg, in_bytes) for k in range(1, L + 1))
 
 
+def rc_tile_bytes(P, N, fmt):
+    """Bytes of one head's low-precision read copy: FP8 E4M3 codes, or NVFP4
+    E2M1 codes (two per byte) + one E4M3 scale per 16 elements + the fp32
+    per-tile scale."""
+    if fmt == "fp8":
+        return P * N
+    if fmt == "nvfp4":
+        return P * N // 2 + P * N // 16 + 4
+    raise ValueError(fmt)
+
+
+def m2_replay_bytes_rc(k, L, P, N, hpg, in_bytes, fmt):
+    """Replay step whose outputs read the low-precision copy instead of the
+    fp32 checkpoint: the copy replaces the fp32 read; on the flush step the fold
+    still reads and writes the fp32 checkpoint and writes the new copy."""
+    state = P * N * 4
+    rc = rc_tile_bytes(P, N, fmt)
+    flush = k == L
+    return m2_replay_bytes(k, L, P, N, hpg, in_bytes) - state + rc + ((state + rc) if flush else 0)
+
+
+def m2_replay_window_bytes_rc(L, P, N, hpg, in_bytes, fmt):
+    return sum(m2_replay_bytes_rc(k, L, P, N, hpg, in_bytes, fmt) for k in range(1, L + 1))
+
+
 def gdn_conventional_bytes(DK, DV, in_bytes):
     state = DK * DV * 4
     return 2 * state + (2 * DK + DV) * in_bytes + 8 + DV * 4

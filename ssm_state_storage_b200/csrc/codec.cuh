@@ -13,6 +13,7 @@
 // recurrence [sitech.ge, "NVIDIA ו-Dao AI Lab הציגו ReplaySSM…", §Bounding
 // quantisation error].
 #pragma once
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace rssm {
@@ -47,6 +48,27 @@ __device__ __forceinline__ float e2m1_decode(uint32_t c) {
   const uint32_t e = (c >> 1) & 3u, m = c & 1u;
   float mag = (e == 0) ? 0.5f * (float)m : __uint_as_float(((e + 126u) << 23) | (m << 22));
   return (c & 8u) ? -mag : mag;
+}
+
+// Two E4M3 codes (bits 0-7 and 8-15 of `two`) -> their values, by the
+// hardware conversion to f16x2 (every E4M3 value is exact in f16); the low
+// byte lands in .x.
+__device__ __forceinline__ float2 e4m3x2_decode(uint32_t two) {
+  uint32_t h2;
+  asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.f16x2.e4m3x2 %0, t;\n}"
+      : "=r"(h2)
+      : "r"(two));
+  return __half22float2(*reinterpret_cast<const __half2 *>(&h2));
+}
+
+// Two E2M1 codes packed in one byte (lo nibble first) -> their values, by
+// the hardware conversion to f16x2 (exact).
+__device__ __forceinline__ float2 e2m1x2_decode(uint32_t byte) {
+  uint32_t h2;
+  asm("{\n .reg .b8 t;\n cvt.u8.u32 t, %1;\n cvt.rn.f16x2.e2m1x2 %0, t;\n}"
+      : "=r"(h2)
+      : "r"(byte));
+  return __half22float2(*reinterpret_cast<const __half2 *>(&h2));
 }
 
 __device__ __forceinline__ float nvfp4_tile_scale(float amax) {

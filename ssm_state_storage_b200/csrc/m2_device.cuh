@@ -382,13 +382,16 @@ __device__ __forceinline__ void view_row(const unsigned char *t, int r, int c8, 
     const int c = 32 * s + 4 * c8;
     if constexpr (QM == 1) {
       const uint32_t w = *reinterpret_cast<const uint32_t *>(t + r * N + c);
-      v[s] = make_float4(e4m3_decode(w & 0xFF), e4m3_decode((w >> 8) & 0xFF),
-                         e4m3_decode((w >> 16) & 0xFF), e4m3_decode(w >> 24));
+      const float2 lo = e4m3x2_decode(w & 0xFFFFu), hi = e4m3x2_decode(w >> 16);
+      v[s] = make_float4(lo.x, lo.y, hi.x, hi.y);
     } else if constexpr (QM == 2) {
+      // value = (E2M1 * s_b) * s_g: the first product is exact, the second
+      // rounded once (as nvfp4_value)
       const uint32_t w = *reinterpret_cast<const uint16_t *>(t + r * (N / 2) + c / 2);
       const float sb = e4m3_decode(t[P * N / 2 + r * (N / 16) + c / 16]);
-      v[s] = make_float4(nvfp4_value(w & 0xF, sb, sg), nvfp4_value((w >> 4) & 0xF, sb, sg),
-                         nvfp4_value((w >> 8) & 0xF, sb, sg), nvfp4_value((w >> 12) & 0xF, sb, sg));
+      const float2 lo = e2m1x2_decode(w & 0xFFu), hi = e2m1x2_decode(w >> 8);
+      v[s] = make_float4(__fmul_rn(lo.x * sb, sg), __fmul_rn(lo.y * sb, sg),
+                         __fmul_rn(hi.x * sb, sg), __fmul_rn(hi.y * sb, sg));
     } else {
       v[s] = *reinterpret_cast<const float4 *>(t + (r * N + c) * 4);
     }

@@ -99,3 +99,23 @@ def test_low_precision_outputs_match_oracle(kind, fmt):
         c = torch.empty(h.shape, dtype=torch.uint8, device="cuda")
         rs.replayssm_quantize("fp8", h, c)
         np.testing.assert_array_equal(oracle.fp8_dequant(c.cpu().numpy()), h.cpu().numpy())
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+def test_read_copy_full_batch_sampled(fmt):
+    """m2_readcopy at its batch of 64 (many work items per CTA, the read-copy
+    ring layout) over 20 steps including a flush; 2 sequences checked."""
+    w = wl.make("m2_readcopy")
+    g = wl.Generator(w)
+    A, D = g.params()
+    S0 = g.initial_state()
+    st = g.steps(20)
+    got = _gpu.m2_replay_run(w, A, D, S0, st, layer=_gpu.layer_for(w, read_fmt=fmt))
+    assert got["state"].status() == 0
+    seqs = [0, 63]
+    sub = {k: v[:, seqs] for k, v in st.items()}
+    orc = oracle.M2Replay(S0[seqs], G=w.G, L=w.L, read_fmt=fmt)
+    y, lt, _ = orc.decode(sub["x"], sub["dt"], sub["Bm"], sub["Cm"], A, D)
+    assert np.array_equal(got["len"][:, seqs], lt)
+    errs = [norm_err(a, b) for a, b in zip(got["y"][:, seqs], y)]
+    assert max(errs) < BOUND[fmt], max(errs)

@@ -92,6 +92,24 @@ def recorded_traffic(batch):
     return float(kv["traffic_bytes_per_launch"])
 
 
+def max_over_ranks(ms, world, device=None):
+    """The slowest rank's time: every rank takes part in one MAX all-reduce
+    (a no-op with one rank).  Times are device times from CUDA events."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, tokens_per_rank, ms_max):
+    """Whole-job throughput of independent replicas: all ranks' tokens over the
+    slowest rank's time (weak scaling: per-rank work is fixed)."""
+    return world * tokens_per_rank / (ms_max * 1e-3)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -272,12 +290,7 @@ def run_ours(args, rank, world):
             fn(offset + i)
         e1.record(stream)
         barrier()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(e0.elapsed_time(e1), world, dev)
 
     for i in range(args.warmup):
         replay_window(i)
@@ -305,8 +318,8 @@ def run_ours(args, rank, world):
     achieved = win_bytes / (ms_per_window * 1e-3) / 1e9
     achieved_full = full_bytes / (ms_per_window_full * 1e-3) / 1e9
     peak, peak_src = peaks()
-    value = world * tok_per_step * args.steps / (ms_replay * 1e-3)
-    value_full = world * tok_per_step * args.steps / (ms_full * 1e-3)
+    value = job_tokens_per_s(world, tok_per_step * args.steps, ms_replay)
+    value_full = job_tokens_per_s(world, tok_per_step * args.steps, ms_full)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -401,14 +414,10 @@ def run_e2e(args, w, layer, state, st, Ad, Dd, dev, world, rs, torch, dist):
     s_in.wait_stream(s_out)
     e1.record(s_in)
     torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     if state.status() != 0:
         raise RuntimeError(f"device status {state.status()} after the e2e run")
-    return {"value": world * w.B * n_steps / (ms * 1e-3), "unit": "tokens/s",
+    return {"value": job_tokens_per_s(world, w.B * n_steps, ms), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d * L, "d2h_bytes_per_step": d2h * L,
             "steps": args.e2e_steps, "pipelined": "H2D / decode / D2H on three streams"}
 

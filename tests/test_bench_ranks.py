@@ -1,0 +1,47 @@
+"""bench.py's multi-rank timing on the CPU: two gloo ranks, each with its own
+device time; every rank gets the slowest one, and the job value counts the
+tokens of all ranks over that time (independent replicas, weak scaling)."""
+import os
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _rank(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        ms = [12.5, 20.0][rank]
+        slowest = bench.max_over_ranks(ms, world)
+        dist.barrier()
+        out.put((rank, slowest, bench.job_tokens_per_s(world, 4096 * 10, slowest)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_slowest_time():
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = 29500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(out.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [20.0, 20.0]
+    assert res[0][2] == pytest.approx(2 * 4096 * 10 / 20e-3)
+
+
+def test_one_rank_is_a_no_op():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+    assert bench.job_tokens_per_s(1, 4096, 2.0) == pytest.approx(4096 / 2e-3)

@@ -200,7 +200,14 @@ rssm_status replayssm_flush(const rssm_desc *desc, rssm_state *state, const floa
  *      (len itself is not advanced);
  *   3. y[b][d][h][p] = output of draft d evaluated from h0 and the len+d+1
  *      records, without forming any intermediate state.
- * accepted_prev [B] int32 in 0..draft_max.  1 <= n_draft <= draft_max. */
+ * accepted_prev [B] int32 in 0..draft_max.  1 <= n_draft <= draft_max.
+ * The draft rows of x, Bm and Cm are bulk-copied by the kernel: their base
+ * pointers and batch strides (in bytes) must be multiples of 16, else
+ * RSSM_ERR_ALIGNMENT is returned before any launch.  H/G <= 8, else
+ * RSSM_ERR_UNSUPPORTED.  Errors found on the device (a length out of range,
+ * heads of a group out of step, accepted_prev[b] > draft_max, a round that
+ * would overrun the capacity) set *status to RSSM_ERR_STATE and leave that
+ * (sequence, group) untouched. */
 rssm_status replayssm_verify_commit(const rssm_desc *desc, rssm_state *state,
                                     const int32_t *accepted_prev, const rssm_step_in *drafts,
                                     int32_t n_draft, float *y, void *stream);

@@ -47,40 +47,6 @@ struct Tile {
 
 // ---------------------------------------------------------------- read copy
 
-// Load the read view of a head tile from its low-precision copy.
-template <int P, int N, int QM>
-__device__ __forceinline__ void load_read_view(const M2Params &p, size_t bh, int warp, int rs,
-                                               int c8, float4 (&v)[P / 32][N / 32]) {
-  using T = Tile<P, N>;
-  if constexpr (QM == 1) {
-    const uint8_t *rc = p.rc + bh * (size_t)(P * N);
-#pragma unroll
-    for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-      for (int s = 0; s < T::C4; ++s) {
-        const int r = T::row(warp, rs, rho), c = T::col(c8, s);
-        const uint32_t w = *reinterpret_cast<const uint32_t *>(rc + (size_t)r * N + c);
-        v[rho][s] = make_float4(e4m3_decode(w & 0xFF), e4m3_decode((w >> 8) & 0xFF),
-                                e4m3_decode((w >> 16) & 0xFF), e4m3_decode(w >> 24));
-      }
-  } else {
-    const uint8_t *rc = p.rc + bh * (size_t)(P * N / 2);
-    const uint8_t *sc = p.rc_scale + bh * (size_t)(P * N / 16);
-    const float sg = p.rc_gscale[bh];
-#pragma unroll
-    for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-      for (int s = 0; s < T::C4; ++s) {
-        const int r = T::row(warp, rs, rho), c = T::col(c8, s);
-        const uint32_t w = *reinterpret_cast<const uint16_t *>(rc + (size_t)r * (N / 2) + c / 2);
-        const float sb = e4m3_decode(sc[(size_t)r * (N / 16) + c / 16]);
-        v[rho][s] = make_float4(nvfp4_value(w & 0xF, sb, sg), nvfp4_value((w >> 4) & 0xF, sb, sg),
-                                nvfp4_value((w >> 8) & 0xF, sb, sg),
-                                nvfp4_value((w >> 12) & 0xF, sb, sg));
-      }
-  }
-}
-
 // Quantise a register tile after a fold.  fmt 1 = FP8, 2 = NVFP4.  With
 // roundtrip the values are replaced by deq(Q(v)) (quantised checkpoint);
 // otherwise the codes are written to the read copy.  Must be called by every
@@ -250,60 +216,6 @@ __device__ __forceinline__ void fold_regs(float4 (&hv)[P / 32][N / 32], float la
       }
     }
   }
-}
-
-// The fold with the record loop outermost: each B_i fragment (fp32 in shared
-// memory) is loaded once and used for all of the thread's rows.
-template <int P, int N, typename TI>
-__device__ __forceinline__ void fold_regs_hoisted(float4 (&hv)[P / 32][N / 32], float lam, int k,
-                                                  const float *wdt, const TI *x, const float *Bf,
-                                                  int warp, int rs, int c8) {
-  using T = Tile<P, N>;
-#pragma unroll
-  for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s) {
-      hv[rho][s].x *= lam;
-      hv[rho][s].y *= lam;
-      hv[rho][s].z *= lam;
-      hv[rho][s].w *= lam;
-    }
-  // two accumulation chains (even / odd records): shorter rounding chains and
-  // independent FMA streams
-  float4 acc[T::RPT][T::C4];
-#pragma unroll
-  for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s) acc[rho][s] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i = 0; i < k; ++i) {
-    float4 bb[T::C4];
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s)
-      bb[s] = *reinterpret_cast<const float4 *>(&Bf[i * N + T::col(c8, s)]);
-    const float w = wdt[i];
-    const bool odd = i & 1;
-#pragma unroll
-    for (int rho = 0; rho < T::RPT; ++rho) {
-      const float xw = w * to_f32(x[i * P + T::row(warp, rs, rho)]);
-#pragma unroll
-      for (int s = 0; s < T::C4; ++s) {
-        float4 &d = odd ? acc[rho][s] : hv[rho][s];
-        d.x = fmaf(xw, bb[s].x, d.x);
-        d.y = fmaf(xw, bb[s].y, d.y);
-        d.z = fmaf(xw, bb[s].z, d.z);
-        d.w = fmaf(xw, bb[s].w, d.w);
-      }
-    }
-  }
-#pragma unroll
-  for (int rho = 0; rho < T::RPT; ++rho)
-#pragma unroll
-    for (int s = 0; s < T::C4; ++s) {
-      hv[rho][s].x += acc[rho][s].x;
-      hv[rho][s].y += acc[rho][s].y;
-      hv[rho][s].z += acc[rho][s].z;
-      hv[rho][s].w += acc[rho][s].w;
-    }
 }
 
 // After a fold: round the checkpoint (qmode 3/4), store it, refresh the read

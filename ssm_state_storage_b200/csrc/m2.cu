@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
       for (int c0 = 0; c0 < RG; c0 += RGC) {
         float4 v[RGC][C4];
 #pragma unroll
-        for (int u = 0; u < RGC; ++u) view_row<P, N, QM>(t, sub * RW + 4 * (c0 + u) + rs, c8, sg, v[u]);
+        for (int u = 0; u < RGC; ++u) view_row<P, N, QM>(t, sub * RW + 4 * (c0 + u) + rs, c8, v[u]);
         if (c0 + RGC == RG) {  // all of this warp's rows are in registers
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.empty[sl]);
@@ -472,7 +472,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
         for (int u = 0; u < RGC; ++u) rows[u] = sub * RW + 4 * (c0 + u) + rs;
 #pragma unroll
         for (int u = 0; u < RGC; ++u) {
-          const float a = sum8(tree_dot<C4>(v[u], c4));
+          float a = sum8(tree_dot<C4>(v[u], c4));
+          if constexpr (QM == 2) a *= sg;  // the NVFP4 view leaves the tile scale out
           if (c8 == 0) yout[rows[u]] = fmaf(lm, a, zj[rows[u]]);
         }
         if (flush) {

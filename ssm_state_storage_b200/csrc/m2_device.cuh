@@ -284,10 +284,11 @@ struct DecodeSmem {
 
 // ------------------------------------------------------------- row helpers
 // One row of a P x N head tile as seen by one lane of the decode kernel:
-// columns 32 s + 4 c8 (s < N/32), four values each.
+// columns 32 s + 4 c8 (s < N/32), four values each (for an NVFP4 copy
+// without its per-tile scale).
 
 template <int P, int N, int QM>
-__device__ __forceinline__ void view_row(const unsigned char *t, int r, int c8, float sg,
+__device__ __forceinline__ void view_row(const unsigned char *t, int r, int c8,
                                          float4 (&v)[N / 32]) {
 #pragma unroll
   for (int s = 0; s < N / 32; ++s) {
@@ -297,13 +298,12 @@ __device__ __forceinline__ void view_row(const unsigned char *t, int r, int c8, 
       const float2 lo = e4m3x2_decode(w & 0xFFFFu), hi = e4m3x2_decode(w >> 16);
       v[s] = make_float4(lo.x, lo.y, hi.x, hi.y);
     } else if constexpr (QM == 2) {
-      // value = (E2M1 * s_b) * s_g: the first product is exact, the second
-      // rounded once (as nvfp4_value)
+      // E2M1 * s_b (exact in fp32); the per-tile scale s_g is left to the
+      // caller, which applies it once to each row's dot product
       const uint32_t w = *reinterpret_cast<const uint16_t *>(t + r * (N / 2) + c / 2);
       const float sb = e4m3_decode(t[P * N / 2 + r * (N / 16) + c / 16]);
       const float2 lo = e2m1x2_decode(w & 0xFFu), hi = e2m1x2_decode(w >> 8);
-      v[s] = make_float4(__fmul_rn(lo.x * sb, sg), __fmul_rn(lo.y * sb, sg),
-                         __fmul_rn(hi.x * sb, sg), __fmul_rn(hi.y * sb, sg));
+      v[s] = make_float4(lo.x * sb, lo.y * sb, hi.x * sb, hi.y * sb);
     } else {
       v[s] = *reinterpret_cast<const float4 *>(t + (r * N + c) * 4);
     }

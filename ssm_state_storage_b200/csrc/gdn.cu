@@ -568,14 +568,16 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
       const int ndot = 2 * k - 1;
       for (int base = 0; base < ndot; base += kThreads / 16) {
         const int d = base + (tid >> 4), c0 = (tid & 15) * 8;
-        double acc = 0.0, acc1 = 0.0;  // two independent fp64 chains
+        // products in fp32 (exact for bf16 inputs: 8 x 8 significant bits),
+        // sums in fp64 over two independent chains
+        double acc = 0.0, acc1 = 0.0;
         if (d < ndot) {
           const int i = d < k - 1 ? d : d - (k - 1);
           const float *other = d < k - 1 ? ks : qs;
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
-            acc = fma((double)to_f32(rK[i * DKc + c0 + e]), (double)other[c0 + e], acc);
-            acc1 = fma((double)to_f32(rK[i * DKc + c0 + e + 1]), (double)other[c0 + e + 1], acc1);
+            acc += (double)(to_f32(rK[i * DKc + c0 + e]) * other[c0 + e]);
+            acc1 += (double)(to_f32(rK[i * DKc + c0 + e + 1]) * other[c0 + e + 1]);
           }
           acc += acc1;
         }

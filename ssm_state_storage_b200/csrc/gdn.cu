@@ -631,23 +631,20 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
       *reinterpret_cast<float4 *>(&S.part[(warp * 2 + 1) * 128 + 4 * lane]) = pq;
     }
     bar_sync(1, kThreads);
-    // ---- P3: z = h0^T k, zq = h0^T q (fixed summation order over the warps)
-    {
-      const int vsel = tid >> 7, c = tid & 127;
-      float acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) acc += S.part[(w * 2 + vsel) * 128 + c];
-      S.z[vsel * 128 + c] = acc;
-    }
-    bar_sync(1, kThreads);
+    // ---- P3 (fused into P4): each thread sums the 8 warps' partials of its
+    // own column, z = h0^T k for threads 0-127, zq = h0^T q for 128-255, in a
+    // fixed order, so no barrier is needed between the two
     // ---- P4: threads 0-127 form u of this record (column c), threads 128-255
     // the output's terms over the older records; then the output's last term
     // needs u, exchanged through shared memory.
     {
-      const int c = tid & 127;
+      const int vsel = tid >> 7, c = tid & 127;
       const float g = gam[0];
+      float zc = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) zc += S.part[(w * 2 + vsel) * 128 + c];
       if (tid < 128) {
-        float a0 = vs[c] - g * S.z[c], a1 = 0.f;
+        float a0 = vs[c] - g * zc, a1 = 0.f;
         int j = 0;
         for (; j + 1 < k - 1; j += 2) {
           a0 = fmaf(-R[j] * kk[j], rU[j * DVc + c], a0);
@@ -658,7 +655,7 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
         if (!flush) p.ubuf[(bh * p.cap + k - 1) * DVc + c] = u;
         S.ucur[c] = u;
       } else {
-        float o0 = g * S.z[128 + c], o1 = 0.f;
+        float o0 = g * zc, o1 = 0.f;
         int i = 0;
         for (; i + 1 < k - 1; i += 2) {
           o0 = fmaf(R[i] * kq[i], rU[i * DVc + c], o0);

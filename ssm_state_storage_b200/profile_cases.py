@@ -1,0 +1,64 @@
+"""Small fixed runs of one kernel each, for ncu captures (one kernel, a few
+launches, a checkpoint larger than the 126 MB L2, a few GB on the device):
+
+    python -m ssm_state_storage_b200.profile_cases verify [batch]
+        8 speculative verify rounds of m2_verify (default batch 64: a 256 MiB
+        checkpoint), the previous round's acceptance committed each round
+    python -m ssm_state_storage_b200.profile_cases gdn [batch]
+        20 decode steps of gdn_serving (default batch 64: a 512 MiB checkpoint)
+
+Each run checks the device status word and exits non-zero if it is set.
+"""
+import sys
+
+import torch
+
+from . import replayssm as rs
+from . import workloads as wl
+
+
+def verify(batch=64, rounds=8):
+    w = wl.make("m2_verify", B=batch)
+    g = wl.Generator(w)
+    A, D = (t.cuda() for t in g.params())
+    S0 = g.initial_state()
+    rd = {k: v.cuda() for k, v in g.rounds(rounds).items()}
+    layer = rs.Layer("m2", w.B, w.H, w.P, w.N, ngroups=w.G, window=w.L, draft_max=w.n_draft,
+                     in_dtype=w.in_dtype)
+    y = torch.empty(w.B, w.n_draft, w.H, w.P, device="cuda")
+    state = rs.ReplayState(layer)
+    rs.replayssm_init(layer, state, S0.cuda())
+    for r in range(rounds):
+        drafts = dict(x=rd["x"][r], dt=rd["dt"][r], Bm=rd["Bm"][r], Cm=rd["Cm"][r], A=A, D=D)
+        rs.replayssm_verify_commit(layer, state, rd["acc"][r - 1] if r else None, drafts, y)
+    torch.cuda.synchronize()
+    return state.status()
+
+
+def gdn(batch=64, steps=20):
+    w = wl.make("gdn_serving", B=batch)
+    g = wl.Generator(w)
+    S0 = g.initial_state()
+    st = {k: v.cuda() for k, v in g.steps(steps).items()}
+    layer = rs.Layer("gdn", w.B, w.H, w.P, w.N, window=w.L, in_dtype=w.in_dtype)
+    state = rs.ReplayState(layer)
+    rs.replayssm_init(layer, state, S0.cuda())
+    y = torch.empty(w.B, w.H, w.P, device="cuda")
+    for t in range(steps):
+        rs.replayssm_decode_step(layer, state, {k: st[k][t] for k in st}, y)
+    torch.cuda.synchronize()
+    return state.status()
+
+
+def main(argv):
+    cases = {"verify": verify, "gdn": gdn}
+    if len(argv) < 1 or argv[0] not in cases:
+        print(__doc__)
+        return 2
+    status = cases[argv[0]](*(int(a) for a in argv[1:2]))
+    print(argv[0], "status", status)
+    return 0 if status == 0 else 1
+
+
+if __name__ == "__main__":
+    sys.exit(main(sys.argv[1:]))

@@ -294,7 +294,8 @@ rssm_status replayssm_verify_commit(const rssm_desc *d, rssm_state *s,
   if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
   if ((st = check_state(d, s)) != RSSM_OK) return st;
   if (n_draft < 1 || n_draft > d->draft_max) return RSSM_ERR_CAPACITY;
-  if (d->nheads / d->ngroups > 8) return RSSM_ERR_UNSUPPORTED;  // one CTA per group
+  // the verify stager maps (draft, head) pairs of a work item onto one warp's lanes
+  if (d->nheads / d->ngroups > 8) return RSSM_ERR_UNSUPPORTED;
   if (!y) return RSSM_ERR_INVALID_ARG;
   if ((st = check_m2_inputs(drafts, true)) != RSSM_OK) return st;
   M2Params p = m2_params(d, s);

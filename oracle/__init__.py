@@ -49,6 +49,10 @@ def lib():
         L.oracle_gdn_replay.argtypes = [i, i, i, i, i, i, i, C.c_double, dp, dp, dp, dp, dp, dp,
                                         ip, dp, dp, dp, dp, dp, dp, ip, ip, lp, lp]
         L.oracle_gdn_flush.argtypes = [i, i, i, i, i, i, i, dp, dp, dp, dp, dp, ip]
+        L.oracle_gdn_verify_replay.argtypes = [i, i, i, i, i, i, i, i, C.c_double, dp, dp, dp,
+                                               dp, dp, dp, ip, dp, dp, dp, dp, dp, ip, dp, ip]
+        L.oracle_gdn_verify_snapshot.argtypes = [i, i, i, i, i, i, C.c_double, dp, dp, dp, dp,
+                                                 dp, dp, ip, dp, lp]
         L.oracle_gdn_materialize.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, ip, dp]
         L.oracle_e4m3_encode.argtypes = [C.c_float]
         L.oracle_e4m3_encode.restype = C.c_uint8
@@ -193,6 +197,21 @@ def gdn_conventional(S0, q, k, v, alpha, beta, scale=1.0):
     return o, S, rd, wr
 
 
+def gdn_verify_snapshot(S0, q, k, v, alpha, beta, acc, scale=1.0):
+    """Snapshot-and-restore speculative decoding of the full GDN state.
+    Returns (o[R,B,Dn,H,DV], S_final, state_copies[B,H])."""
+    S = _f64(S0).copy()
+    q, k, v, alpha, beta = map(_f64, (q, k, v, alpha, beta))
+    acc = _i32(acc)
+    R, B, Dn, H, DK = q.shape
+    DV = v.shape[-1]
+    o = np.zeros((R, B, Dn, H, DV))
+    copies = np.zeros((B, H), np.int64)
+    _check(lib().oracle_gdn_verify_snapshot(R, B, H, DK, DV, Dn, float(scale), S, q, k, v,
+                                            alpha, beta, acc, o, copies), "gdn_verify_snapshot")
+    return o, S, copies
+
+
 class GDNReplay:
     def __init__(self, h0, L=16, cap=None, scale=1.0):
         self.h0 = _f64(h0).copy()
@@ -225,6 +244,21 @@ class GDNReplay:
         _check(lib().oracle_gdn_flush(self.B, self.H, self.DK, self.DV, self.L, self.cap,
                                       int(force), self.h0, self.rec_k, self.rec_v,
                                       self.rec_alpha, self.rec_beta, self.len), "gdn_flush")
+
+    def verify(self, q, k, v, alpha, beta, acc):
+        """R speculative rounds: append Dn drafts, evaluate them output-only,
+        commit acc[r, b] of them.  q is [R,B,Dn,H,DK].  Returns (o, len_trace[R,B,H])."""
+        q, k, v, alpha, beta = map(_f64, (q, k, v, alpha, beta))
+        acc = _i32(acc)
+        R, B, Dn, H, _ = q.shape
+        o = np.zeros((R, B, Dn, H, self.DV))
+        lt = np.zeros((R, B, H), np.int32)
+        _check(lib().oracle_gdn_verify_replay(R, B, H, self.DK, self.DV, self.L, self.cap, Dn,
+                                              self.scale, self.h0, self.rec_q, self.rec_k,
+                                              self.rec_v, self.rec_alpha, self.rec_beta,
+                                              self.len, q, k, v, alpha, beta, acc, o, lt),
+               "gdn_verify_replay")
+        return o, lt
 
     def materialize(self):
         S = np.zeros_like(self.h0)

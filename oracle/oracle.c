@@ -503,6 +503,104 @@ int oracle_gdn_replay(int T, int B, int H, int DK, int DV, int L, int cap,
   return bad ? -1 : 0;
 }
 
+/* Speculative verify for Gated DeltaNet, replay form (the Mamba-2 round
+ * carried over to the delta rule, [sitech §Reducing state traffic...]): per
+ * round the Dn drafts are appended after the committed records, each draft's
+ * output is evaluated from h0 and records 0..len+d with no intermediate
+ * state, then the accepted prefix is committed by advancing len (rejected
+ * drafts stay behind, to be overwritten), folding when len reaches L.
+ * Drafts: q, k [R][B][Dn][H][DK], v [R][B][Dn][H][DV], alpha, beta
+ * [R][B][Dn][H]; acc [R][B]; o [R][B][Dn][H][DV]; len_trace [R][B][H]. */
+int oracle_gdn_verify_replay(int R, int B, int H, int DK, int DV, int L, int cap,
+                             int Dn, double scale, double *h0, double *rec_q,
+                             double *rec_k, double *rec_v, double *rec_alpha,
+                             double *rec_beta, int *len, const double *q,
+                             const double *k, const double *v,
+                             const double *alpha, const double *beta,
+                             const int *acc, double *o, int *len_trace) {
+  if (R < 0 || B < 0 || H <= 0 || DK <= 0 || DV <= 0) return -1;
+  if (L <= 0 || Dn <= 0 || cap < L + Dn - 1 || cap > MAXCAP) return -1;
+  int bad = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : bad)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h) {
+      const size_t bh = ix2(b, H, h);
+      double *hh = h0 + bh * DK * DV;
+      double *rq = rec_q + bh * cap * DK, *rk = rec_k + bh * cap * DK;
+      double *rv = rec_v + bh * cap * DV;
+      double *ra = rec_alpha + bh * cap, *rb = rec_beta + bh * cap;
+      double *u = (double *)malloc(sizeof(double) * cap * DV);
+      double *z = (double *)malloc(sizeof(double) * DV);
+      int n = len[bh];
+      for (int r = 0; r < R && !bad; ++r) {
+        const int a = acc[(size_t)r * B + b];
+        if (n < 0 || n >= L || n + Dn > cap || a < 0 || a > Dn) { bad |= 1; break; }
+        for (int d = 0; d < Dn; ++d) {
+          const size_t rbdh = (((size_t)r * B + b) * Dn + d) * H + h;
+          memcpy(rq + (size_t)(n + d) * DK, q + rbdh * DK, sizeof(double) * DK);
+          memcpy(rk + (size_t)(n + d) * DK, k + rbdh * DK, sizeof(double) * DK);
+          memcpy(rv + (size_t)(n + d) * DV, v + rbdh * DV, sizeof(double) * DV);
+          ra[n + d] = alpha[rbdh];
+          rb[n + d] = beta[rbdh];
+        }
+        for (int d = 0; d < Dn; ++d) {
+          const size_t rbdh = (((size_t)r * B + b) * Dn + d) * H + h;
+          gdn_replay_out(DK, DV, n + d + 1, scale, hh, rq, rk, rv, ra, rb, o + rbdh * DV, u, z);
+        }
+        n += a;
+        if (n >= L) {
+          gdn_fold(DK, DV, hh, n, rk, rv, ra, rb, z);
+          n = 0;
+        }
+        if (len_trace) len_trace[(size_t)r * B * H + bh] = n;
+      }
+      len[bh] = n;
+      free(u);
+      free(z);
+    }
+  return bad ? -1 : 0;
+}
+
+/* The conventional comparison: snapshot the full state, step through the
+ * drafts, restore, step through the accepted ones again
+ * [hamidun §Where the state problem appears]. */
+int oracle_gdn_verify_snapshot(int R, int B, int H, int DK, int DV, int Dn, double scale,
+                               double *S, const double *q, const double *k,
+                               const double *v, const double *alpha,
+                               const double *beta, const int *acc, double *o,
+                               long long *state_copies) {
+  if (R < 0 || B < 0 || H <= 0 || DK <= 0 || DV <= 0 || Dn <= 0) return -1;
+  int bad = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : bad)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h) {
+      const size_t bh = ix2(b, H, h);
+      double *s = S + bh * DK * DV;
+      double *snap = (double *)malloc(sizeof(double) * DK * DV);
+      double *w = (double *)malloc(sizeof(double) * DV);
+      for (int r = 0; r < R; ++r) {
+        const int a = acc[(size_t)r * B + b];
+        if (a < 0 || a > Dn) { bad |= 1; break; }
+        memcpy(snap, s, sizeof(double) * DK * DV);
+        state_copies[bh] += 1;
+        for (int d = 0; d < Dn; ++d) {
+          const size_t rbdh = (((size_t)r * B + b) * Dn + d) * H + h;
+          gdn_step(DK, DV, s, k + rbdh * DK, v + rbdh * DV, alpha[rbdh], beta[rbdh], w);
+          gdn_out(DK, DV, s, q + rbdh * DK, scale, o + rbdh * DV);
+        }
+        memcpy(s, snap, sizeof(double) * DK * DV);
+        state_copies[bh] += 1;
+        for (int d = 0; d < a; ++d) {
+          const size_t rbdh = (((size_t)r * B + b) * Dn + d) * H + h;
+          gdn_step(DK, DV, s, k + rbdh * DK, v + rbdh * DV, alpha[rbdh], beta[rbdh], w);
+        }
+      }
+      free(snap);
+      free(w);
+    }
+  return bad ? -1 : 0;
+}
+
 int oracle_gdn_flush(int B, int H, int DK, int DV, int L, int cap, int force,
                      double *h0, const double *rec_k, const double *rec_v,
                      const double *rec_alpha, const double *rec_beta, int *len) {

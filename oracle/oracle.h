@@ -101,6 +101,24 @@ int oracle_gdn_replay(int T, int B, int H, int DK, int DV, int L, int cap,
                       double *o, int *len_trace, int *flush_trace,
                       long long *reads, long long *writes);
 
+/* Gated DeltaNet speculative verify: replay form (drafts appended, outputs
+ * from h0 + buffer, accepted prefix committed) and the snapshot-and-restore
+ * conventional form.  Layouts as for the Mamba-2 rounds, with q, k [DK],
+ * v, o [DV], alpha, beta scalars per (round, sequence, draft, head). */
+int oracle_gdn_verify_replay(int R, int B, int H, int DK, int DV, int L, int cap,
+                             int Dn, double scale, double *h0, double *rec_q,
+                             double *rec_k, double *rec_v, double *rec_alpha,
+                             double *rec_beta, int *len, const double *q,
+                             const double *k, const double *v,
+                             const double *alpha, const double *beta,
+                             const int *acc, double *o, int *len_trace);
+
+int oracle_gdn_verify_snapshot(int R, int B, int H, int DK, int DV, int Dn, double scale,
+                               double *S, const double *q, const double *k,
+                               const double *v, const double *alpha,
+                               const double *beta, const int *acc, double *o,
+                               long long *state_copies);
+
 int oracle_gdn_flush(int B, int H, int DK, int DV, int L, int cap, int force,
                      double *h0, const double *rec_k, const double *rec_v,
                      const double *rec_alpha, const double *rec_beta, int *len);

@@ -7,6 +7,20 @@ If the library is missing, every entry point raises.
 
 PyTorch is used for device memory and streams: `ReplayState` allocates the
 caller-owned buffers the C ABI expects (sizes from replayssm_state_bytes).
+
+A Mamba-2 layer decoded step by step (shapes of one layer, bf16 inputs):
+
+    layer = Layer("m2", batch, nheads, headdim, dstate, ngroups=G, window=16,
+                  in_dtype=torch.bfloat16)
+    state = ReplayState(layer)
+    replayssm_init(layer, state, S0)               # fp32 [B][H][P][N] on the GPU
+    for t in range(T):                             # x [B][H][P], dt [B][H], Bm/Cm [B][G][N]
+        replayssm_decode_step(layer, state, dict(x=x[t], dt=dt[t], Bm=Bm[t], Cm=Cm[t],
+                                                 A=A, D=D), y[t])
+    replayssm_materialize(layer, state, S_out, A)  # the full state, out of place
+
+Speculative rounds use replayssm_verify_commit (drafts with a draft axis after
+the batch axis, the previous round's accepted counts) and replayssm_commit.
 """
 from __future__ import annotations
 

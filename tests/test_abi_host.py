@@ -86,3 +86,26 @@ def test_cpu_tensors_are_refused():
     x = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(rs.ReplayError):
         rs._step_in(L, dict(x=x, dt=x[..., 0], Bm=x, Cm=x, A=torch.zeros(8), D=torch.zeros(8)))
+
+
+def test_empty_batch_returns_ok_without_reading_pointers(lib):
+    """batch = 0: every stateful call answers RSSM_OK on the host, with null
+    state and input pointers, and launches nothing; argument kinds the call
+    cannot serve are still refused."""
+    st, si = rs.State(), rs.StepIn()
+    for kind in ("m2", "gdn"):
+        L = _m2(batch=0) if kind == "m2" else rs.Layer("gdn", 0, 32, 128, 128)
+        d = L.desc()
+        assert lib.replayssm_init(C.byref(d), C.byref(st), None, None) == 0
+        assert lib.replayssm_decode_step(C.byref(d), C.byref(st), C.byref(si), None, None) == 0
+        assert lib.replayssm_flush(C.byref(d), C.byref(st), None, 1, None) == 0
+        assert lib.replayssm_full_decode_step(C.byref(d), None, C.byref(si), None, None, 0,
+                                              None) == 0
+        assert lib.replayssm_materialize(C.byref(d), C.byref(st), None, None, None) == 0
+    d = _m2(batch=0, draft_max=4).desc()
+    assert lib.replayssm_verify_commit(C.byref(d), C.byref(st), None, C.byref(si), 4, None,
+                                       None) == 0
+    assert lib.replayssm_commit(C.byref(d), C.byref(st), None, None, None) == 0
+    g = rs.Layer("gdn", 0, 32, 128, 128).desc()
+    assert lib.replayssm_verify_commit(C.byref(g), C.byref(st), None, C.byref(si), 1, None,
+                                       None) == 8          # unsupported for GDN

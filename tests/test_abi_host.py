@@ -109,3 +109,40 @@ def test_empty_batch_returns_ok_without_reading_pointers(lib):
     g = rs.Layer("gdn", 0, 32, 128, 128).desc()
     assert lib.replayssm_verify_commit(C.byref(g), C.byref(st), None, C.byref(si), 1, None,
                                        None) == 8          # unsupported for GDN
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="uses never-dereferenced fake device addresses: host-only check")
+def test_host_checks_on_fake_addresses(lib):
+    """Alignment, draft-count and draft-row checks answer before any launch.
+    The addresses are fake (never dereferenced); every call returns at a host
+    check, so the test runs only where no GPU is present."""
+    L = _m2(batch=2, nheads=16, ngroups=2, draft_max=4)
+    d = L.desc()
+    st = rs.State()
+    ok = 0x10000
+    st.h0, st.len, st.status = C.c_void_p(ok), C.c_void_p(ok), C.c_void_p(ok)
+    for i in range(4):
+        st.buf[i] = ok
+    si = rs.StepIn()
+    for i in range(4):
+        si.in_[i] = ok
+    si.A = si.D = C.c_void_p(ok)
+    st.h0 = C.c_void_p(ok + 4)                               # misaligned checkpoint
+    assert lib.replayssm_decode_step(C.byref(d), C.byref(st), C.byref(si), C.c_void_p(ok),
+                                     None) == 4
+    st.h0 = C.c_void_p(ok)
+    assert lib.replayssm_verify_commit(C.byref(d), C.byref(st), None, C.byref(si), 5,
+                                       C.c_void_p(ok), None) == 5   # n_draft > draft_max
+    assert lib.replayssm_verify_commit(C.byref(d), C.byref(st), None, C.byref(si), 0,
+                                       C.c_void_p(ok), None) == 5   # n_draft < 1
+    si.in_[0] = ok + 2                                       # misaligned draft x rows
+    assert lib.replayssm_verify_commit(C.byref(d), C.byref(st), None, C.byref(si), 4,
+                                       C.c_void_p(ok), None) == 4
+    si.in_[0] = ok
+    si.batch_stride[2] = 2 * 16 * 128 + 1                    # B batch stride not 16-byte
+    assert lib.replayssm_verify_commit(C.byref(d), C.byref(st), None, C.byref(si), 4,
+                                       C.c_void_p(ok), None) == 4
+    big = _m2(batch=2, nheads=32, ngroups=2, draft_max=4).desc()   # 16 heads per group
+    assert lib.replayssm_verify_commit(C.byref(big), C.byref(st), None, C.byref(si), 4,
+                                       C.c_void_p(ok), None) == 8

@@ -28,7 +28,10 @@ def _rank(rank, world, port, out):
 def test_two_ranks_take_the_slowest_time():
     ctx = mp.get_context("spawn")
     out = ctx.Queue()
-    port = 29500 + os.getpid() % 1000
+    import socket
+    with socket.socket() as sk:      # a free port on the loopback interface
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
     procs = [ctx.Process(target=_rank, args=(r, 2, port, out)) for r in range(2)]
     for p in procs:
         p.start()

@@ -63,3 +63,23 @@ def test_read_copy_error_stays_bounded_quantised_checkpoint_drifts(draw, fmt, de
         assert ck[late].mean() > 2.0 * rc[late].mean()
     else:
         assert ck[late].mean() < 1.5 * ck[early].mean()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_gdn_replay_matches_oracle_over_64_flushes(dtype):
+    """Gated DeltaNet over 1024 steps = 64 folds: each fold feeds the cached
+    corrections u_i of its window back into the checkpoint, so an error there
+    would compound; the per-step output error against the fp64 conventional
+    gated delta rule stays within the fp32 tolerance."""
+    import torch
+    w = wl.make("gdn_serving", B=2, H=4,
+                in_dtype=torch.bfloat16 if dtype == "bf16" else torch.float32)
+    g = wl.Generator(w)
+    S0 = g.initial_state()
+    st = g.steps(T)
+    got = _gpu.gdn_replay_run(w, S0, st)
+    oc, Sc, _, _ = oracle.gdn_conventional(S0, st["q"], st["k"], st["v"], st["alpha"], st["beta"])
+    errs = [rel_err(a, b) for a, b in zip(got["y"], oc)]
+    assert got["state"].status() == 0
+    assert max(errs) < 1e-4, max(errs)
+    assert rel_err(_gpu.f64(got["state"].h0), Sc) < 1e-4

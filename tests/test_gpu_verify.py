@@ -171,3 +171,41 @@ def test_verify_bad_acceptance_sets_status():
         big = {k: (v.repeat_interleave(2, dim=1) if v.dim() > 1 else v) for k, v in drafts.items()}
         rs.replayssm_verify_commit(layer, state, None, big, torch.empty(w.B, 8, w.H, w.P,
                                                                          device="cuda"))
+
+
+def test_decode_after_verify_rounds_with_ragged_lengths():
+    """Speculative rounds leave sequences at different buffer lengths, so in
+    the decode steps that follow different sequences flush on different steps
+    of one launch.  6 verify rounds at batch 16, the last acceptance
+    committed, then 40 decode steps; lengths and buffered records bit-exact,
+    outputs and checkpoints within the fp32 tolerance."""
+    w, A, D, S0, rd = _draw(6, B=16, H=16, G=2)
+    layer, state, y, lens = _gpu_rounds(w, A, D, S0, rd)
+    g = wl.Generator(w)
+    g.initial_state()
+    g.rounds(6)
+    st = g.steps(40)
+    orc = oracle.M2Replay(S0, G=w.G, L=w.L, cap=w.L + w.n_draft - 1)
+    orc.verify(rd["x"], rd["dt"], rd["Bm"], rd["Cm"], A, D, rd["acc"])
+    # the oracle's rounds commit each round's acceptance; close the last one
+    assert np.array_equal(lens[-1], orc.len)
+    start = orc.len[:, 0].copy()
+    assert len(set(start.tolist())) >= 4, start  # genuinely ragged
+    yo, lt, ft = orc.decode(st["x"], st["dt"], st["Bm"], st["Cm"], A, D)
+    dev = _gpu.to_dev(st)
+    Ad, Dd = A.cuda(), D.cuda()
+    yg = torch.empty(40, w.B, w.H, w.P, device="cuda")
+    lg = torch.empty(40, w.B, w.H, dtype=torch.int32, device="cuda")
+    for t in range(40):
+        inp = dict(x=dev["x"][t], dt=dev["dt"][t], Bm=dev["Bm"][t], Cm=dev["Cm"][t], A=Ad, D=Dd)
+        rs.replayssm_decode_step(layer, state, inp, yg[t])
+        lg[t] = state.len
+    torch.cuda.synchronize()
+    assert state.status() == 0
+    assert np.array_equal(lg.cpu().numpy(), lt)
+    # flushes happen on different steps for different sequences
+    first_flush = [int(np.argmax(ft[:, b, 0])) for b in range(w.B)]
+    assert len(set(first_flush)) >= 4, first_flush
+    assert per_step_rel_err(yg.cpu().numpy(), yo) < TOL
+    assert rel_err(_gpu.f64(state.h0), orc.h0) < TOL
+    assert _gpu.m2_buffer_matches(state, orc, w.H // w.G)

@@ -136,3 +136,53 @@ def test_read_copy_error_does_not_accumulate(oracle_mod):
         e_rc = norm_err(y_rc[tail], y_ref[tail])
         e_q = norm_err(y_q[tail], y_ref[tail])
         assert e_rc < e_q, (fmt, e_rc, e_q)
+
+
+def _e4m3_value(c):
+    """E4M3 decoded from the format definition (OCP MX v1.0 §5.3: 1 sign bit,
+    4 exponent bits with bias 7, 3 mantissa bits, subnormals at exponent 0),
+    independent of the oracle's decoder; checked against the golden table."""
+    s = -1.0 if c & 0x80 else 1.0
+    e, m = (c >> 3) & 0xF, c & 7
+    return s * (m / 8.0 * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7))
+
+
+def _block_ratios(x, scales, gs):
+    """Per 16-element block: its largest magnitude over the block's step s_b * s_g."""
+    sb = np.vectorize(_e4m3_value)(scales)
+    bmax = np.abs(x).reshape(*x.shape[:-1], -1, 16).max(-1)
+    return bmax, bmax / (sb * gs[:, None, None])
+
+
+def test_nvfp4_block_scale_maps_block_max_to_top_code(oracle_mod):
+    """The block scale is fixed by the format, not by the oracle's formula: the
+    largest magnitude of every block must land on E2M1's top value 6 within
+    the E4M3 rounding of the scale (3 mantissa bits: a relative step of at most
+    2^-4 either way), i.e. bmax / (s_b s_g) in [6/(1+2^-4), 6/(1-2^-4)] =
+    [5.65, 6.4] whenever the scale bmax / (6 s_g) is an E4M3 normal number.
+    A block scale twice too large (bmax -> ~3) or half too small (bmax ->
+    ~12, saturating) fails this.  The block holding the tile maximum gets the
+    largest finite E4M3 scale, 448, which pins the per-tile scale."""
+    for fmt, code, val in read_formats():
+        if fmt == "e4m3":
+            assert _e4m3_value(code) == val, hex(code)
+    rng = np.random.default_rng(3)
+    # blocks whose magnitudes span ~5 decades inside one tile, plus zeros
+    scale = np.exp(rng.uniform(-6, 3, (6, 16, 8, 1))).repeat(16, -1).reshape(6, 16, 128)
+    x = rng.standard_normal((6, 16, 128)) * scale
+    x = np.float32(x)
+    x[2, 5, 32:48] = 0.0
+    codes, scales, gs = oracle_mod.nvfp4_quant(x)
+    bmax, ratio = _block_ratios(x, scales, gs)
+    lo, hi = 6.0 / (1.0 + 2.0 ** -4), 6.0 / (1.0 - 2.0 ** -4)
+    normal = bmax / (6.0 * gs[:, None, None]) >= 2.0 ** -6
+    assert normal.sum() > 0.9 * normal.size  # the pin covers nearly every block
+    assert np.all((ratio[normal] >= lo) & (ratio[normal] <= hi)), (ratio[normal].min(), ratio[normal].max())
+    assert np.all(scales[bmax == 0] == 0)
+    for t in range(x.shape[0]):
+        r, b = np.unravel_index(np.argmax(bmax[t]), bmax[t].shape)
+        assert _e4m3_value(scales[t, r, b]) == 448.0
+    # the pin rejects a mis-scaled block scale in either direction
+    for wrong in (2.0, 0.5):
+        bad = bmax / (np.vectorize(_e4m3_value)(scales) * wrong * gs[:, None, None])
+        assert not np.all((bad[normal] >= lo) & (bad[normal] <= hi)), wrong

@@ -168,6 +168,20 @@ const char *replayssm_status_string(rssm_status s);
  * RSSM_ERR_CUDA return ("no error" if there was none).  Host only. */
 const char *replayssm_last_cuda_error(void);
 
+/* Test hook for the failure path of the kernels' bounded waits; host only,
+ * not for production use.  Every wait in the persistent kernels gives up
+ * after a time limit and the kernel then writes RSSM_ERR_TIMEOUT to the
+ * status word, stops its remaining work items and returns (every bulk copy it
+ * issued lands first; nothing traps).  consumer_wait_ns > 0 sets the limit of
+ * the compute warps' waits (default 2 s; <= 0 restores the default);
+ * withhold_item >= 0 makes the record-staging warp skip that work item, so the
+ * compute warps' wait for it runs out (-1: none).  Work items: Mamba-2
+ * decode and verify (sequence * G + group) * chunks + chunk, with chunks = 1
+ * when a group has at most 8 heads; GDN decode sequence * H + head.  The
+ * values apply to every launch made after the call, from any host thread.
+ * Returns RSSM_ERR_INVALID_ARG for withhold_item < -1. */
+rssm_status replayssm_set_test_hooks(int64_t consumer_wait_ns, int32_t withhold_item);
+
 /* Start a state from a full state S0 (same layout as h0; device pointer):
  * h0 <- S0 (rounded to ckpt_fmt when set), len <- 0, read copy built from h0,
  * status word cleared.  S0 may equal state->h0. */
@@ -200,14 +214,19 @@ rssm_status replayssm_flush(const rssm_desc *desc, rssm_state *state, const floa
  *      (len itself is not advanced);
  *   3. y[b][d][h][p] = output of draft d evaluated from h0 and the len+d+1
  *      records, without forming any intermediate state.
- * accepted_prev [B] int32 in 0..draft_max.  1 <= n_draft <= draft_max.
+ * accepted_prev [B] int32 in 0..draft_max, and at most the n_draft of the
+ * previous call (the device checks only the draft_max bound: a count above
+ * the previous round's draft count would commit slots that round never
+ * wrote).  1 <= n_draft <= draft_max.
  * The draft rows of x, Bm and Cm are bulk-copied by the kernel: their base
  * pointers and batch strides (in bytes) must be multiples of 16, else
  * RSSM_ERR_ALIGNMENT is returned before any launch.  H/G <= 8, else
  * RSSM_ERR_UNSUPPORTED.  Errors found on the device (a length out of range,
  * heads of a group out of step, accepted_prev[b] > draft_max, a round that
  * would overrun the capacity) set *status to RSSM_ERR_STATE and leave that
- * (sequence, group) untouched. */
+ * (sequence, group)'s lengths, checkpoint and committed records untouched
+ * (when a group's heads are split over several work items, its draft B/C
+ * rows may still be written to free slots at or above its length). */
 rssm_status replayssm_verify_commit(const rssm_desc *desc, rssm_state *state,
                                     const int32_t *accepted_prev, const rssm_step_in *drafts,
                                     int32_t n_draft, float *y, void *stream);

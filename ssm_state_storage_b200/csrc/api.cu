@@ -1,11 +1,13 @@
 // api.cu -- the C ABI declared in include/replayssm.h: host-side validation
 // of descriptors, pointers and capacities, then kernel launches on the
 // caller's stream.  No allocation, no synchronisation.
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
 #include "common.cuh"
 #include "internal.h"
+#include "pipeline.cuh"
 
 using namespace rssm;
 
@@ -66,6 +68,10 @@ rssm_status check_state(const rssm_desc *d, const rssm_state *s) {
 inline cudaStream_t to_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
+// Test hooks of the bounded waits (replayssm_set_test_hooks).
+std::atomic<uint64_t> g_wait_ns{kWaitLimitNs};
+std::atomic<int> g_hold_item{-1};
+
 inline rssm_status from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return RSSM_OK;
   g_last_cuda_error = e;
@@ -88,6 +94,8 @@ M2Params m2_params(const rssm_desc *d, const rssm_state *s) {
   p.draft_max = d->draft_max;
   p.in_bf16 = d->in_dtype == RSSM_BF16;
   p.qmode = d->read_fmt != RSSM_FMT_NONE ? d->read_fmt : (d->ckpt_fmt != RSSM_FMT_NONE ? 2 + d->ckpt_fmt : 0);
+  p.wait_ns = g_wait_ns.load();
+  p.hold_item = g_hold_item.load();
   if (s) {
     p.h0 = s->h0;
     p.xbuf = s->buf[0];
@@ -136,6 +144,8 @@ GDNParams gdn_params(const rssm_desc *d, const rssm_state *s) {
   p.cap = cap_of(d);
   p.in_bf16 = d->in_dtype == RSSM_BF16;
   p.scale = d->scale;
+  p.wait_ns = g_wait_ns.load();
+  p.hold_item = g_hold_item.load();
   if (s) {
     p.h0 = s->h0;
     p.qbuf = s->buf[0];
@@ -223,6 +233,13 @@ const char *replayssm_status_string(rssm_status s) {
 }
 
 const char *replayssm_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
+
+rssm_status replayssm_set_test_hooks(int64_t consumer_wait_ns, int32_t withhold_item) {
+  if (withhold_item < -1) return RSSM_ERR_INVALID_ARG;
+  g_wait_ns.store(consumer_wait_ns > 0 ? (uint64_t)consumer_wait_ns : kWaitLimitNs);
+  g_hold_item.store(withhold_item);
+  return RSSM_OK;
+}
 
 rssm_status replayssm_init(const rssm_desc *d, rssm_state *s, const float *S0, void *stream) {
   rssm_status st = check_desc(d);

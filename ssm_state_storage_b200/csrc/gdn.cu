@@ -364,12 +364,13 @@ struct GdnPtrs {
 // (lane 0) the bulk copies of the buffered k and u records.
 template <typename TI>
 __device__ __forceinline__ bool gdn_stage(const GDNParams &p, const GdnLayout &lay,
-                                          const GdnPtrs &S, int item, int it, int lane) {
+                                          const GdnPtrs &S, int item, int it, int lane,
+                                          volatile int *abort_flag) {
   const int L = lay.L;
   const int rb = it % lay.NR;
   const uint32_t rphase = (it / lay.NR) & 1;
   bool ok = true;
-  if (lane == 0) ok = mbar_wait(&S.rempty[rb], rphase ^ 1);
+  if (lane == 0) ok = mbar_wait(&S.rempty[rb], rphase ^ 1, kWaitLimitNs, abort_flag) && !*abort_flag;
   if (!__shfl_sync(0xffffffffu, (int)ok, 0)) return false;
   const int b = item / p.H, h = item - (item / p.H) * p.H;
   const size_t bh = (size_t)item;
@@ -451,7 +452,8 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
     bool failed = false;
     for (int item = blockIdx.x; item < nitems && !failed; item += gridDim.x) {
       for (int half = 0; half < 2; ++half) {
-        if (*abort_flag || !mbar_wait(&S.empty[slot], sphase ^ 1)) {
+        if (*abort_flag || !mbar_wait(&S.empty[slot], sphase ^ 1, kWaitLimitNs, abort_flag) ||
+            *abort_flag) {
           failed = true;
           break;
         }
@@ -470,23 +472,29 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
     if (failed) {
       if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
       *abort_flag = 1;
-      for (int s = 0; s < lay.NS; ++s)
-        if (issued & (1u << s)) mbar_wait(&S.full[s], (parity >> s) & 1u);
     }
+    // every copy issued here lands before the warp returns (see stream_tiles)
+    for (int s = 0; s < lay.NS; ++s)
+      if (issued & (1u << s)) mbar_wait(&S.full[s], (parity >> s) & 1u);
     return;
   }
   if (warp == 9) {  // stager
     int it = 0;
+    ArmedRecords armed;
     for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
       const bool abort_now = __any_sync(0xffffffffu, *abort_flag != 0);
-      if (abort_now || !gdn_stage<TI>(p, lay, S, item, it, lane)) {
-        if (lane == 0 && !abort_now) {
+      if (!abort_now && item == p.hold_item) continue;  // test hook: never staged
+      if (abort_now || !gdn_stage<TI>(p, lay, S, item, it, lane, abort_flag)) {
+        if (lane == 0 && !*abort_flag) {
           report(p.status, RSSM_ERR_TIMEOUT);
           *abort_flag = 1;
         }
-        return;
+        break;
       }
+      armed.arm(it % lay.NR, (it / lay.NR) & 1);
     }
+    if (lane == 0) armed.drain(S.rfull, lay.NR);  // no record copy outlives the warp
+    __syncwarp();
     return;
   }
 
@@ -510,9 +518,9 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
     float *gam = kq + ((L + 3) & ~3);
     float *Kf = gam + 4;
 
-    const bool got = mbar_wait(&S.rfull[rb], rphase);
+    const bool got = mbar_wait(&S.rfull[rb], rphase, p.wait_ns, abort_flag);
     if (!got) {
-      report(p.status, RSSM_ERR_TIMEOUT);
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
       *abort_flag = 1;
     }
     if (bar_or(1, kThreads, !got || *abort_flag)) break;
@@ -520,8 +528,8 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
     const int pos = 2 * it + half;  // this warp's half-tile in the producer's order
     if (reinterpret_cast<const int *>(tail)[2]) {
       if (tid == 0) report(p.status, RSSM_ERR_STATE);
-      if (!mbar_wait(&S.full[pos % lay.NS], (pos / lay.NS) & 1)) {
-        report(p.status, RSSM_ERR_TIMEOUT);
+      if (!mbar_wait(&S.full[pos % lay.NS], (pos / lay.NS) & 1, p.wait_ns, abort_flag)) {
+        if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
         *abort_flag = 1;
       }
       __syncwarp();
@@ -596,8 +604,8 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
 
     // ---- P2: this warp's 16 rows into registers; partial h0^T k and h0^T q
     const int sl = pos % lay.NS;
-    if (!mbar_wait(&S.full[sl], (pos / lay.NS) & 1)) {
-      report(p.status, RSSM_ERR_TIMEOUT);
+    if (!mbar_wait(&S.full[sl], (pos / lay.NS) & 1, p.wait_ns, abort_flag)) {
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
       *abort_flag = 1;
     }
     float4 hv[16];

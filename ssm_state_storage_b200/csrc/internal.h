@@ -37,6 +37,10 @@ struct M2Params {
   int step_index;
   // verify
   int n_draft;
+  // bounded waits: the limit of every consumer-side wait, and (test hook) a
+  // work item whose records the stager withholds, -1 for none
+  uint64_t wait_ns;
+  int hold_item;
 };
 
 struct GDNParams {
@@ -57,6 +61,8 @@ struct GDNParams {
   float *S;
   const int32_t *limit;
   int step_index;
+  uint64_t wait_ns;  // as in M2Params
+  int hold_item;
 };
 
 enum FoldMode { kFoldFlush = 0, kFoldCommit = 1, kFoldMaterialize = 2 };

@@ -160,7 +160,7 @@ struct Stage {
 template <int P, int N, typename TI>
 __device__ __forceinline__ bool stage_item(const M2Params &p, const DecodeLayout &lay,
                                            const DecodeSmemPtrs &S, int item, int it, int nchunk,
-                                           int lane) {
+                                           int lane, volatile int *abort_flag) {
   constexpr int NPL = N / 32;          // B and C values per lane
   constexpr int XPL = 8 * P / 32;      // x values per lane (up to 8 heads)
   constexpr int DPL = 8 * 16 / 32;     // dt slots per lane (up to 8 heads x 16)
@@ -168,7 +168,7 @@ __device__ __forceinline__ bool stage_item(const M2Params &p, const DecodeLayout
   const int rb = it % lay.NR;
   const uint32_t rphase = (it / lay.NR) & 1;
   bool ok = true;
-  if (lane == 0) ok = mbar_wait(&S.rempty[rb], rphase ^ 1);
+  if (lane == 0) ok = mbar_wait(&S.rempty[rb], rphase ^ 1, kWaitLimitNs, abort_flag) && !*abort_flag;
   if (!__shfl_sync(0xffffffffu, (int)ok, 0)) return false;
   int b, g, chunk, h_first;
   item_coords(p, item, nchunk, hc, b, g, chunk, h_first);
@@ -254,17 +254,24 @@ __device__ __forceinline__ void decode_stager(const M2Params &p, const DecodeLay
                                               const DecodeSmemPtrs &S, volatile int *abort_flag,
                                               int nitems, int nchunk, int lane) {
   int it = 0;
+  ArmedRecords armed;
   for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
     // warp-uniform view of the abort flag: every lane takes the same branch
     const bool abort_now = __any_sync(0xffffffffu, *abort_flag != 0);
-    if (abort_now || !stage_item<P, N, TI>(p, lay, S, item, it, nchunk, lane)) {
-      if (lane == 0 && !abort_now) {
+    if (!abort_now && item == p.hold_item) continue;  // test hook: never staged
+    if (abort_now || !stage_item<P, N, TI>(p, lay, S, item, it, nchunk, lane, abort_flag)) {
+      if (lane == 0 && !*abort_flag) {
         report(p.status, RSSM_ERR_TIMEOUT);
         *abort_flag = 1;
       }
-      return;  // nothing of ours is in flight: a wait gave up before any copy
+      break;
     }
+    armed.arm(it % lay.NR, (it / lay.NR) & 1);
   }
+  // the items staged ahead may never be consumed if the consumers stop: wait
+  // for their record copies before the warp (and possibly the CTA) ends
+  if (lane == 0) armed.drain(S.rfull, lay.NR);
+  __syncwarp();
 }
 
 // Tile producer (one lane): streams the items' checkpoint (or read-copy)
@@ -353,9 +360,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
     const TI *rB = reinterpret_cast<const TI *>(S.recB) + (size_t)rb * L * N;
     const TI *rX = reinterpret_cast<const TI *>(S.recX) + (size_t)rb * hc * L * P;
 
-    const bool got = mbar_wait(&S.rfull[rb], rphase);
+    const bool got = mbar_wait(&S.rfull[rb], rphase, p.wait_ns, abort_flag);
     if (!got) {
-      report(p.status, RSSM_ERR_TIMEOUT);
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
       *abort_flag = 1;
     }
     if (bar_or(1, kThreads, !got || *abort_flag)) break;  // uniform exit
@@ -365,8 +372,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
       // skip the item, keeping the ring in step with the producer
       for (int q0 = 0; q0 < hc; q0 += HPQ) {
         const uint32_t pos = (uint32_t)it * hc + q0 + hq;
-        if (!mbar_wait(&S.full[pos % lay.NS], (pos / lay.NS) & 1)) {
-          report(p.status, RSSM_ERR_TIMEOUT);
+        if (!mbar_wait(&S.full[pos % lay.NS], (pos / lay.NS) & 1, p.wait_ns, abort_flag)) {
+          if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
           *abort_flag = 1;
         }
         __syncwarp();
@@ -446,8 +453,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
       const size_t bh = bh0 + j;
       const uint32_t pos = (uint32_t)it * hc + j;  // producer's issue order
       const int sl = pos % lay.NS;
-      if (!mbar_wait(&S.full[sl], (pos / lay.NS) & 1)) {
-        report(p.status, RSSM_ERR_TIMEOUT);
+      if (!mbar_wait(&S.full[sl], (pos / lay.NS) & 1, p.wait_ns, abort_flag)) {
+        if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
         *abort_flag = 1;
       }
       const unsigned char *t = S.ring + sl * lay.tile_stride;

@@ -431,7 +431,10 @@ __device__ __forceinline__ void stream_tiles(const M2Params &p, uint64_t *full, 
   bool failed = false;
   for (int item = blockIdx.x; item < nitems && !failed; item += gridDim.x) {
     for (int j = 0; j < hc; ++j) {
-      if (*abort_flag || !mbar_wait(&empty[slot], sphase ^ 1)) {
+      // re-check the flag after the wait: a consumer that gave up sets it
+      // before releasing its slot, and no copy may follow an abort
+      if (*abort_flag || !mbar_wait(&empty[slot], sphase ^ 1, kWaitLimitNs, abort_flag) ||
+          *abort_flag) {
         failed = true;
         break;
       }
@@ -457,10 +460,15 @@ __device__ __forceinline__ void stream_tiles(const M2Params &p, uint64_t *full, 
   if (failed) {
     if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
     *abort_flag = 1;
-    for (int s = 0; s < NS; ++s)
-      if (issued & (1u << s)) mbar_wait(&full[s], (parity >> s) & 1u);
   }
+  // Whether or not the run aborted, return only once every copy issued here
+  // has landed: consumers that give up later must not leave the CTA exiting
+  // with a copy still writing its shared memory.
+  for (int s = 0; s < NS; ++s)
+    if (issued & (1u << s)) mbar_wait(&full[s], (parity >> s) & 1u);
 }
+
+
 
 int sm_count() {
   int dev = 0, n = 0;

@@ -102,13 +102,14 @@ struct VerifyLayout {
 template <int P, int N, typename TI>
 __device__ __forceinline__ bool verify_stage(const M2Params &p, const VerifyLayout &lay,
                                              unsigned char *smem, uint64_t *rfull,
-                                             uint64_t *rempty, int item, int it, int lane) {
+                                             uint64_t *rempty, int item, int it, int lane,
+                                             volatile int *abort_flag) {
   constexpr int DPL = (8 * 20 + 31) / 32;  // prefix dt slots per lane (hc <= 8, cap <= 20)
   const int hc = lay.hc, cap = lay.cap, L = lay.L, nd = p.n_draft;
   const int rb = it % lay.NR;
   const uint32_t rphase = (it / lay.NR) & 1;
   bool ok = true;
-  if (lane == 0) ok = mbar_wait(&rempty[rb], rphase ^ 1);
+  if (lane == 0) ok = mbar_wait(&rempty[rb], rphase ^ 1, kWaitLimitNs, abort_flag) && !*abort_flag;
   if (!__shfl_sync(0xffffffffu, (int)ok, 0)) return false;
   int b, g, chunk, h_first;
   item_coords(p, item, lay.nchunk, hc, b, g, chunk, h_first);
@@ -284,16 +285,22 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
   }
   if (warp == kVWarps + 1) {
     int it = 0;
+    ArmedRecords armed;
     for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
       const bool abort_now = __any_sync(0xffffffffu, *abort_flag != 0);
-      if (abort_now || !verify_stage<P, N, TI>(p, lay, smem, rfull, rempty, item, it, lane)) {
-        if (lane == 0 && !abort_now) {
+      if (!abort_now && item == p.hold_item) continue;  // test hook: never staged
+      if (abort_now ||
+          !verify_stage<P, N, TI>(p, lay, smem, rfull, rempty, item, it, lane, abort_flag)) {
+        if (lane == 0 && !*abort_flag) {
           report(p.status, RSSM_ERR_TIMEOUT);
           *abort_flag = 1;
         }
-        return;
+        break;
       }
+      armed.arm(it % lay.NR, (it / lay.NR) & 1);
     }
+    if (lane == 0) armed.drain(rfull, lay.NR);  // no record copy outlives the warp
+    __syncwarp();
     return;
   }
 
@@ -344,9 +351,10 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
     float *Bf = db, *wf = Bf + cap * N, *lamf = wf + pad4(hc * cap), *lamd = lamf + pad4(hc);
     float *z = lamd + kMD * hc;
 
-    const bool got = (lay.NR > 1 || take_turn(it)) && mbar_wait(&rfull[rb], rphase);
+    const bool got =
+        (lay.NR > 1 || take_turn(it)) && mbar_wait(&rfull[rb], rphase, p.wait_ns, abort_flag);
     if (!got) {
-      report(p.status, RSSM_ERR_TIMEOUT);
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
       *abort_flag = 1;
     }
     if (bar_or(gbar, kGThreads, !got || *abort_flag)) break;
@@ -358,8 +366,8 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
       }
       for (int j = 0; j < hc; ++j) {
         const uint32_t pos = (uint32_t)it * hc + j;
-        if (!mbar_wait(&full[pos % lay.NS], (pos / lay.NS) & 1)) {
-          report(p.status, RSSM_ERR_TIMEOUT);
+        if (!mbar_wait(&full[pos % lay.NS], (pos / lay.NS) & 1, p.wait_ns, abort_flag)) {
+          if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
           *abort_flag = 1;
         }
         __syncwarp();
@@ -525,8 +533,8 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
       const size_t bh = bh0 + j;
       const uint32_t pos = (uint32_t)it * hc + j;
       const int sl = pos % lay.NS;
-      if (!mbar_wait(&full[sl], (pos / lay.NS) & 1)) {
-        report(p.status, RSSM_ERR_TIMEOUT);
+      if (!mbar_wait(&full[sl], (pos / lay.NS) & 1, p.wait_ns, abort_flag)) {
+        if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
         *abort_flag = 1;
       }
       if (j == hc - 1) pass_turn();
@@ -605,14 +613,18 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
 }
 
 // Chunked verify only: append the draft B and C rows of group (b, g) at the
-// group's committed length, read back from the length the verify kernel just
-// wrote.  An item the verify kernel rejected (its status already reports it)
-// is skipped when the slots would not fit.
+// group's committed length, read back from the lengths the verify kernel just
+// wrote.  A group whose heads are not all at the same length (the verify
+// kernel rejected some of its chunks and reported it in the status word) is
+// skipped, so no buffered record another head still uses is overwritten; for
+// a rejected group whose heads agree the rows land in free slots (>= len).
 template <typename TI>
 __global__ void __launch_bounds__(128) m2_verify_append_bc_kernel(const M2Params p) {
   const int b = blockIdx.x / p.G, g = blockIdx.x - (blockIdx.x / p.G) * p.G;
   const size_t bg = (size_t)b * p.G + g;
-  const int nb = p.len[(size_t)b * p.H + (size_t)g * p.hpg];
+  const int32_t *lg = p.len + (size_t)b * p.H + (size_t)g * p.hpg;
+  const int nb = lg[0];
+  if (__syncthreads_or(threadIdx.x < p.hpg && lg[threadIdx.x] != nb)) return;
   if (nb < 0 || nb + p.n_draft > p.cap) return;
   const TI *Bin = static_cast<const TI *>(p.Bm) + b * p.bs_B;
   const TI *Cin = static_cast<const TI *>(p.Cm) + b * p.bs_C;

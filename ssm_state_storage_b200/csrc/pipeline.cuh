@@ -53,15 +53,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase of the given parity to complete; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// Wait for the phase of the given parity to complete.  Returns false when
+// `limit_ns` of wall-clock time pass first, or -- if `abort` is given -- as
+// soon as another warp of the CTA has set *abort (its peer stopped, so the
+// awaited arrival may never come).  Waits for this thread's own bulk copies
+// in flight pass no abort flag: those copies complete on their own.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitLimitNs,
+                                          volatile int *abort = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
+    if ((i & 255u) == 0) {
+      if (global_ns() - t0 > limit_ns) return false;
+      if (abort && *abort) return false;
+    }
   }
 }
+
+// Record bulk copies armed by a stager warp: per record buffer, whether it
+// has been armed and the phase parity of its latest arming.  On exit the
+// stager waits (bounded, regardless of any abort) for the latest phase of
+// every armed buffer, so that no record copy is in flight when the CTA ends.
+struct ArmedRecords {
+  uint32_t armed = 0, parity = 0;
+  __device__ __forceinline__ void arm(int rb, uint32_t ph) {
+    armed |= 1u << rb;
+    parity = (parity & ~(1u << rb)) | (ph << rb);
+  }
+  __device__ __forceinline__ void drain(uint64_t *rfull, int nr) const {
+    for (int r = 0; r < nr; ++r)
+      if (armed & (1u << r)) mbar_wait(&rfull[r], (parity >> r) & 1u);
+  }
+};
 
 // Global -> shared bulk copy completing on `bar` (bytes % 16 == 0, both
 // addresses 16-byte aligned).

@@ -85,6 +85,7 @@ ENTRY_POINTS = {
                                         C.c_void_p, C.c_void_p]),
     "replayssm_quantize": (C.c_int, [C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p,
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "replayssm_set_test_hooks": (C.c_int, [C.c_int64, C.c_int32]),
 }
 
 _lib = None
@@ -350,3 +351,11 @@ def replayssm_status_string(code: int) -> str:
 def replayssm_validate(layer: Layer) -> int:
     d = layer.desc()
     return int(lib().replayssm_validate(C.byref(d)))
+
+
+def replayssm_set_test_hooks(consumer_wait_ns: int = 0, withhold_item: int = -1):
+    """Test hook of the bounded device waits (see include/replayssm.h):
+    shorten the compute warps' wait limit and make the staging warp skip one
+    work item.  Call with no arguments to restore the defaults."""
+    _ok(lib().replayssm_set_test_hooks(int(consumer_wait_ns), int(withhold_item)),
+        "replayssm_set_test_hooks")

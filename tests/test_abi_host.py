@@ -146,3 +146,11 @@ def test_host_checks_on_fake_addresses(lib):
     big = _m2(batch=2, nheads=32, ngroups=2, draft_max=4).desc()   # 16 heads per group
     assert lib.replayssm_verify_commit(C.byref(big), C.byref(st), None, C.byref(si), 4,
                                        C.c_void_p(ok), None) == 8
+
+
+def test_test_hooks_entry_point_validates_and_resets():
+    from ssm_state_storage_b200 import replayssm as rs
+    with pytest.raises(rs.ReplayError, match="invalid"):
+        rs.replayssm_set_test_hooks(1000, -2)
+    rs.replayssm_set_test_hooks(1000, 3)
+    rs.replayssm_set_test_hooks()  # back to the defaults

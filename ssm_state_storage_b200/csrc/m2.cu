@@ -26,6 +26,7 @@
 // rows w*P/8 + rs + 4*rho and columns 32*s + 4*c8, so each quarter-warp reads
 // one 128-byte line and the row sums need only 3 shuffle levels.
 #include "m2_device.cuh"
+#include "umma.cuh"
 
 namespace rssm {
 namespace {
@@ -50,18 +51,26 @@ namespace {
 // the producer warp: C_k [N], dt records [hc][L], A [hc], D [hc], header.
 struct DecodeLayout {
   int NS, NR, hc, L, tile_bytes, tile_stride, stage_floats, scratch_floats;
-  int off_bars, off_recB, off_recX, off_stage, off_scr, off_ring, total;
+  int off_bars, off_recB, off_recX, off_stage, off_scr, off_umma, off_ring, total;
+  int umma_b_bytes;  // tensor-core fold: bytes of one head group's B operands (3 terms)
 
   __host__ __device__ static int align128(int v) { return (v + 127) & ~127; }
 
-  __host__ static DecodeLayout make(int P, int N, int hc, int L, int es, int qm, int budget) {
+  // mma: the flush fold runs on the tensor cores (operand areas added, no
+  // fp32 copy of the B records); hpq: heads in flight at once.
+  __host__ static DecodeLayout make(int P, int N, int hc, int L, int es, int qm, int budget,
+                                    bool mma = false, int hpq = 1) {
     DecodeLayout d;
     d.hc = hc;
     d.L = L;
     d.tile_bytes = qm == 1 ? P * N : qm == 2 ? P * N / 2 + P * N / 16 : P * N * 4;
     d.tile_stride = align128(d.tile_bytes);
     d.stage_floats = N + pad4(hc * L) + 2 * pad4(hc) + 4;
-    d.scratch_floats = 2 * pad4(L) + pad4(hc * L) + pad4(hc) + 32 + L * N + hc * P;
+    d.scratch_floats = 2 * pad4(L) + pad4(hc * L) + pad4(hc) + 32 + (mma ? 0 : L * N) + hc * P;
+    // A operand: the group's B records as a 128 x 16 K-slab; per head group
+    // the three split terms of its head's weighted x records, P x 16 each
+    d.umma_b_bytes = mma ? 3 * P * 32 : 0;
+    const int umma_bytes = mma ? N * 32 + hpq * d.umma_b_bytes : 0;
     const int rec_b = L * N * es, rec_x = hc * L * P * es;
     // Prefer three record buffers (the stager then runs two items ahead, which
     // hides its two dependent memory round trips) as long as the ring keeps
@@ -69,7 +78,9 @@ struct DecodeLayout {
     for (d.NR = 3; d.NR >= 1; --d.NR) {
       int o = 0;
       d.off_bars = o;
-      o += align128(8 * (2 * 8 + 2 * 4));  // room for up to 8 slots and 4 record buffers
+      // up to 8 ring slots and 4 record buffers (192 bytes), then two fold-MMA
+      // barriers and the tensor-memory base address
+      o += align128(8 * (2 * 8 + 2 * 4) + 2 * 8 + 4);
       d.off_recB = o;
       o += align128(d.NR * rec_b);
       d.off_recX = o;
@@ -78,6 +89,8 @@ struct DecodeLayout {
       o += align128(d.NR * d.stage_floats * 4);
       d.off_scr = o;
       o += align128(2 * d.scratch_floats * 4);
+      d.off_umma = o;
+      o += align128(umma_bytes);
       d.off_ring = o;
       const int room = budget - o;
       d.NS = room / d.tile_stride;
@@ -119,8 +132,9 @@ __device__ __forceinline__ void view_from_smem(const unsigned char *t, float sg,
 }
 
 struct DecodeSmemPtrs {
-  uint64_t *full, *empty, *rfull, *rempty;
-  unsigned char *ring;
+  uint64_t *full, *empty, *rfull, *rempty, *mma;
+  uint32_t *tmem_slot;
+  unsigned char *ring, *umma;
   unsigned char *recB, *recX;
   float *stage, *scr;
   __device__ DecodeSmemPtrs(unsigned char *smem, const DecodeLayout &lay) {
@@ -128,6 +142,9 @@ struct DecodeSmemPtrs {
     empty = full + 8;
     rfull = empty + 8;
     rempty = rfull + 4;
+    mma = rempty + 4;  // one per head group: its fold MMAs completed
+    tmem_slot = reinterpret_cast<uint32_t *>(mma + 2);
+    umma = smem + lay.off_umma;
     ring = smem + lay.off_ring;
     recB = smem + lay.off_recB;
     recX = smem + lay.off_recX;
@@ -286,14 +303,126 @@ __device__ __forceinline__ void decode_tiles(const M2Params &p, const DecodeLayo
                          lay.hc, abort_flag, nitems, nchunk);
 }
 
+
+// ------------------------------------------------- tensor-core flush fold
+// On the flush step the fold's rank-k update runs on the tensor cores:
+//   D_j[n][r] = sum_i B_i[n] * (w_{j,i} x_{j,i}[r])        (M = N = 128, N' = P, K = 16)
+// as a bf16 MMA with an fp32 accumulator in tensor memory.  B_i is bf16
+// (exact); the fp32 products w x are split into three bf16 terms (three
+// MMAs into the same accumulator), so every partial product is exact and the
+// increment keeps fp32 accuracy.  The epilogue then forms
+//   h0[r][n] <- Lam_j h0[r][n] + D_j[n][r]
+// with tensor-memory lane n (= state column) per thread, so each warp's
+// loads of the old tile and stores of the new one cover 32 consecutive
+// columns of a row.
+
+// A operand: the group's B records, A[n][i] = B_i[n] (zero for i >= k),
+// written by all consumer threads.
+template <int N, typename TI>
+__device__ __forceinline__ void build_fold_a(unsigned char *dst, const TI *rB, int k, int tid) {
+  for (int e = tid; e < N * 8; e += kThreads) {
+    const int n = e % N, q = e / N, i0 = 2 * q;
+    const TI b0 = i0 < k ? rB[i0 * N + n] : TI{}, b1 = i0 + 1 < k ? rB[(i0 + 1) * N + n] : TI{};
+    __nv_bfloat162 v;
+    v.x = b0;
+    v.y = b1;
+    *reinterpret_cast<__nv_bfloat162 *>(dst + umma::kmajor_offset(n, i0)) = v;
+  }
+}
+
+// B operands of head j: the three bf16 terms of w_i x_i[r] as P x 16
+// K-slabs, written by the head group's WPH warps (gt = thread in group).
+template <int P, typename TI>
+__device__ __forceinline__ void build_fold_b(unsigned char *dst, const TI *xj, const float *wj,
+                                             int k, int gt, int gthreads) {
+  for (int e = gt; e < P * 8; e += gthreads) {
+    const int r = e % P, q = e / P, i0 = 2 * q;
+    const float v0 = i0 < k ? wj[i0] * to_f32(xj[i0 * P + r]) : 0.f;
+    const float v1 = i0 + 1 < k ? wj[i0 + 1] * to_f32(xj[(i0 + 1) * P + r]) : 0.f;
+    __nv_bfloat162 h, m, l;
+    umma::split3_bf16(v0, h.x, m.x, l.x);
+    umma::split3_bf16(v1, h.y, m.y, l.y);
+    const uint32_t o = umma::kmajor_offset(r, i0);
+    *reinterpret_cast<__nv_bfloat162 *>(dst + o) = h;
+    *reinterpret_cast<__nv_bfloat162 *>(dst + P * 32 + o) = m;
+    *reinterpret_cast<__nv_bfloat162 *>(dst + 2 * P * 32 + o) = l;
+  }
+}
+
+// Epilogue of head bh's fold by the WPH warps of one head group (`sub` = warp
+// in group): the new checkpoint, and for a read copy its new codes.  The old
+// tile comes from the ring slot (QM 0) or, with a read copy in the slot, from
+// the fp32 checkpoint in global memory.  NVFP4 (QM 2) takes a second pass
+// over the values this thread stored, after the group agrees on the tile
+// maximum (named barrier 2 + hq, `red` = the group's 8 maxima).
+template <int P, int N, int QM, int WPH>
+__device__ __forceinline__ void fold_epilogue(const M2Params &p, size_t bh, const float *tile,
+                                              float lam, uint32_t tcol, int sub, int lane,
+                                              float *red, int hq) {
+  static_assert(N == 128, "tensor-memory lanes are the 128 state columns");
+  constexpr int NW = WPH / 4;  // warps sharing one tensor-memory lane quarter
+  constexpr int CW = P / NW;   // checkpoint rows per warp
+  const int n = 32 * (sub & 3) + lane, r0 = (sub >> 2) * CW;
+  const uint32_t taddr = tcol + ((uint32_t)(32 * (sub & 3)) << 16) + (uint32_t)r0;
+  float *hg = p.h0 + bh * (size_t)(P * N);
+  float amax = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < CW; c += 32) {
+    float d[32];
+    umma::ld32(taddr + c, d);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int r = r0 + c + i;
+      const float t = QM == 0 ? tile[r * N + n] : hg[r * N + n];
+      const float hn = fmaf(lam, t, d[i]);
+      hg[r * N + n] = hn;
+      if constexpr (QM == 1) p.rc[bh * (size_t)(P * N) + r * N + n] = (uint8_t)e4m3_encode(hn);
+      if constexpr (QM == 2) amax = fmaxf(amax, fabsf(hn));
+    }
+  }
+  if constexpr (QM == 2) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (lane == 0) red[sub] = amax;
+    bar_sync(2 + hq, WPH * 32);
+    float tmax = red[0];
+    for (int w2 = 1; w2 < WPH; ++w2) tmax = fmaxf(tmax, red[w2]);
+    const float sg = nvfp4_tile_scale(tmax);
+    uint8_t *rc = p.rc + bh * (size_t)(P * N / 2);
+    uint8_t *sc = p.rc_scale + bh * (size_t)(P * N / 16);
+#pragma unroll 4
+    for (int i = 0; i < CW; ++i) {
+      const int r = r0 + i;
+      const float hn = hg[r * N + n];  // this thread's own store
+      float bm = fabsf(hn);
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+      const uint32_t scode = nvfp4_block_code(bm, sg);
+      const float dstep = nvfp4_step(scode, sg);
+      const float qv = dstep > 0.f ? __fdiv_rn(hn, dstep) : 0.f;
+      const float qn = __shfl_xor_sync(0xffffffffu, qv, 1);
+      if ((lane & 1) == 0) rc[r * (N / 2) + n / 2] = (uint8_t)e2m1x2_encode(qv, qn);
+      if ((lane & 15) == 0) sc[r * (N / 16) + n / 16] = (uint8_t)scode;
+    }
+    if (sub == 0 && lane == 0) p.rc_gscale[bh] = sg;
+    bar_sync(2 + hq, WPH * 32);  // red[] is reused by the group's next head
+  }
+}
+
 constexpr int kDecodeThreads = kThreads + 64;  // 8 consumer warps, tile producer, stager
 
-template <int P, int N, typename TI, int QM, int WPH>
+template <int P, int N, typename TI, int QM, int WPH, bool MMA>
 __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Params p,
                                                                   const DecodeLayout lay) {
   using T = Tile<P, N>;
   constexpr int C4 = T::C4;
   constexpr bool kReadCopy = (QM == 1 || QM == 2);
+  static_assert(!MMA || (N == 128 && QM <= 2 && std::is_same<TI, __nv_bfloat16>::value),
+                "tensor-core fold: bf16 records, 128 state columns, fp32 or read-copy checkpoint");
+  constexpr int HPQ = 8 / WPH;  // heads in flight (one head group each)
+  constexpr uint32_t kTmemCols = MMA ? (HPQ * P <= 128 ? 128 : 256) : 0;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int abort_word;
   volatile int *abort_flag = &abort_word;
@@ -313,8 +442,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
       mbar_init(&S.rfull[r], 1);
       mbar_init(&S.rempty[r], 8);
     }
+    mbar_init(&S.mma[0], 1);
+    mbar_init(&S.mma[1], 1);
     *abort_flag = 0;
     mbar_fence_init();
+  }
+  if constexpr (MMA) {
+    if (warp == 0) umma::alloc(S.tmem_slot, kTmemCols);
+    umma::fence_before_sync();
   }
   __syncthreads();
   if (warp == 8) {
@@ -339,9 +474,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
   // takes row 4g + rs, lane c8 columns 32s + 4c8).  A warp first pulls its
   // rows into registers (then the slot is released), so the outputs and the
   // fold run while the producer already refills the slot.
-  constexpr int HPQ = 8 / WPH, RW = P / WPH, RG = RW / 4;
+  constexpr int RW = P / WPH, RG = RW / 4;
   constexpr int RGC = RG < 4 ? RG : 4;  // row groups held in registers at once
-  const int hq = warp / WPH, sub = warp - hq * WPH;
+  const int hq = warp / WPH, sub = warp - hq * WPH, gt = tid - hq * WPH * 32;
+  uint32_t tmem = 0, n_mma = 0;  // tensor-memory base; fold MMA batches this group committed
+  if constexpr (MMA) {
+    umma::fence_after_sync();
+    tmem = *S.tmem_slot;
+  }
+  unsigned char *umma_a = S.umma, *umma_b = S.umma + N * 32 + hq * lay.umma_b_bytes;
   int it = 0;
   for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
     const int rb = it % lay.NR;
@@ -351,8 +492,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
     float *wdt = scr + 2 * pad4(L);
     float *lam = wdt + pad4(hc * L);
     float *red = lam + pad4(hc);
-    float *Bf = red + 32;  // fp32 copy of the group's B records [k][N]
-    float *z = Bf + L * N;  // buffered-record and skip terms of y [hc][P]
+    float *Bf = red + 32;  // fp32 copy of the group's B records [k][N] (SIMT fold only)
+    float *z = Bf + (MMA ? 0 : L * N);  // buffered-record and skip terms of y [hc][P]
     int b, g, chunk, h_first;
     item_coords(p, item, nchunk, hc, b, g, chunk, h_first);
     const size_t bh0 = (size_t)b * p.H + h_first;
@@ -403,9 +544,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
       }
       if (tid < hc) p.dtbuf[(bh0 + tid) * p.cap + k - 1] = st.dt[tid * L + k - 1];
     }
-    // ---- fp32 B records (for the fold), B_i.C_k dots, decay weights
-    if (flush)
+    // ---- the fold's B operand (fp32 records, or the MMA's A operand), B_i.C_k
+    // dots, decay weights
+    if constexpr (MMA) {
+      if (flush) {
+        build_fold_a<N, TI>(umma_a, rB, k, tid);
+        fence_proxy_async_smem();  // visible to the tensor cores after the barrier below
+      }
+    } else if (flush) {
       for (int e = tid; e < k * N; e += kThreads) Bf[e] = to_f32(rB[e]);
+    }
     {
       // 16 threads per record, fp64 (these dots of N rounded products would
       // otherwise dominate the output error when the inputs are fp32); the
@@ -453,6 +601,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
       const size_t bh = bh0 + j;
       const uint32_t pos = (uint32_t)it * hc + j;  // producer's issue order
       const int sl = pos % lay.NS;
+      const bool mma_fold = MMA && flush;
+      if (mma_fold) {
+        // this head's fold increment on the tensor cores, issued before its
+        // tile arrives; the group's previous epilogue has finished reading
+        // the accumulator columns (tensor-memory loads waited, fence, barrier)
+        build_fold_b<P, TI>(umma_b, rX + j * L * P, wdt + j * L, k, gt, WPH * 32);
+        fence_proxy_async_smem();
+        umma::fence_before_sync();
+        bar_sync(4 + hq, WPH * 32);
+        if (gt == 0) {
+          umma::fence_after_sync();
+          const uint32_t id = umma::idesc_bf16_f32(128, P);
+          const uint64_t ad = umma::smem_desc(umma_a);
+#pragma unroll
+          for (int t3 = 0; t3 < 3; ++t3)
+            umma::mma_bf16(tmem + hq * P, ad, umma::smem_desc(umma_b + t3 * P * 32), id, t3 > 0);
+          umma::commit(&S.mma[hq]);
+        }
+      }
       if (!mbar_wait(&S.full[sl], (pos / lay.NS) & 1, p.wait_ns, abort_flag)) {
         if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
         *abort_flag = 1;
@@ -470,7 +637,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
         float4 v[RGC][C4];
 #pragma unroll
         for (int u = 0; u < RGC; ++u) view_row<P, N, QM>(t, sub * RW + 4 * (c0 + u) + rs, c8, v[u]);
-        if (c0 + RGC == RG) {  // all of this warp's rows are in registers
+        // all of this warp's rows are in registers: release the slot (the
+        // tensor-core fold of an fp32 tile still reads it in its epilogue)
+        if (c0 + RGC == RG && !(mma_fold && QM == 0)) {
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.empty[sl]);
         }
@@ -483,7 +652,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
           if constexpr (QM == 2) a *= sg;  // the NVFP4 view leaves the tile scale out
           if (c8 == 0) yout[rows[u]] = fmaf(lm, a, zj[rows[u]]);
         }
-        if (flush) {
+        if (flush && !MMA) {
           if constexpr (kReadCopy) {
 #pragma unroll
             for (int u = 0; u < RGC; ++u) load_row<N>(tile, rows[u], c8, v[u]);
@@ -498,7 +667,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
           }
         }
       }
-      if constexpr (QM == 2 || QM == 4) {
+      if constexpr (MMA) {
+        if (mma_fold) {
+          const bool done = mbar_wait(&S.mma[hq], n_mma & 1u, p.wait_ns, abort_flag);
+          ++n_mma;
+          if (!done) {
+            if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+            *abort_flag = 1;
+          }
+          umma::fence_after_sync();
+          fold_epilogue<P, N, QM, WPH>(p, bh, reinterpret_cast<const float *>(t), lm,
+                                       tmem + hq * P, sub, lane, red + 8 * hq, hq);
+          umma::fence_before_sync();
+          if constexpr (QM == 0) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.empty[sl]);
+          }
+        }
+      }
+      if constexpr ((QM == 2 || QM == 4) && !MMA) {
         if (flush) {
           // NVFP4 needs the whole tile's maximum: combine the WPH warps of
           // this head, then requantise the rows just written (each thread
@@ -530,6 +717,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.rempty[rb]);
     if (tid < hc) p.len[bh0 + tid] = flush ? 0 : k;
+  }
+  if constexpr (MMA) {
+    // every fold MMA has completed before the tensor memory is released (a
+    // group that stopped early may not have waited for its last batch)
+    if (gt == 0 && n_mma > 0) mbar_wait(&S.mma[hq], (n_mma - 1) & 1u);
+    umma::fence_before_sync();
+    bar_sync(1, kThreads);
+    umma::fence_after_sync();
+    if (warp == 0) umma::dealloc(tmem, kTmemCols);
   }
 }
 
@@ -691,24 +887,45 @@ cudaError_t launch_decode(K kernel, const M2Params &p, const DecodeLayout &lay, 
 }
 
 template <int P, int N, typename TI, int WPH>
-cudaError_t decode_wph(const M2Params &p, const DecodeLayout &lay, cudaStream_t s) {
+cudaError_t decode_wph(const M2Params &p, const DecodeLayout &lay, bool mma, cudaStream_t s) {
+  if constexpr (N == 128 && std::is_same<TI, __nv_bfloat16>::value) {
+    if (mma) {
+      switch (p.qmode) {
+        case 0: return launch_decode(m2_decode_kernel<P, N, TI, 0, WPH, true>, p, lay, s);
+        case 1: return launch_decode(m2_decode_kernel<P, N, TI, 1, WPH, true>, p, lay, s);
+        case 2: return launch_decode(m2_decode_kernel<P, N, TI, 2, WPH, true>, p, lay, s);
+        default: return cudaErrorInvalidValue;
+      }
+    }
+  }
   switch (p.qmode) {
-    case 0: return launch_decode(m2_decode_kernel<P, N, TI, 0, WPH>, p, lay, s);
-    case 1: return launch_decode(m2_decode_kernel<P, N, TI, 1, WPH>, p, lay, s);
-    case 2: return launch_decode(m2_decode_kernel<P, N, TI, 2, WPH>, p, lay, s);
-    case 3: return launch_decode(m2_decode_kernel<P, N, TI, 3, WPH>, p, lay, s);
-    case 4: return launch_decode(m2_decode_kernel<P, N, TI, 4, WPH>, p, lay, s);
+    case 0: return launch_decode(m2_decode_kernel<P, N, TI, 0, WPH, false>, p, lay, s);
+    case 1: return launch_decode(m2_decode_kernel<P, N, TI, 1, WPH, false>, p, lay, s);
+    case 2: return launch_decode(m2_decode_kernel<P, N, TI, 2, WPH, false>, p, lay, s);
+    case 3: return launch_decode(m2_decode_kernel<P, N, TI, 3, WPH, false>, p, lay, s);
+    case 4: return launch_decode(m2_decode_kernel<P, N, TI, 4, WPH, false>, p, lay, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
+// The flush fold runs on the tensor cores for bf16 records, 128 state
+// columns and an fp32 checkpoint (with or without a read copy), when the
+// operand areas fit beside the ring; otherwise, and for fp32 inputs (whose
+// records are not exact in bf16) or a quantised checkpoint, on the SIMT pipes.
 template <int P, int N, typename TI>
 cudaError_t decode_qm(const M2Params &p, cudaStream_t s) {
   const int hc = decode_chunk(p.hpg);
-  const DecodeLayout lay = DecodeLayout::make(P, N, hc, p.L, (int)sizeof(TI), p.qmode, 220 * 1024);
+  const int hpq = hc >= 2 ? 2 : 1;  // two heads in flight (4 warps each) when possible
+  const int es = (int)sizeof(TI);
+  DecodeLayout lay{};
+  bool mma = N == 128 && std::is_same<TI, __nv_bfloat16>::value && p.qmode <= 2;
+  if (mma) {
+    lay = DecodeLayout::make(P, N, hc, p.L, es, p.qmode, 220 * 1024, true, hpq);
+    if (lay.NS < 2) mma = false;
+  }
+  if (!mma) lay = DecodeLayout::make(P, N, hc, p.L, es, p.qmode, 220 * 1024);
   if (lay.NS < 2) return cudaErrorInvalidConfiguration;
-  // two heads in flight (4 warps each) when the item has at least two heads
-  return hc >= 2 ? decode_wph<P, N, TI, 4>(p, lay, s) : decode_wph<P, N, TI, 8>(p, lay, s);
+  return hpq == 2 ? decode_wph<P, N, TI, 4>(p, lay, mma, s) : decode_wph<P, N, TI, 8>(p, lay, mma, s);
 }
 
 template <int P, int N, typename TI, int MODE>

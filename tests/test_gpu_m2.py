@@ -39,6 +39,7 @@ def _oracle_replay(w, A, D, S0, st, **kw):
     ("m2_tiny", 64, {}),                       # 4 flushes, fp32 inputs
     ("m2_serving", 40, {"B": 3}),              # bf16, 16 groups, ragged batch
     ("m2_serving", 24, {"B": 2, "P": 128, "N": 64, "H": 16, "G": 4}),
+    ("m2_serving", 36, {"B": 2, "P": 128, "H": 16, "G": 2}),  # 128 x 128 tiles, 2 folds
 ])
 def test_m2_replay_decode_matches_oracle(name, T, kw):
     w, A, D, S0, st = _draw(name, T, **kw)

@@ -301,6 +301,9 @@ def run_ours(args, rank, world):
     if state.status() != 0:
         raise RuntimeError(f"device status {state.status()} after the replay run")
 
+    steps_us = per_launch_us(lambda i: rs.replayssm_decode_step(layer, state, step_in[i % pool], y,
+                                                                stream), L, 10, stream, torch, dev)
+
     for i in range(args.warmup):
         full_window(i)
     ms_full = timed(full_window, args.steps, args.warmup)
@@ -341,6 +344,7 @@ def run_ours(args, rank, world):
                        "achieved_gbs": achieved_full, "frac": achieved_full / peak,
                        "kernel": "m2_full_kernel"},
         "replay_over_full": value / value_full,
+        "step_times": steps_us,
         "bytes_per_head_token": {"replay": win_bytes / (w.B * w.H * L),
                                  "full_state": full_bytes / (w.B * w.H * L)},
         "clocks": clocks,
@@ -354,6 +358,8 @@ def run_ours(args, rank, world):
         line["gdn"] = bench_gdn(args, dev, peak, rs, bm, wl, torch)
         torch.cuda.empty_cache()
         line["verify"] = bench_verify(args, dev, peak, rs, bm, wl, torch)
+        torch.cuda.empty_cache()
+        line["verify_gdn"] = bench_verify_gdn(args, dev, peak, rs, bm, wl, torch)
         torch.cuda.empty_cache()
         line["read_copy"] = bench_readcopy(args, dev, peak, rs, bm, wl, torch, ms_per_window)
         torch.cuda.empty_cache()
@@ -422,6 +428,24 @@ def run_e2e(args, w, layer, state, st, Ad, Dd, dev, world, rs, torch, dist):
             "steps": args.e2e_steps, "pipelined": "H2D / decode / D2H on three streams"}
 
 
+def per_launch_us(step, L, windows, stream, torch, dev):
+    """CUDA-event time of every launch of `windows` windows of L decode steps
+    (an event between consecutive launches on the launching stream), averaged
+    per position in the window: the last position is the flush step."""
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(L * windows + 1)]
+    ev[0].record(stream)
+    for i in range(L * windows):
+        step(i)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    per = [0.0] * L
+    for i in range(L * windows):
+        per[i % L] += ev[i].elapsed_time(ev[i + 1]) * 1e3 / windows
+    return {"nonflush_avg_us": sum(per[:-1]) / max(L - 1, 1), "flush_us": per[-1],
+            "per_position_us": [round(v, 1) for v in per], "windows": windows}
+
+
 def _events_ms(fn, n, stream, torch, dev):
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
@@ -463,23 +487,32 @@ def bench_gdn(args, dev, peak, rs, bm, wl, torch):
         full_window(i)
     ms_r = _events_ms(replay_window, n, stream, torch, dev)
     ms_f = _events_ms(full_window, n, stream, torch, dev)
+    steps_us = per_launch_us(lambda i: rs.replayssm_decode_step(layer, state, step_in[i % pool], o,
+                                                                stream), L, 10, stream, torch, dev)
     if state.status() != 0:
         raise RuntimeError(f"device status {state.status()} after the GDN run")
     inb = 2
     wb = bm.gdn_replay_window_bytes(L, w.N, w.P, inb) * w.B * w.H
+    wb_rec = bm.gdn_replay_window_bytes_records(L, w.N, w.P, inb) * w.B * w.H
     fb = bm.gdn_conventional_bytes(w.N, w.P, inb) * w.B * w.H * L
     ach_r = wb / (ms_r / n * 1e-3) / 1e9
+    ach_rec = wb_rec / (ms_r / n * 1e-3) / 1e9
     ach_f = fb / (ms_f / n * 1e-3) / 1e9
     tok = w.B * L * n
     return {"workload": "gdn_serving", "value": tok / (ms_r * 1e-3), "unit": "tokens/s",
             "ms_per_window": ms_r / n,
             "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
-                         "frac": ach_r / peak, "kernel": "gdn_decode_kernel"},
+                         "frac": ach_r / peak, "kernel": "gdn_decode_kernel",
+                         "bytes": "records with their cached corrections u (as stored)",
+                         "frac_input_records_only": ach_rec / peak,
+                         "achieved_input_records_only": ach_rec},
             "full_state": {"value": tok / (ms_f * 1e-3), "unit": "tokens/s",
                            "achieved_gbs": ach_f, "frac": ach_f / peak,
                            "kernel": "gdn_kernel<full>"},
             "replay_over_full": ms_f / ms_r,
+            "step_times": steps_us,
             "bytes_per_head_token": {"replay": wb / (w.B * w.H * L),
+                                     "replay_input_records_only": wb_rec / (w.B * w.H * L),
                                      "full_state": fb / (w.B * w.H * L)},
             "gpu_launches": n * L}
 
@@ -627,6 +660,91 @@ def bench_verify(args, dev, peak, rs, bm, wl, torch):
                                  "kernels": "cudaMemcpyAsync x2 + m2_full_kernel x8"},
             "replay_over_snapshot": ms_s / ms_r,
             "gpu_launches": rounds}
+
+
+def bench_verify_gdn(args, dev, peak, rs, bm, wl, torch):
+    """gdn_verify: Gated DeltaNet gdn_serving heads at batch 256, 4 drafts per
+    round, acceptance ~ U{0..4}; replay verify/commit against snapshot-and-
+    restore decoding of the full state."""
+    w = wl.make("gdn_verify")
+    pool = 16
+    g = wl.Generator(w)
+    S0 = g.initial_state()
+    rd = g.rounds(pool)
+    acc_host = rd["acc"].clone()
+    rd = {k: v.to(dev) for k, v in rd.items()}
+    names = ("q", "k", "v", "alpha", "beta")
+    layer = rs.Layer("gdn", w.B, w.H, w.P, w.N, window=w.L, draft_max=w.n_draft,
+                     in_dtype=w.in_dtype)
+    state = rs.ReplayState(layer, device=dev)
+    rs.replayssm_init(layer, state, S0.to(dev))
+    y = torch.empty(w.B, w.n_draft, w.H, w.P, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    drafts = [{k: rd[k][r] for k in names} for r in range(pool)]
+    n = args.sub_steps
+    for r in range(3):
+        rs.replayssm_verify_commit(layer, state, rd["acc"][(r - 1) % pool] if r else None,
+                                   drafts[r % pool], y, stream)
+    rs.replayssm_commit(layer, state, rd["acc"][2 % pool], stream=stream)
+    torch.cuda.synchronize(dev)
+    lens0 = state.len[:, 0].cpu().long()
+
+    def timed_round(r):
+        rs.replayssm_verify_commit(layer, state, rd["acc"][(r + 2) % pool] if r else None,
+                                   drafts[(r + 3) % pool], y, stream)
+
+    ms_r = _events_ms(timed_round, n, stream, torch, dev)
+    if state.status() != 0:
+        raise RuntimeError(f"device status {state.status()} after the GDN verify run")
+    lens = lens0.clone()
+    total = 0.0
+    for r in range(n):
+        a = acc_host[(r + 2) % pool].long() if r else torch.zeros_like(lens)
+        n1 = lens + a
+        fold = n1 >= w.L
+        per = [bm.gdn_verify_round_bytes(int(n1[b]), bool(fold[b]), w.n_draft, w.N, w.P, 2)
+               for b in range(w.B)]
+        total += sum(per) * w.H
+        lens = torch.where(fold, torch.zeros_like(n1), n1)
+    ach_r = total / (ms_r * 1e-3) / 1e9
+
+    fl = rs.Layer("gdn", w.B, w.H, w.P, w.N, window=w.L, in_dtype=w.in_dtype)
+    S = S0.to(dev)
+    snap = torch.empty_like(S)
+    ysn = torch.empty(w.B, w.n_draft, w.H, w.P, device=dev)
+    junk = torch.empty(w.B, w.H, w.P, device=dev)
+
+    def snap_round(r):
+        i = r % pool
+        snap.copy_(S)
+        for d in range(w.n_draft):
+            rs.replayssm_full_decode_step(fl, S, {k: rd[k][i][:, d] for k in names}, ysn[:, d],
+                                          stream=stream)
+        S.copy_(snap)
+        for d in range(w.n_draft):
+            rs.replayssm_full_decode_step(fl, S, {k: rd[k][i][:, d] for k in names}, junk,
+                                          limit=rd["acc"][i], step_index=d, stream=stream)
+
+    for r in range(2):
+        snap_round(r)
+    ms_s = _events_ms(snap_round, n, stream, torch, dev)
+    st_b = w.N * w.P * 4
+    conv = bm.gdn_conventional_bytes(w.N, w.P, 2)
+    snap_bytes = 0.0
+    for r in range(n):
+        a = acc_host[r % pool].double()
+        snap_bytes += float((4 * st_b + (w.n_draft + a) * conv).sum()) * w.H
+    ach_s = snap_bytes / (ms_s * 1e-3) / 1e9
+    return {"workload": "gdn_verify", "rounds_per_s": n / (ms_r * 1e-3),
+            "ms_per_round": ms_r / n,
+            "drafts_evaluated_per_s": w.B * w.n_draft * n / (ms_r * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
+                         "frac": ach_r / peak, "kernel": "gdn_verify_kernel"},
+            "snapshot_restore": {"rounds_per_s": n / (ms_s * 1e-3), "ms_per_round": ms_s / n,
+                                 "achieved_gbs": ach_s, "frac": ach_s / peak,
+                                 "kernels": "cudaMemcpyAsync x2 + gdn_kernel<full> x8"},
+            "replay_over_snapshot": ms_s / ms_r,
+            "gpu_launches": n}
 
 
 def run_drift(args, rank):

@@ -91,7 +91,7 @@ typedef struct {
   int32_t dstate;    /* Mamba-2 N (64 or 128); GDN DK (128)                      */
   int32_t ngroups;   /* Mamba-2 G (H % G == 0, H/G <= 16); GDN: ignored          */
   int32_t window;    /* records per flush, 1..16 (the pages use 16)              */
-  int32_t draft_max; /* most drafts per verify round, 0..4 (Mamba-2)            */
+  int32_t draft_max; /* most drafts per verify round, 0..4                      */
   int32_t in_dtype;  /* rssm_dtype of the step inputs                            */
   int32_t read_fmt;  /* rssm_fmt of the read copy (Mamba-2 only)                 */
   int32_t ckpt_fmt;  /* rssm_fmt the checkpoint is rounded to at each fold: the
@@ -206,7 +206,7 @@ rssm_status replayssm_decode_step(const rssm_desc *desc, rssm_state *state,
 rssm_status replayssm_flush(const rssm_desc *desc, rssm_state *state, const float *A,
                             int32_t force, void *stream);
 
-/* Speculative verify round (Mamba-2) [sitech §Reducing state traffic...]:
+/* Speculative verify round [sitech §Reducing state traffic...]:
  *   1. if accepted_prev != NULL: len += accepted_prev[b] (the previous round's
  *      accepted drafts are already in their slots) and, when len >= window,
  *      fold all len records into h0 and set len = 0;
@@ -214,13 +214,19 @@ rssm_status replayssm_flush(const rssm_desc *desc, rssm_state *state, const floa
  *      (len itself is not advanced);
  *   3. y[b][d][h][p] = output of draft d evaluated from h0 and the len+d+1
  *      records, without forming any intermediate state.
+ * Mamba-2 drafts: x [B][n][H][P], dt [B][n][H], Bm/Cm [B][n][G][N], y
+ * [B][n][H][P].  Gated DeltaNet drafts [hamidun §Why hybrid models became
+ * the norm]: q, k [B][n][H][DK], v [B][n][H][DV], alpha, beta [B][n][H], o
+ * [B][n][H][DV]; each draft's delta-rule correction u (buf[5]) is stored with
+ * it, so an accepted draft leaves exactly the correction sequential decoding
+ * would have cached.
  * accepted_prev [B] int32 in 0..draft_max, and at most the n_draft of the
  * previous call (the device checks only the draft_max bound: a count above
  * the previous round's draft count would commit slots that round never
  * wrote).  1 <= n_draft <= draft_max.
- * The draft rows of x, Bm and Cm are bulk-copied by the kernel: their base
- * pointers and batch strides (in bytes) must be multiples of 16, else
- * RSSM_ERR_ALIGNMENT is returned before any launch.  H/G <= 8, else
+ * Mamba-2: the draft rows of x, Bm and Cm are bulk-copied by the kernel:
+ * their base pointers and batch strides (in bytes) must be multiples of 16,
+ * else RSSM_ERR_ALIGNMENT is returned before any launch; H/G <= 8, else
  * RSSM_ERR_UNSUPPORTED.  Errors found on the device (a length out of range,
  * heads of a group out of step, accepted_prev[b] > draft_max, a round that
  * would overrun the capacity) set *status to RSSM_ERR_STATE and leave that
@@ -231,7 +237,8 @@ rssm_status replayssm_verify_commit(const rssm_desc *desc, rssm_state *state,
                                     const int32_t *accepted_prev, const rssm_step_in *drafts,
                                     int32_t n_draft, float *y, void *stream);
 
-/* Close a verify round: len += accepted[b]; fold when len >= window. */
+/* Close a verify round: len += accepted[b]; fold when len >= window.  A:
+ * Mamba-2 decay rates [H] (NULL for GDN). */
 rssm_status replayssm_commit(const rssm_desc *desc, rssm_state *state, const int32_t *accepted,
                              const float *A, void *stream);
 

@@ -91,3 +91,33 @@ def gdn_replay_bytes(k, L, DK, DV, in_bytes):
 
 def gdn_replay_window_bytes(L, DK, DV, in_bytes):
     return sum(gdn_replay_bytes(k, L, DK, DV, in_bytes) for k in range(1, L + 1))
+
+
+def gdn_replay_bytes_records(k, L, DK, DV, in_bytes):
+    """The same step counted with the plain record of the layer inputs only
+    (q, k, v in the input dtype, alpha, beta fp32) and no cached corrections:
+    a past record contributes the fields a replay needs (k, v, alpha, beta),
+    the current record is read and appended, the output written, and the
+    checkpoint written on the flush step."""
+    state = DK * DV * 4
+    rec_read = (DK + DV) * in_bytes + 8
+    cur = (2 * DK + DV) * in_bytes + 8
+    flush = k == L
+    append = 0 if flush else cur
+    return state + (k - 1) * rec_read + cur + append + DV * 4 + (state if flush else 0)
+
+
+def gdn_replay_window_bytes_records(L, DK, DV, in_bytes):
+    return sum(gdn_replay_bytes_records(k, L, DK, DV, in_bytes) for k in range(1, L + 1))
+
+
+def gdn_verify_round_bytes(n1, fold, nd, DK, DV, in_bytes):
+    """One Gated DeltaNet speculative round for one head: read h0, the n1
+    committed records (key, cached correction, alpha), the nd drafts (q, k, v,
+    alpha, beta); append the drafts with their corrections; write nd outputs;
+    write h0 once when the commit folds."""
+    state = DK * DV * 4
+    rec = DK * in_bytes + DV * 4 + 4
+    draft = (2 * DK + DV) * in_bytes + 8
+    return (state + n1 * rec + nd * draft + nd * (draft + DV * 4) + nd * DV * 4
+            + (state if fold else 0))

@@ -41,7 +41,6 @@ rssm_status check_desc(const rssm_desc *d) {
   } else {
     if (!gdn_supported(d->dstate, d->headdim)) return RSSM_ERR_SHAPE;
     if (d->read_fmt != RSSM_FMT_NONE || d->ckpt_fmt != RSSM_FMT_NONE) return RSSM_ERR_UNSUPPORTED;
-    if (d->draft_max != 0) return RSSM_ERR_UNSUPPORTED;
     if ((int64_t)d->batch * d->nheads > INT32_MAX) return RSSM_ERR_SHAPE;
   }
   return RSSM_OK;
@@ -144,6 +143,7 @@ GDNParams gdn_params(const rssm_desc *d, const rssm_state *s) {
   p.cap = cap_of(d);
   p.in_bf16 = d->in_dtype == RSSM_BF16;
   p.scale = d->scale;
+  p.draft_max = d->draft_max;
   p.wait_ns = g_wait_ns.load();
   p.hold_item = g_hold_item.load();
   if (s) {
@@ -160,7 +160,8 @@ GDNParams gdn_params(const rssm_desc *d, const rssm_state *s) {
   return p;
 }
 
-rssm_status gdn_inputs(GDNParams &p, const rssm_step_in *in) {
+// nd: the length of the draft axis after the batch axis (1 for a decode step)
+rssm_status gdn_inputs(GDNParams &p, const rssm_step_in *in, int nd = 1) {
   if (!in) return RSSM_ERR_INVALID_ARG;
   for (int i = 0; i < 5; ++i)
     if (!in->in[i]) return RSSM_ERR_INVALID_ARG;
@@ -169,12 +170,12 @@ rssm_status gdn_inputs(GDNParams &p, const rssm_step_in *in) {
   p.v = in->in[2];
   p.alpha = static_cast<const float *>(in->in[3]);
   p.beta = static_cast<const float *>(in->in[4]);
-  p.bs_q = stride_or(in->batch_stride[0], (int64_t)p.H * p.DK);
-  p.bs_k = stride_or(in->batch_stride[1], (int64_t)p.H * p.DK);
-  p.bs_v = stride_or(in->batch_stride[2], (int64_t)p.H * p.DV);
-  p.bs_a = stride_or(in->batch_stride[3], (int64_t)p.H);
-  p.bs_b = stride_or(in->batch_stride[4], (int64_t)p.H);
-  p.bs_y = stride_or(in->y_batch_stride, (int64_t)p.H * p.DV);
+  p.bs_q = stride_or(in->batch_stride[0], (int64_t)nd * p.H * p.DK);
+  p.bs_k = stride_or(in->batch_stride[1], (int64_t)nd * p.H * p.DK);
+  p.bs_v = stride_or(in->batch_stride[2], (int64_t)nd * p.H * p.DV);
+  p.bs_a = stride_or(in->batch_stride[3], (int64_t)nd * p.H);
+  p.bs_b = stride_or(in->batch_stride[4], (int64_t)nd * p.H);
+  p.bs_y = stride_or(in->y_batch_stride, (int64_t)nd * p.H * p.DV);
   return RSSM_OK;
 }
 
@@ -306,11 +307,19 @@ rssm_status replayssm_verify_commit(const rssm_desc *d, rssm_state *s,
                                     int32_t n_draft, float *y, void *stream) {
   rssm_status st = check_desc(d);
   if (st != RSSM_OK) return st;
-  if (d->kind != RSSM_MAMBA2) return RSSM_ERR_UNSUPPORTED;
   if (d->read_fmt != RSSM_FMT_NONE || d->ckpt_fmt != RSSM_FMT_NONE) return RSSM_ERR_UNSUPPORTED;
   if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
   if ((st = check_state(d, s)) != RSSM_OK) return st;
   if (n_draft < 1 || n_draft > d->draft_max) return RSSM_ERR_CAPACITY;
+  if (d->kind == RSSM_GDN) {
+    if (!y) return RSSM_ERR_INVALID_ARG;
+    GDNParams p = gdn_params(d, s);
+    if ((st = gdn_inputs(p, drafts, n_draft)) != RSSM_OK) return st;
+    p.y = y;
+    p.acc = accepted_prev;
+    p.n_draft = n_draft;
+    return from_cuda(gdn_launch_verify(p, to_stream(stream)));
+  }
   // the verify stager maps (draft, head) pairs of a work item onto one warp's lanes
   if (d->nheads / d->ngroups > 8) return RSSM_ERR_UNSUPPORTED;
   if (!y) return RSSM_ERR_INVALID_ARG;
@@ -333,10 +342,15 @@ rssm_status replayssm_commit(const rssm_desc *d, rssm_state *s, const int32_t *a
                              const float *A, void *stream) {
   rssm_status st = check_desc(d);
   if (st != RSSM_OK) return st;
-  if (d->kind != RSSM_MAMBA2) return RSSM_ERR_UNSUPPORTED;
   if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
   if ((st = check_state(d, s)) != RSSM_OK) return st;
-  if (!accepted || !A) return RSSM_ERR_INVALID_ARG;
+  if (!accepted) return RSSM_ERR_INVALID_ARG;
+  if (d->kind == RSSM_GDN) {
+    GDNParams p = gdn_params(d, s);
+    p.acc = accepted;
+    return from_cuda(gdn_launch_fold(p, kFoldCommit, to_stream(stream)));
+  }
+  if (!A) return RSSM_ERR_INVALID_ARG;
   M2Params p = m2_params(d, s);
   p.acc = accepted;
   p.A = A;

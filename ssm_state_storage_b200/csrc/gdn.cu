@@ -30,26 +30,30 @@
 #include "common.cuh"
 #include "internal.h"
 #include "pipeline.cuh"
+#include "umma.cuh"
 
 namespace rssm {
 namespace {
 
 constexpr int DKc = 128, DVc = 128;
-constexpr int kMaxRec = 16;          // GDN buffers hold at most one window
+constexpr int kMaxRec = kMaxCap;     // a window plus the tail of a speculative round
 constexpr int kRows = DKc / 8;       // rows per warp
-constexpr int kZ = kMaxRec + 1;      // records + q
 
-enum GdnMode { kGdnDecode = 0, kGdnFlush = 1, kGdnMaterialize = 2, kGdnFull = 3 };
+enum GdnMode { kGdnDecode = 0, kGdnFlush = 1, kGdnMaterialize = 2, kGdnFull = 3, kGdnCommit = 4 };
 
+// Shared memory of gdn_kernel for at most MR records (the conventional step
+// has exactly one).
+template <int MR>
 struct GdnSmem {
+  static constexpr int kZ = MR + 1;  // records + q
   float k[kZ][DKc];       // k_0..k_{n-1}, then q
-  float u[kMaxRec][DVc];  // v_i, overwritten by u_i
+  float u[MR][DVc];       // v_i, overwritten by u_i
   float part[8][kZ][DVc];
   float z[kZ][DVc];
-  float alpha[kMaxRec], beta[kMaxRec], gamma[kMaxRec];
-  float ratio[kMaxRec][kMaxRec];
-  float gram[kMaxRec][kMaxRec];
-  float kq[kMaxRec];
+  float alpha[MR], beta[MR], gamma[MR];
+  float ratio[MR][MR];
+  float gram[MR][MR];
+  float kq[MR];
   int n, act;
 };
 
@@ -62,7 +66,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 template <typename TI, int MODE>
 __global__ void __launch_bounds__(kThreads, 2) gdn_kernel(const GDNParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  GdnSmem &S = *reinterpret_cast<GdnSmem *>(smem_raw);
+  using Smem = GdnSmem<MODE == kGdnFull ? 1 : kMaxRec>;
+  Smem &S = *reinterpret_cast<Smem *>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh_i = blockIdx.x;
   const int b = bh_i / p.H, h = bh_i - b * p.H;
@@ -80,6 +85,12 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_kernel(const GDNParams p) {
         ok = n0 >= 0 && n0 < p.L;
         n = n0 + 1;
         act = 1;
+      } else if (MODE == kGdnCommit) {  // len += accepted; fold when it reaches the window
+        const int a = p.acc[b];
+        ok = n0 >= 0 && n0 < p.L && a >= 0 && a <= p.draft_max && n0 + a <= p.cap;
+        n = n0 + a;
+        act = n >= p.L;
+        if (ok && !act) p.len[bh] = n;
       } else {
         ok = n0 >= 0 && n0 <= p.cap;
         n = n0;
@@ -190,8 +201,8 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_kernel(const GDNParams p) {
       else S.gram[i][j] = acc;
     }
   }
-  if (tid < n * n) {
-    const int i = tid / n, j = tid - (tid / n) * n;
+  for (int e = tid; e < n * n; e += kThreads) {
+    const int i = e / n, j = e - (e / n) * n;
     if (j <= i) {
       float r = 1.f;
       for (int m = j + 1; m <= i; ++m) r *= S.alpha[m];
@@ -258,12 +269,13 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_kernel(const GDNParams p) {
     for (int rho = 0; rho < kRows; ++rho)
       st_stream(dst + (size_t)(kRows * warp + rho) * DVc + 4 * lane, hv[rho]);
   }
-  if (tid == 0 && (MODE == kGdnDecode || MODE == kGdnFlush)) p.len[bh] = fold ? 0 : n;
+  if (tid == 0 && (MODE == kGdnDecode || MODE == kGdnFlush || MODE == kGdnCommit))
+    p.len[bh] = fold ? 0 : n;
 }
 
 template <typename TI, int MODE>
 cudaError_t launch(const GDNParams &p, cudaStream_t s) {
-  const size_t smem = sizeof(GdnSmem);
+  const size_t smem = sizeof(GdnSmem<MODE == kGdnFull ? 1 : kMaxRec>);
   cudaError_t e = cudaFuncSetAttribute(gdn_kernel<TI, MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -301,10 +313,12 @@ constexpr int kHalfBytes = kHalfRows * DVc * 4;          // 32 KiB
 
 struct GdnLayout {
   int NS, NR, L;
-  int off_bars, off_recK, off_recU, off_stage, off_db, off_single, off_ring, total;
+  int off_bars, off_recK, off_recU, off_stage, off_db, off_single, off_umma, off_ring, total;
   int stage_floats, db_floats;
   __host__ static int a128(int v) { return (v + 127) & ~127; }
-  __host__ static GdnLayout make(int L, int es, int budget) {
+  // mma: the flush fold's operands (three split terms of the weighted
+  // corrections, 128 x 16 bf16 each, and the keys, 128 x 16) get an area
+  __host__ static GdnLayout make(int L, int es, int budget, bool mma = false) {
     GdnLayout d;
     d.L = L;
     // stage: q, kc, v [128] fp32 | alpha [L] | beta | hdr(2 ints)
@@ -314,7 +328,7 @@ struct GdnLayout {
     for (d.NR = 3; d.NR >= 1; --d.NR) {
       int o = 0;
       d.off_bars = o;
-      o += a128(8 * (2 * 8 + 2 * 4));
+      o += a128(8 * (2 * 8 + 2 * 4) + 8 + 4);  // ring, records, fold MMA, tensor-memory base
       d.off_recK = o;
       o += a128(d.NR * L * DKc * es);
       d.off_recU = o;
@@ -325,6 +339,8 @@ struct GdnLayout {
       o += a128(2 * d.db_floats * 4);
       d.off_single = o;  // part [8][2][128] | z [2][128] | ucur [128] | opart [128]
       o += a128((8 * 2 * 128 + 2 * 128 + 2 * 128) * 4);
+      d.off_umma = o;
+      o += mma ? 4 * 128 * 32 : 0;
       d.off_ring = o;
       d.NS = (budget - o) / kHalfBytes;
       if (d.NS > 8) d.NS = 8;
@@ -339,14 +355,18 @@ struct GdnLayout {
 };
 
 struct GdnPtrs {
-  uint64_t *full, *empty, *rfull, *rempty;
-  unsigned char *recK, *ring;
+  uint64_t *full, *empty, *rfull, *rempty, *mma;
+  uint32_t *tmem_slot;
+  unsigned char *recK, *ring, *umma;
   float *recU, *stage, *db, *part, *z, *ucur, *opart;
   __device__ GdnPtrs(unsigned char *smem, const GdnLayout &l) {
     full = reinterpret_cast<uint64_t *>(smem + l.off_bars);
     empty = full + 8;
     rfull = empty + 8;
     rempty = rfull + 4;
+    mma = rempty + 4;
+    tmem_slot = reinterpret_cast<uint32_t *>(mma + 1);
+    umma = smem + l.off_umma;
     recK = smem + l.off_recK;
     recU = reinterpret_cast<float *>(smem + l.off_recU);
     stage = reinterpret_cast<float *>(smem + l.off_stage);
@@ -420,9 +440,41 @@ __device__ __forceinline__ bool gdn_stage(const GDNParams &p, const GdnLayout &l
   return true;
 }
 
+// Tensor-core flush fold (bf16 keys): the rank-k increment
+//   D[c][row] = sum_i (R_i u_i[c]) k_i[row]          (M = DV = 128, N' = DK = 128, K = 16)
+// as a bf16 MMA with an fp32 accumulator in tensor memory; the fp32 products
+// R_i u_i are split into three bf16 terms (three MMAs), the keys are exact in
+// bf16.  Epilogue h0[row][c] <- gamma h0[row][c] + D[c][row] with lane c per
+// thread: warps 0-3 take rows 0-63 (half-tile 0), warps 4-7 rows 64-127.
 template <typename TI>
+__device__ __forceinline__ void gdn_build_fold_operands(unsigned char *ua, const float *rU,
+                                                        const float *ucur, const float *R,
+                                                        const TI *rK, int k, int tid) {
+  unsigned char *ub = ua + 3 * 128 * 32;
+  for (int e = tid; e < 128 * 8; e += kThreads) {
+    const int c = e % 128, q = e / 128, i0 = 2 * q, i1 = i0 + 1;
+    auto uval = [&](int i) -> float {
+      return i < k - 1 ? rU[i * DVc + c] : (i == k - 1 ? ucur[c] : 0.f);
+    };
+    const float v0 = i0 < k ? R[i0] * uval(i0) : 0.f, v1 = i1 < k ? R[i1] * uval(i1) : 0.f;
+    __nv_bfloat162 h, m, l, kb;
+    umma::split3_bf16(v0, h.x, m.x, l.x);
+    umma::split3_bf16(v1, h.y, m.y, l.y);
+    const uint32_t o = umma::kmajor_offset(c, i0);
+    *reinterpret_cast<__nv_bfloat162 *>(ua + o) = h;
+    *reinterpret_cast<__nv_bfloat162 *>(ua + 128 * 32 + o) = m;
+    *reinterpret_cast<__nv_bfloat162 *>(ua + 2 * 128 * 32 + o) = l;
+    // keys: row index c here runs over d_k
+    kb.x = i0 < k ? rK[i0 * DKc + c] : TI{};
+    kb.y = i1 < k ? rK[i1 * DKc + c] : TI{};
+    *reinterpret_cast<__nv_bfloat162 *>(ub + o) = kb;
+  }
+}
+
+template <typename TI, bool MMA>
 __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNParams p,
                                                                    const GdnLayout lay) {
+  static_assert(!MMA || std::is_same<TI, __nv_bfloat16>::value, "tensor-core fold: bf16 keys");
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int abort_word;
   volatile int *abort_flag = &abort_word;
@@ -440,8 +492,13 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
       mbar_init(&S.rfull[r], 1);
       mbar_init(&S.rempty[r], 8);
     }
+    mbar_init(S.mma, 1);
     *abort_flag = 0;
     mbar_fence_init();
+  }
+  if constexpr (MMA) {
+    if (warp == 0) umma::alloc(S.tmem_slot, 128);
+    umma::fence_before_sync();
   }
   __syncthreads();
 
@@ -502,6 +559,11 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
   // holds rows 16w..16w+15 (local rows 16(w%4).. of half-tile w/4) and
   // columns 4*lane..4*lane+3.
   const int half = warp >> 2, row0 = 16 * warp;
+  uint32_t tmem = 0, n_mma = 0;
+  if constexpr (MMA) {
+    umma::fence_after_sync();
+    tmem = *S.tmem_slot;
+  }
   int it = 0;
   for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
     const int rb = it % lay.NR;
@@ -599,7 +661,7 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
         }
       }
     }
-    if (flush)
+    if (flush && !MMA)
       for (int e = tid; e < k * DKc; e += kThreads) Kf[e] = to_f32(rK[e]);
 
     // ---- P2: this warp's 16 rows into registers; partial h0^T k and h0^T q
@@ -613,8 +675,11 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
 #pragma unroll
     for (int rho = 0; rho < 16; ++rho)
       hv[rho] = *reinterpret_cast<const float4 *>(tile + (16 * (warp & 3) + rho) * DVc + 4 * lane);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&S.empty[sl]);
+    const bool mma_fold = MMA && flush;
+    if (!mma_fold) {  // the tensor-core fold reads the half-tile again in its epilogue
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.empty[sl]);
+    }
     {
       float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
 #pragma unroll
@@ -679,8 +744,51 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
       const float o = fmaf(kq[k - 1], S.ucur[c], S.opart[c]);  // R_{k-1} = 1
       p.y[b * p.bs_y + (size_t)h * DVc + c] = p.scale * o;
     }
+    if constexpr (MMA) {
+      if (mma_fold) {
+        // ---- P5 on the tensor cores: the previous fold's accumulator reads
+        // finished before the barrier (wait::ld, fence)
+        gdn_build_fold_operands<TI>(S.umma, rU, S.ucur, R, rK, k, tid);
+        fence_proxy_async_smem();
+        umma::fence_before_sync();
+        bar_sync(1, kThreads);
+        if (tid == 0) {
+          umma::fence_after_sync();
+          const uint32_t id = umma::idesc_bf16_f32(128, 128);
+          const uint64_t bd = umma::smem_desc(S.umma + 3 * 128 * 32);
+#pragma unroll
+          for (int t3 = 0; t3 < 3; ++t3)
+            umma::mma_bf16(tmem, umma::smem_desc(S.umma + t3 * 128 * 32), bd, id, t3 > 0);
+          umma::commit(S.mma);
+        }
+        const bool done = mbar_wait(S.mma, n_mma & 1u, p.wait_ns, abort_flag);
+        ++n_mma;
+        if (!done) {
+          if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        umma::fence_after_sync();
+        const int c = 32 * (warp & 3) + lane, rbase = 64 * half;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)rbase;
+        const float g = gam[0];
+        float *dst = p.h0 + bh * (DKc * DVc);
+#pragma unroll 1
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          float d[32];
+          umma::ld32(taddr + c0, d);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int r = c0 + i;  // row within the half-tile
+            dst[(size_t)(rbase + r) * DVc + c] = fmaf(g, tile[r * DVc + c], d[i]);
+          }
+        }
+        umma::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[sl]);
+      }
+    }
     // ---- P5 (flush): h0 <- gamma h0 + sum_i R_i k_i u_i^T, written once
-    if (flush) {
+    if (flush && !MMA) {
       const float g = gam[0];
 #pragma unroll
       for (int rho = 0; rho < 16; ++rho) hv[rho] = mul4x(g, hv[rho]);
@@ -706,6 +814,262 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
     if (lane == 0) mbar_arrive(&S.rempty[rb]);
     if (tid == 0) p.len[bh] = flush ? 0 : k;
   }
+  if constexpr (MMA) {
+    if (tid == 0 && n_mma > 0) mbar_wait(S.mma, (n_mma - 1) & 1u);  // no MMA outlives the memory
+    umma::fence_before_sync();
+    bar_sync(1, kThreads);
+    umma::fence_after_sync();
+    if (warp == 0) umma::dealloc(tmem, 128);
+  }
+}
+
+
+// ============================================================ verify round
+// Speculative verify round of Gated DeltaNet [sitech.ge, "NVIDIA ו-Dao AI Lab
+// הציגו ReplaySSM…", §Reducing state traffic and simplifying rollback], one
+// CTA of 256 threads per (sequence, head):
+//   1. commit of the previous round: n1 = len + accepted; when n1 reaches the
+//      window the n1 buffered records are folded into h0 with their cached
+//      corrections u_i (h0 <- gamma h0 + sum_i R_i k_i u_i^T, written once) and
+//      the drafts follow an empty buffer (nb = 0), else nb = n1;
+//   2. draft d becomes record e = nb + d.  One pass over the checkpoint tile
+//      gives every draft's h0^T k_d and h0^T q_d (2 nd columns); then, draft
+//      by draft (each needs the corrections of the earlier ones),
+//        u_e = beta_e (v_e - gamma_e h0^T k_e - sum_{j<e} R(e,j) (k_j.k_e) u_j)
+//        o_d = scale (gamma_e h0^T q_d + sum_{i<=e} R(e,i) (k_i.q_d) u_i)
+//      with gamma_e = prod_{m<=e} alpha_m and R(e,j) = prod_{j<m<=e} alpha_m over
+//      the committed records followed by the drafts;
+//   3. the drafts and their u_e are appended at slots nb .. nb+nd-1 and len =
+//      nb: the u_e of a draft that is accepted later is exactly the correction
+//      sequential decoding would have cached for it.
+// Decay products are prefix products in fp64 (R(e,j) = Q_e / Q_j with all
+// alpha > 0); the key dots are fp32 products summed in fp64.
+constexpr int kVD = 4;               // most drafts per round
+constexpr int kVSeq = kMaxRec + kVD;  // records a draft sequence can reach (with slack)
+
+struct GdnVerifySmem {
+  float Kc[kMaxRec][DKc];     // committed keys (records 0..n1-1)
+  float U[kVSeq][DVc];        // cached corrections, then this round's drafts'
+  float Kd[kVD][DKc], Qd[kVD][DKc], Vd[kVD][DVc];
+  float part[8][2 * kVD][DVc];
+  float z[2 * kVD][DVc];      // h0^T k_d, then h0^T q_d
+  float G[kVD][kVSeq];        // k_j . k_{e_d}
+  float KQ[kVD][kVSeq];       // k_i . q_d
+  float R[kVD][kVSeq];        // R(e_d, j)
+  float gam[kVD];
+  float af[kMaxRec], Rf[kMaxRec];  // committed alphas; fold weights
+  float ad[kVD], bd[kVD];          // draft alpha, beta
+  float gf;
+  int n1, nb, fold, bad;
+};
+
+template <typename TI>
+__global__ void __launch_bounds__(kThreads, 2) gdn_verify_kernel(const GDNParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  GdnVerifySmem &S = *reinterpret_cast<GdnVerifySmem *>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.x / p.H, h = blockIdx.x - (blockIdx.x / p.H) * p.H;
+  const size_t bh = blockIdx.x;
+  const int nd = p.n_draft;
+
+  if (tid == 0) {
+    const int n0 = p.len[bh];
+    const int a = p.acc ? p.acc[b] : 0;
+    const int n1 = n0 + a, fold = n1 >= p.L, nb = fold ? 0 : n1;
+    const int bad = n0 < 0 || n0 >= p.L || a < 0 || a > p.draft_max || n1 > p.cap ||
+                    nb + nd > p.cap;
+    if (bad) report(p.status, RSSM_ERR_STATE);
+    S.n1 = n1;
+    S.nb = nb;
+    S.fold = fold;
+    S.bad = bad;
+  }
+  __syncthreads();
+  if (S.bad) return;
+  const int n1 = S.n1, nb = S.nb, ne = nb + nd;  // draft sequence: records 0..ne-1
+  const bool fold = S.fold;
+
+  // ---- checkpoint tile into registers (rows 16w + rho, columns 4 lane ..)
+  float *tile = p.h0 + bh * (DKc * DVc);
+  float4 hv[kRows];
+#pragma unroll
+  for (int rho = 0; rho < kRows; ++rho)
+    hv[rho] = ld_stream(tile + (size_t)(kRows * warp + rho) * DVc + 4 * lane);
+
+  // ---- stage committed records and the drafts (fp32)
+  const TI *kb = static_cast<const TI *>(p.kbuf) + bh * p.cap * DKc;
+  const float *ub = p.ubuf + bh * p.cap * DVc;
+  for (int e = tid; e < n1 * DKc; e += kThreads) {
+    S.Kc[e / DKc][e % DKc] = to_f32(kb[e]);
+    S.U[e / DVc][e % DVc] = ub[e];
+  }
+  for (int e = tid; e < nd * DKc; e += kThreads) {
+    const int d = e / DKc, c = e % DKc;
+    const int64_t o = (int64_t)(d * p.H + h) * DKc + c;
+    S.Qd[d][c] = ld_in<TI>(p.q, b * p.bs_q + o);
+    S.Kd[d][c] = ld_in<TI>(p.k, b * p.bs_k + o);
+    S.Vd[d][c] = ld_in<TI>(p.v, b * p.bs_v + (int64_t)(d * p.H + h) * DVc + c);
+  }
+  if (tid < n1) S.af[tid] = p.abuf[bh * p.cap + tid];
+  if (tid < nd) {
+    S.ad[tid] = p.alpha[b * p.bs_a + tid * p.H + h];
+    S.bd[tid] = p.beta[b * p.bs_b + tid * p.H + h];
+  }
+  __syncthreads();
+
+  // ---- decay factors (warps 0, 1) and key dots (16 threads per dot)
+  if (warp == 0) {  // fold: R_i = prod_{i<m<n1} alpha_m, gamma = prod_{m<n1} alpha_m
+    double pr = lane < n1 ? (double)S.af[lane] : 1.0;  // inclusive prefix product
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double t = __shfl_up_sync(0xffffffffu, pr, o);
+      if (lane >= o) pr *= t;
+    }
+    const double last = __shfl_sync(0xffffffffu, pr, (n1 > 0 ? n1 : 1) - 1);
+    if (fold && lane < n1) S.Rf[lane] = (float)(last / pr);
+    if (lane == 0) S.gf = (float)last;
+  } else if (warp == 1) {  // drafts: Q_m over the draft sequence, R(e,j) = Q_e / Q_j
+    const float am = lane < nb ? S.af[lane] : (lane < ne ? S.ad[lane - nb] : 1.f);
+    double pr = am;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double t = __shfl_up_sync(0xffffffffu, pr, o);
+      if (lane >= o) pr *= t;
+    }
+#pragma unroll
+    for (int d = 0; d < kVD; ++d) {
+      const double qe = __shfl_sync(0xffffffffu, pr, (nb + d) & 31);
+      if (d < nd) {
+        if (lane <= nb + d) S.R[d][lane] = (float)(qe / pr);
+        if (lane == 0) S.gam[d] = (float)qe;
+      }
+    }
+  }
+  {
+    // dots: (d, j < e_d) keys . k_d, then (d, i <= e_d) keys . q_d
+    const int nkk = nd * nb + nd * (nd - 1) / 2, nkq = nd * nb + nd * (nd + 1) / 2;
+    const int ndot = nkk + nkq;
+    for (int base = 0; base < ndot; base += kThreads / 16) {
+      const int t = base + (tid >> 4), c0 = (tid & 15) * 8;
+      double acc = 0.0, acc1 = 0.0;
+      int d = 0, j = 0;
+      bool isq = false;
+      if (t < ndot) {
+        int r = t < nkk ? t : t - nkk;
+        isq = t >= nkk;
+        // enumerate (d, j): draft d has nb + d (keys) or nb + d + 1 (queries) partners
+        for (d = 0; d < nd; ++d) {
+          const int cnt = nb + d + (isq ? 1 : 0);
+          if (r < cnt) break;
+          r -= cnt;
+        }
+        j = r;
+        const float *kj = j < nb ? S.Kc[j] : S.Kd[j - nb];
+        const float *other = isq ? S.Qd[d] : S.Kd[d];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          acc += (double)(kj[c0 + e] * other[c0 + e]);
+          acc1 += (double)(kj[c0 + e + 1] * other[c0 + e + 1]);
+        }
+        acc += acc1;
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+      if (t < ndot && (tid & 15) == 0) {
+        if (isq) S.KQ[d][j] = (float)acc;
+        else S.G[d][j] = (float)acc;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- commit fold in registers, written once
+  const int row0 = kRows * warp;
+  if (fold) {
+    const float g = S.gf;
+#pragma unroll
+    for (int rho = 0; rho < kRows; ++rho) hv[rho] = mul4x(g, hv[rho]);
+    for (int i = 0; i < n1; ++i) {
+      const float4 ui = *reinterpret_cast<const float4 *>(&S.U[i][4 * lane]);
+      const float ri = S.Rf[i];
+#pragma unroll
+      for (int rho = 0; rho < kRows; ++rho) hv[rho] = fma4x(ri * S.Kc[i][row0 + rho], ui, hv[rho]);
+    }
+#pragma unroll
+    for (int rho = 0; rho < kRows; ++rho)
+      st_stream(tile + (size_t)(row0 + rho) * DVc + 4 * lane, hv[rho]);
+  }
+
+  // ---- h^T k_d and h^T q_d: partial sums over this warp's 16 rows
+  for (int v = 0; v < 2 * nd; ++v) {
+    const float *vec = v < nd ? S.Kd[v] : S.Qd[v - nd];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int rho = 0; rho < kRows; ++rho) acc = fma4x(vec[row0 + rho], hv[rho], acc);
+    *reinterpret_cast<float4 *>(&S.part[warp][v][4 * lane]) = acc;
+  }
+  __syncthreads();
+  for (int e = tid; e < 2 * nd * DVc; e += kThreads) {
+    const int v = e / DVc, c = e % DVc;
+    float zc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) zc += S.part[w][v][c];
+    S.z[v][c] = zc;
+  }
+  __syncthreads();
+
+  // ---- drafts in order: correction u_e, output o_d (one thread per column)
+  if (tid < DVc) {
+    const int c = tid;
+    for (int d = 0; d < nd; ++d) {
+      const int e = nb + d;
+      float a0 = S.Vd[d][c] - S.gam[d] * S.z[d][c], a1 = 0.f;
+      int j = 0;
+      for (; j + 1 < e; j += 2) {
+        a0 = fmaf(-S.R[d][j] * S.G[d][j], S.U[j][c], a0);
+        a1 = fmaf(-S.R[d][j + 1] * S.G[d][j + 1], S.U[j + 1][c], a1);
+      }
+      if (j < e) a0 = fmaf(-S.R[d][j] * S.G[d][j], S.U[j][c], a0);
+      const float u = S.bd[d] * (a0 + a1);
+      S.U[e][c] = u;
+      p.ubuf[(bh * p.cap + e) * DVc + c] = u;
+      float o0 = S.gam[d] * S.z[nd + d][c], o1 = 0.f;
+      int i = 0;
+      for (; i + 1 <= e; i += 2) {
+        o0 = fmaf(S.R[d][i] * S.KQ[d][i], S.U[i][c], o0);
+        o1 = fmaf(S.R[d][i + 1] * S.KQ[d][i + 1], S.U[i + 1][c], o1);
+      }
+      if (i <= e) o0 = fmaf(S.R[d][i] * S.KQ[d][i], S.U[i][c], o0);
+      p.y[b * p.bs_y + (size_t)(d * p.H + h) * DVc + c] = p.scale * (o0 + o1);
+    }
+  }
+  // ---- append the drafts at slots nb .. nb+nd-1 (input values, unrounded)
+  for (int e = tid; e < nd * DKc; e += kThreads) {
+    const int d = e / DKc, c = e % DKc;
+    const int64_t o = (int64_t)(d * p.H + h) * DKc + c;
+    const size_t slot = (bh * p.cap + nb + d) * DKc + c;
+    static_cast<TI *>(p.qbuf)[slot] = static_cast<const TI *>(p.q)[b * p.bs_q + o];
+    static_cast<TI *>(p.kbuf)[slot] = static_cast<const TI *>(p.k)[b * p.bs_k + o];
+    static_cast<TI *>(p.vbuf)[(bh * p.cap + nb + d) * DVc + c] =
+        static_cast<const TI *>(p.v)[b * p.bs_v + (int64_t)(d * p.H + h) * DVc + c];
+  }
+  if (tid < nd) {
+    p.abuf[bh * p.cap + nb + tid] = S.ad[tid];
+    p.bbuf[bh * p.cap + nb + tid] = S.bd[tid];
+  }
+  if (tid == 0) p.len[bh] = nb;
+}
+
+template <typename TI>
+cudaError_t gdn_verify_launch(const GDNParams &p, cudaStream_t s) {
+  const size_t smem = sizeof(GdnVerifySmem);
+  cudaError_t e = cudaFuncSetAttribute(gdn_verify_kernel<TI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  gdn_verify_kernel<TI><<<(unsigned)(p.B * p.H), kThreads, smem, s>>>(p);
+  return cudaGetLastError();
 }
 
 int gdn_sm_count() {
@@ -715,16 +1079,23 @@ int gdn_sm_count() {
   return n > 0 ? n : 148;
 }
 
+// bf16 keys fold on the tensor cores (when the operand area fits beside a
+// ring of at least 4 half-tiles); fp32 keys, which are not exact in bf16, on
+// the SIMT pipes.
 template <typename TI>
 cudaError_t gdn_launch_persistent(const GDNParams &p, cudaStream_t s) {
-  const GdnLayout lay = GdnLayout::make(p.L, (int)sizeof(TI), 220 * 1024);
+  constexpr bool kMma = std::is_same<TI, __nv_bfloat16>::value;
+  GdnLayout lay = GdnLayout::make(p.L, (int)sizeof(TI), 220 * 1024, kMma);
+  const bool mma = kMma && lay.NS >= 4;
+  if (!mma) lay = GdnLayout::make(p.L, (int)sizeof(TI), 220 * 1024);
   if (lay.NS < 4) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(gdn_decode_kernel<TI>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+  auto kernel = mma ? gdn_decode_kernel<TI, kMma> : gdn_decode_kernel<TI, false>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
   if (e != cudaSuccess) return e;
   const int nitems = p.B * p.H;
   const int grid = nitems < gdn_sm_count() ? nitems : gdn_sm_count();
-  gdn_decode_kernel<TI><<<grid, kThreads + 64, lay.total, s>>>(p, lay);
+  kernel<<<grid, kThreads + 64, lay.total, s>>>(p, lay);
   return cudaGetLastError();
 }
 
@@ -741,12 +1112,18 @@ cudaError_t gdn_launch_fold(const GDNParams &p, int mode, cudaStream_t s) {
   if (p.B * p.H == 0) return cudaSuccess;
   if (mode == kFoldFlush) return launch_dt<kGdnFlush>(p, s);
   if (mode == kFoldMaterialize) return launch_dt<kGdnMaterialize>(p, s);
+  if (mode == kFoldCommit) return launch_dt<kGdnCommit>(p, s);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t gdn_launch_full(const GDNParams &p, cudaStream_t s) {
   if (p.B * p.H == 0) return cudaSuccess;
   return launch_dt<kGdnFull>(p, s);
+}
+
+cudaError_t gdn_launch_verify(const GDNParams &p, cudaStream_t s) {
+  if (p.B * p.H == 0) return cudaSuccess;
+  return p.in_bf16 ? gdn_verify_launch<__nv_bfloat16>(p, s) : gdn_verify_launch<float>(p, s);
 }
 
 }  // namespace rssm

@@ -63,6 +63,9 @@ struct GDNParams {
   int step_index;
   uint64_t wait_ns;  // as in M2Params
   int hold_item;
+  // speculative rounds
+  const int32_t *acc;
+  int draft_max, n_draft;
 };
 
 enum FoldMode { kFoldFlush = 0, kFoldCommit = 1, kFoldMaterialize = 2 };
@@ -77,6 +80,7 @@ bool m2_heads_supported(int hpg);  // heads per group: <= 8 or a multiple of 8
 cudaError_t gdn_launch_decode(const GDNParams &p, cudaStream_t s);
 cudaError_t gdn_launch_fold(const GDNParams &p, int mode, cudaStream_t s);
 cudaError_t gdn_launch_full(const GDNParams &p, cudaStream_t s);
+cudaError_t gdn_launch_verify(const GDNParams &p, cudaStream_t s);
 bool gdn_supported(int DK, int DV);
 
 // Read copy of ntile tiles [rows][cols]; fmt 1 = FP8, 2 = NVFP4.  With

@@ -368,14 +368,20 @@ __device__ __forceinline__ void fold_epilogue(const M2Params &p, size_t bh, cons
   float amax = 0.f;
 #pragma unroll 1
   for (int c = 0; c < CW; c += 32) {
-    float d[32];
+    // all 32 old values first: the stores below (the byte stores of the copy
+    // may alias anything) would otherwise serialise every load behind them
+    float t[32], d[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int r = r0 + c + i;
+      t[i] = QM == 0 ? tile[r * N + n] : __ldcs(hg + r * N + n);
+    }
     umma::ld32(taddr + c, d);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int r = r0 + c + i;
-      const float t = QM == 0 ? tile[r * N + n] : hg[r * N + n];
-      const float hn = fmaf(lam, t, d[i]);
-      hg[r * N + n] = hn;
+      const float hn = fmaf(lam, t[i], d[i]);
+      __stcs(hg + r * N + n, hn);
       if constexpr (QM == 1) p.rc[bh * (size_t)(P * N) + r * N + n] = (uint8_t)e4m3_encode(hn);
       if constexpr (QM == 2) amax = fmaxf(amax, fabsf(hn));
     }
@@ -390,21 +396,27 @@ __device__ __forceinline__ void fold_epilogue(const M2Params &p, size_t bh, cons
     const float sg = nvfp4_tile_scale(tmax);
     uint8_t *rc = p.rc + bh * (size_t)(P * N / 2);
     uint8_t *sc = p.rc_scale + bh * (size_t)(P * N / 16);
-#pragma unroll 4
-    for (int i = 0; i < CW; ++i) {
-      const int r = r0 + i;
-      const float hn = hg[r * N + n];  // this thread's own store
-      float bm = fabsf(hn);
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
-      const uint32_t scode = nvfp4_block_code(bm, sg);
-      const float dstep = nvfp4_step(scode, sg);
-      const float qv = dstep > 0.f ? __fdiv_rn(hn, dstep) : 0.f;
-      const float qn = __shfl_xor_sync(0xffffffffu, qv, 1);
-      if ((lane & 1) == 0) rc[r * (N / 2) + n / 2] = (uint8_t)e2m1x2_encode(qv, qn);
-      if ((lane & 15) == 0) sc[r * (N / 16) + n / 16] = (uint8_t)scode;
+#pragma unroll 1
+    for (int c = 0; c < CW; c += 32) {
+      float hv[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) hv[i] = hg[(r0 + c + i) * N + n];  // this thread's own stores
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = r0 + c + i;
+        const float hn = hv[i];
+        float bm = fabsf(hn);
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+        const uint32_t scode = nvfp4_block_code(bm, sg);
+        const float dstep = nvfp4_step(scode, sg);
+        const float qv = dstep > 0.f ? __fdiv_rn(hn, dstep) : 0.f;
+        const float qn = __shfl_xor_sync(0xffffffffu, qv, 1);
+        if ((lane & 1) == 0) rc[r * (N / 2) + n / 2] = (uint8_t)e2m1x2_encode(qv, qn);
+        if ((lane & 15) == 0) sc[r * (N / 16) + n / 16] = (uint8_t)scode;
+      }
     }
     if (sub == 0 && lane == 0) p.rc_gscale[bh] = sg;
     bar_sync(2 + hq, WPH * 32);  // red[] is reused by the group's next head

@@ -295,20 +295,24 @@ def replayssm_flush(layer: Layer, state: ReplayState, A: torch.Tensor | None = N
 
 def replayssm_verify_commit(layer: Layer, state: ReplayState, accepted_prev, drafts: dict,
                             y: torch.Tensor, stream=None):
-    """drafts: x [B,n,H,P], dt [B,n,H], Bm/Cm [B,n,G,N], A, D; y [B,n,H,P]."""
+    """Mamba-2 drafts: x [B,n,H,P], dt [B,n,H], Bm/Cm [B,n,G,N], A, D; y [B,n,H,P].
+    Gated DeltaNet drafts: q, k [B,n,H,DK], v [B,n,H,DV], alpha, beta [B,n,H];
+    y [B,n,H,DV]."""
     d, cs = layer.desc(), state.cstate()
-    n = drafts["x"].shape[1]
+    n = drafts["x" if layer.kind == "m2" else "q"].shape[1]
     si = _step_in(layer, drafts, y)
     acc = _dense(accepted_prev, torch.int32, "accepted_prev") if accepted_prev is not None else None
     _ok(lib().replayssm_verify_commit(C.byref(d), C.byref(cs), acc, C.byref(si), int(n),
                                       y.data_ptr(), _stream(stream)), "replayssm_verify_commit")
 
 
-def replayssm_commit(layer: Layer, state: ReplayState, accepted: torch.Tensor, A: torch.Tensor,
-                     stream=None):
+def replayssm_commit(layer: Layer, state: ReplayState, accepted: torch.Tensor,
+                     A: torch.Tensor | None = None, stream=None):
+    """Close a speculative round (A: Mamba-2 decay rates; None for GDN)."""
     d, cs = layer.desc(), state.cstate()
+    a = _dense(A, torch.float32, "A") if A is not None else None
     _ok(lib().replayssm_commit(C.byref(d), C.byref(cs), _dense(accepted, torch.int32, "accepted"),
-                               _dense(A, torch.float32, "A"), _stream(stream)), "replayssm_commit")
+                               a, _stream(stream)), "replayssm_commit")
 
 
 def replayssm_full_decode_step(layer: Layer, S: torch.Tensor, inp: dict, y: torch.Tensor,

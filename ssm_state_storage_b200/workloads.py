@@ -23,6 +23,7 @@ Workloads (sizes of the SSM layer decode step):
                q/k/v, fp32 alpha/beta, fp32 checkpoint, 512 steps, window 16.
   m2_readcopy  m2_serving shapes at batch 64 over 8192 steps.
   m2_verify    m2_serving heads at batch 512, 4 drafts per round, 256 rounds.
+  gdn_verify   gdn_serving heads at batch 256, 4 drafts per round, 256 rounds.
 
 Distributions: x, B, C ~ N(0,1); dt = softplus(N(0,1) - 2);
 A_h = -exp(U(0, ln 16)); D_h ~ N(0,1); initial state 0.1 * N(0,1) (standard
@@ -66,6 +67,8 @@ WORKLOADS = {
     "m2_readcopy": Workload("m2_readcopy", "m2", B=64, H=128, P=64, N=128, G=16, T=8192, seed=1003),
     "m2_verify": Workload("m2_verify", "m2", B=512, H=128, P=64, N=128, G=16, T=256, seed=1004,
                           n_draft=4),
+    "gdn_verify": Workload("gdn_verify", "gdn", B=256, H=32, P=128, N=128, G=32, T=256,
+                           seed=1005, n_draft=4),
 }
 
 
@@ -172,25 +175,30 @@ class Generator:
                     alpha=torch.stack(als), beta=torch.stack(bes))
 
     def rounds(self, R: int):
-        """Next R speculative rounds of a Mamba-2 workload: drafts stacked
-        [R][B][Dn]... plus acceptance lengths acc[R][B] (int32)."""
+        """Next R speculative rounds: drafts stacked [R][B][Dn]... plus
+        acceptance lengths acc[R][B] (int32).  Mamba-2: x, dt, Bm, Cm in the
+        input dtype; GDN: q, k, v in the input dtype, alpha, beta fp32."""
         w = self.w
-        assert w.kind == "m2" and w.n_draft > 0
+        assert w.n_draft > 0
         dt_ = w.in_dtype
-        out = {k: [] for k in ("x", "dt", "Bm", "Cm")}
+        if w.kind == "m2":
+            names, draw = ("x", "dt", "Bm", "Cm"), _Seq.m2_step
+            dts = {k: dt_ for k in names}
+        else:
+            names, draw = ("q", "k", "v", "alpha", "beta"), _Seq.gdn_step
+            dts = {"q": dt_, "k": dt_, "v": dt_, "alpha": F32, "beta": F32}
+        out = {k: [] for k in names}
         accs = []
         for _ in range(R):
             per = {k: [] for k in out}
             acc_r = []
             for s in self._s:
-                ds = [s.m2_step() for _ in range(w.n_draft)]
-                per["x"].append(torch.stack([d[0] for d in ds]))
-                per["dt"].append(torch.stack([d[1] for d in ds]))
-                per["Bm"].append(torch.stack([d[2] for d in ds]))
-                per["Cm"].append(torch.stack([d[3] for d in ds]))
+                ds = [draw(s) for _ in range(w.n_draft)]
+                for i, k in enumerate(names):
+                    per[k].append(torch.stack([d[i] for d in ds]))
                 acc_r.append(s.accept())
             for k in out:
-                out[k].append(torch.stack(per[k]).to(dt_))
+                out[k].append(torch.stack(per[k]).to(dts[k]))
             accs.append(torch.tensor(acc_r, dtype=torch.int32))
         res = {k: torch.stack(v) for k, v in out.items()}
         res["acc"] = torch.stack(accs)

@@ -62,7 +62,9 @@ def test_validation_and_sizes(lib):
     g = rs.Layer("gdn", 8, 32, 128, 128)
     assert rs.replayssm_validate(g) == 0 and g.capacity() == 16
     assert rs.replayssm_validate(rs.Layer("gdn", 8, 32, 64, 128)) == 2
-    assert rs.replayssm_validate(rs.Layer("gdn", 8, 32, 128, 128, draft_max=2)) == 8
+    assert rs.replayssm_validate(rs.Layer("gdn", 8, 32, 128, 128, draft_max=2)) == 0
+    assert rs.Layer("gdn", 8, 32, 128, 128, draft_max=4).capacity() == 19
+    assert rs.replayssm_validate(rs.Layer("gdn", 8, 32, 128, 128, read_fmt="fp8")) == 8
     assert rs.replayssm_status_string(9) == "buffer state out of range"
 
 
@@ -106,9 +108,13 @@ def test_empty_batch_returns_ok_without_reading_pointers(lib):
     assert lib.replayssm_verify_commit(C.byref(d), C.byref(st), None, C.byref(si), 4, None,
                                        None) == 0
     assert lib.replayssm_commit(C.byref(d), C.byref(st), None, None, None) == 0
-    g = rs.Layer("gdn", 0, 32, 128, 128).desc()
+    g = rs.Layer("gdn", 0, 32, 128, 128, draft_max=4).desc()
+    assert lib.replayssm_verify_commit(C.byref(g), C.byref(st), None, C.byref(si), 4, None,
+                                       None) == 0
+    assert lib.replayssm_commit(C.byref(g), C.byref(st), None, None, None) == 0
+    g = rs.Layer("gdn", 0, 32, 128, 128, read_fmt="fp8").desc()
     assert lib.replayssm_verify_commit(C.byref(g), C.byref(st), None, C.byref(si), 1, None,
-                                       None) == 8          # unsupported for GDN
+                                       None) == 8          # no GDN read copy
 
 
 @pytest.mark.skipif(torch.cuda.is_available(),

@@ -54,6 +54,12 @@ def lib():
         L.oracle_gdn_verify_snapshot.argtypes = [i, i, i, i, i, i, C.c_double, dp, dp, dp, dp,
                                                  dp, dp, ip, dp, lp]
         L.oracle_gdn_materialize.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, ip, dp]
+        L.oracle_kda_conventional.argtypes = [i, i, i, i, i, C.c_double, dp, dp, dp, dp, dp, dp,
+                                              dp, lp, lp]
+        L.oracle_kda_replay.argtypes = [i, i, i, i, i, i, i, C.c_double, dp, dp, dp, dp, dp, dp,
+                                        ip, dp, dp, dp, dp, dp, dp, ip, ip, lp, lp]
+        L.oracle_kda_flush.argtypes = [i, i, i, i, i, i, i, dp, dp, dp, dp, dp, ip]
+        L.oracle_kda_materialize.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, ip, dp]
         L.oracle_e4m3_encode.argtypes = [C.c_float]
         L.oracle_e4m3_encode.restype = C.c_uint8
         L.oracle_e4m3_decode.argtypes = [C.c_uint8]
@@ -265,6 +271,67 @@ class GDNReplay:
         _check(lib().oracle_gdn_materialize(self.B, self.H, self.DK, self.DV, self.cap, self.h0,
                                             self.rec_k, self.rec_v, self.rec_alpha,
                                             self.rec_beta, self.len, S), "gdn_materialize")
+        return S
+
+
+# ---------------------------------------------------------- Kimi Delta Attention
+
+def kda_conventional(S0, q, k, v, alpha, beta, scale=1.0):
+    """Token-by-token gated delta rule with per-channel decay alpha [T,B,H,DK].
+    Returns (o[T,B,H,DV], S_final, reads, writes)."""
+    S = _f64(S0).copy()
+    q, k, v, alpha, beta = map(_f64, (q, k, v, alpha, beta))
+    T, B, H, DK = q.shape
+    DV = v.shape[3]
+    o = np.zeros((T, B, H, DV))
+    rd = np.zeros((B, H), np.int64)
+    wr = np.zeros((B, H), np.int64)
+    _check(lib().oracle_kda_conventional(T, B, H, DK, DV, float(scale), S, q, k, v, alpha, beta,
+                                         o, rd, wr), "kda_conventional")
+    return o, S, rd, wr
+
+
+class KDAReplay:
+    """Checkpoint + record buffer (q, k, v, per-channel alpha, beta) for every
+    (sequence, head) of a Kimi Delta Attention layer."""
+
+    def __init__(self, h0, L=16, cap=None, scale=1.0):
+        self.h0 = _f64(h0).copy()
+        B, H, DK, DV = self.h0.shape
+        self.B, self.H, self.DK, self.DV = B, H, DK, DV
+        self.L, self.cap, self.scale = L, (cap if cap is not None else L), float(scale)
+        cap = self.cap
+        self.rec_q = np.zeros((B, H, cap, DK))
+        self.rec_k = np.zeros((B, H, cap, DK))
+        self.rec_v = np.zeros((B, H, cap, DV))
+        self.rec_alpha = np.zeros((B, H, cap, DK))
+        self.rec_beta = np.zeros((B, H, cap))
+        self.len = np.zeros((B, H), np.int32)
+        self.reads = np.zeros((B, H), np.int64)
+        self.writes = np.zeros((B, H), np.int64)
+
+    def decode(self, q, k, v, alpha, beta):
+        q, k, v, alpha, beta = map(_f64, (q, k, v, alpha, beta))
+        T = q.shape[0]
+        o = np.zeros((T, self.B, self.H, self.DV))
+        lt = np.zeros((T, self.B, self.H), np.int32)
+        ft = np.zeros((T, self.B, self.H), np.int32)
+        _check(lib().oracle_kda_replay(T, self.B, self.H, self.DK, self.DV, self.L, self.cap,
+                                       self.scale, self.h0, self.rec_q, self.rec_k, self.rec_v,
+                                       self.rec_alpha, self.rec_beta, self.len, q, k, v, alpha,
+                                       beta, o, lt, ft, self.reads, self.writes), "kda_replay")
+        return o, lt, ft
+
+    def flush(self, force=False):
+        _check(lib().oracle_kda_flush(self.B, self.H, self.DK, self.DV, self.L, self.cap,
+                                      int(force), self.h0, self.rec_k, self.rec_v,
+                                      self.rec_alpha, self.rec_beta, self.len), "kda_flush")
+
+    def materialize(self):
+        S = np.zeros_like(self.h0)
+        _check(lib().oracle_kda_materialize(self.B, self.H, self.DK, self.DV, self.cap, self.h0,
+                                            self.rec_k, self.rec_v, self.rec_alpha,
+                                            self.rec_beta, self.len, S), "kda_materialize")
         return S
 
 

@@ -650,6 +650,197 @@ int oracle_gdn_materialize(int B, int H, int DK, int DV, int cap,
 /*                    Low-precision formats [OCP MX v1.0]                 */
 /* ===================================================================== */
 
+
+/* ----------------------------------------------------- Kimi Delta Attention
+ * The third layer type the pages name [hamidun §Why hybrid models became the
+ * norm]: the gated delta rule with a decay per key channel instead of one
+ * scalar (Kimi Linear, Moonshot AI 2025).  State S [DK][DV], alpha_t in
+ * (0,1)^DK:
+ *   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *   o_t = scale S_t^T q_t.
+ * Replay form, written out here step by step from h0 (Gamma_i = the running
+ * elementwise product alpha_0 .. alpha_i, formed directly):
+ *   u_i = beta_i (v_i - h0^T (Gamma_i o k_i)
+ *                 - sum_{j<i} [sum_r k_j[r] (prod_{j<m<=i} alpha_m[r]) k_i[r]] u_j)
+ *   o   = scale (h0^T (Gamma_t o q) + sum_{i<=t} [sum_r k_i[r] (prod_{i<m<=t} alpha_m[r]) q[r]] u_i)
+ * and the fold steps the recurrence through the records. */
+static void kda_step(int DK, int DV, double *s, const double *kv, const double *vv,
+                     const double *av, double beta, double *w) {
+  for (int r = 0; r < DK; ++r)
+    for (int j = 0; j < DV; ++j) s[(size_t)r * DV + j] *= av[r];
+  for (int j = 0; j < DV; ++j) {
+    double acc = 0.0;
+    for (int r = 0; r < DK; ++r) acc += kv[r] * s[(size_t)r * DV + j];
+    w[j] = acc;
+  }
+  for (int r = 0; r < DK; ++r)
+    for (int j = 0; j < DV; ++j)
+      s[(size_t)r * DV + j] += beta * kv[r] * (vv[j] - w[j]);
+}
+
+/* prod_{a < m <= b} alpha_m[r] over records (a = -1: from the first) */
+static double kda_ratio(int DK, const double *ra, int a, int b, int r) {
+  double p = 1.0;
+  for (int m = a + 1; m <= b; ++m) p *= ra[(size_t)m * DK + r];
+  return p;
+}
+
+static void kda_replay_out(int DK, int DV, int kc, double scale, const double *h0,
+                           const double *rq, const double *rk, const double *rv,
+                           const double *ra, const double *rb, double *o, double *u,
+                           double *z) {
+  for (int i = 0; i < kc; ++i) {
+    const double *ki = rk + (size_t)i * DK;
+    for (int j = 0; j < DV; ++j) {
+      double acc = 0.0;
+      for (int r = 0; r < DK; ++r) acc += h0[(size_t)r * DV + j] * kda_ratio(DK, ra, -1, i, r) * ki[r];
+      z[j] = acc;
+    }
+    double *ui = u + (size_t)i * DV;
+    for (int j = 0; j < DV; ++j) ui[j] = rv[(size_t)i * DV + j] - z[j];
+    for (int jj = 0; jj < i; ++jj) {
+      double kk = 0.0;
+      for (int r = 0; r < DK; ++r)
+        kk += rk[(size_t)jj * DK + r] * kda_ratio(DK, ra, jj, i, r) * ki[r];
+      for (int j = 0; j < DV; ++j) ui[j] -= kk * u[(size_t)jj * DV + j];
+    }
+    for (int j = 0; j < DV; ++j) ui[j] *= rb[i];
+  }
+  const double *qk = rq + (size_t)(kc - 1) * DK;
+  for (int j = 0; j < DV; ++j) {
+    double acc = 0.0;
+    for (int r = 0; r < DK; ++r) acc += h0[(size_t)r * DV + j] * kda_ratio(DK, ra, -1, kc - 1, r) * qk[r];
+    o[j] = acc;
+  }
+  for (int i = 0; i < kc; ++i) {
+    double kq = 0.0;
+    for (int r = 0; r < DK; ++r)
+      kq += rk[(size_t)i * DK + r] * kda_ratio(DK, ra, i, kc - 1, r) * qk[r];
+    for (int j = 0; j < DV; ++j) o[j] += kq * u[(size_t)i * DV + j];
+  }
+  for (int j = 0; j < DV; ++j) o[j] *= scale;
+}
+
+static void kda_fold(int DK, int DV, double *h0, int kc, const double *rk, const double *rv,
+                     const double *ra, const double *rb, double *w) {
+  for (int i = 0; i < kc; ++i)
+    kda_step(DK, DV, h0, rk + (size_t)i * DK, rv + (size_t)i * DV, ra + (size_t)i * DK, rb[i], w);
+}
+
+int oracle_kda_conventional(int T, int B, int H, int DK, int DV, double scale, double *S,
+                            const double *q, const double *k, const double *v,
+                            const double *alpha, const double *beta, double *o,
+                            long long *reads, long long *writes) {
+  if (T < 0 || B < 0 || H <= 0 || DK <= 0 || DV <= 0) return -1;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h) {
+      const size_t bh = ix2(b, H, h);
+      double *s = S + bh * DK * DV;
+      double *w = (double *)malloc(sizeof(double) * DV);
+      for (int t = 0; t < T; ++t) {
+        const size_t tbh = ((size_t)t * B + b) * H + h;
+        kda_step(DK, DV, s, k + tbh * DK, v + tbh * DV, alpha + tbh * DK, beta[tbh], w);
+        for (int j = 0; j < DV; ++j) {
+          double acc = 0.0;
+          for (int r = 0; r < DK; ++r) acc += s[(size_t)r * DV + j] * q[tbh * DK + r];
+          o[tbh * DV + j] = scale * acc;
+        }
+        if (reads) reads[bh] += 1;
+        if (writes) writes[bh] += 1;
+      }
+      free(w);
+    }
+  return 0;
+}
+
+int oracle_kda_replay(int T, int B, int H, int DK, int DV, int L, int cap, double scale,
+                      double *h0, double *rec_q, double *rec_k, double *rec_v,
+                      double *rec_alpha, double *rec_beta, int *len, const double *q,
+                      const double *k, const double *v, const double *alpha,
+                      const double *beta, double *o, int *len_trace, int *flush_trace,
+                      long long *reads, long long *writes) {
+  if (T < 0 || B < 0 || H <= 0 || DK <= 0 || DV <= 0 || L <= 0 || cap < L || cap > MAXCAP)
+    return -1;
+  int bad = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : bad)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h) {
+      const size_t bh = ix2(b, H, h);
+      double *hh = h0 + bh * DK * DV;
+      double *rq = rec_q + bh * cap * DK, *rk = rec_k + bh * cap * DK;
+      double *rv = rec_v + bh * cap * DV, *ra = rec_alpha + bh * cap * DK;
+      double *rb = rec_beta + bh * cap;
+      double *u = (double *)malloc(sizeof(double) * cap * DV);
+      double *z = (double *)malloc(sizeof(double) * DV);
+      int n = len[bh];
+      for (int t = 0; t < T && !bad; ++t) {
+        if (n < 0 || n >= L) { bad |= 1; break; }
+        const size_t tbh = ((size_t)t * B + b) * H + h;
+        /* append the step's record [sitech §How ReplaySSM works] */
+        memcpy(rq + (size_t)n * DK, q + tbh * DK, sizeof(double) * DK);
+        memcpy(rk + (size_t)n * DK, k + tbh * DK, sizeof(double) * DK);
+        memcpy(rv + (size_t)n * DV, v + tbh * DV, sizeof(double) * DV);
+        memcpy(ra + (size_t)n * DK, alpha + tbh * DK, sizeof(double) * DK);
+        rb[n] = beta[tbh];
+        ++n;
+        kda_replay_out(DK, DV, n, scale, hh, rq, rk, rv, ra, rb, o + tbh * DV, u, z);
+        if (reads) reads[bh] += 1;
+        int flushed = 0;
+        if (n == L) {
+          kda_fold(DK, DV, hh, n, rk, rv, ra, rb, z);
+          n = 0;
+          flushed = 1;
+          if (writes) writes[bh] += 1;
+        }
+        if (len_trace) len_trace[tbh] = n;
+        if (flush_trace) flush_trace[tbh] = flushed;
+      }
+      len[bh] = n;
+      free(u);
+      free(z);
+    }
+  return bad ? -1 : 0;
+}
+
+int oracle_kda_flush(int B, int H, int DK, int DV, int L, int cap, int force, double *h0,
+                     const double *rec_k, const double *rec_v, const double *rec_alpha,
+                     const double *rec_beta, int *len) {
+  if (B < 0 || H <= 0 || DK <= 0 || DV <= 0 || cap > MAXCAP) return -1;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h) {
+      const size_t bh = ix2(b, H, h);
+      const int n = len[bh];
+      if (n < 0 || n > cap) return -1;
+      if (!(n >= L || (force && n > 0))) continue;
+      double *w = (double *)malloc(sizeof(double) * DV);
+      kda_fold(DK, DV, h0 + bh * DK * DV, n, rec_k + bh * cap * DK, rec_v + bh * cap * DV,
+               rec_alpha + bh * cap * DK, rec_beta + bh * cap, w);
+      free(w);
+      len[bh] = 0;
+    }
+  return 0;
+}
+
+int oracle_kda_materialize(int B, int H, int DK, int DV, int cap, const double *h0,
+                           const double *rec_k, const double *rec_v, const double *rec_alpha,
+                           const double *rec_beta, const int *len, double *S_out) {
+  if (B < 0 || H <= 0 || DK <= 0 || DV <= 0 || cap > MAXCAP) return -1;
+  memcpy(S_out, h0, sizeof(double) * (size_t)B * H * DK * DV);
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h) {
+      const size_t bh = ix2(b, H, h);
+      const int n = len[bh];
+      if (n < 0 || n > cap) return -1;
+      double *w = (double *)malloc(sizeof(double) * DV);
+      kda_fold(DK, DV, S_out + bh * DK * DV, n, rec_k + bh * cap * DK, rec_v + bh * cap * DV,
+               rec_alpha + bh * cap * DK, rec_beta + bh * cap, w);
+      free(w);
+    }
+  return 0;
+}
+
+
 /* FP8 E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits; exponent field 0
  * holds subnormals m/8 * 2^-6; S.1111.111 is NaN; no infinities; the largest
  * finite magnitude is 1.75 * 2^8 = 448 (code 0x7E). */

@@ -1,6 +1,7 @@
 /*
  * oracle.h -- plain, slow, fp64 CPU model of the ReplaySSM SSM-layer decode
- * step (Mamba-2 and Gated DeltaNet), used to check the CUDA path.
+ * step (Mamba-2, Gated DeltaNet, Kimi Delta Attention), used to check the
+ * CUDA path.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may include, link or
  * call this code: only the tests, the smoke check and the CPU-baseline leg of
@@ -18,6 +19,8 @@
  *               para acelerar modelos híbridos", body paragraphs 2-3.
  *   [Dao & Gu 2024]  "Transformers are SSMs" -- the Mamba-2 (SSD) recurrence.
  *   [Yang et al. 2025] "Gated Delta Networks" -- the gated delta rule.
+ *   [Kimi Linear 2025] Moonshot AI, "Kimi Linear" -- Kimi Delta Attention,
+ *                    the gated delta rule with a per-channel decay.
  *   [OCP MX v1.0]    OCP Microscaling Formats spec -- FP8 E4M3 / FP4 E2M1.
  *
  * Layout conventions (all arrays dense, row-major, the last index innermost):
@@ -124,6 +127,34 @@ int oracle_gdn_flush(int B, int H, int DK, int DV, int L, int cap, int force,
                      const double *rec_alpha, const double *rec_beta, int *len);
 
 int oracle_gdn_materialize(int B, int H, int DK, int DV, int cap,
+                           const double *h0, const double *rec_k,
+                           const double *rec_v, const double *rec_alpha,
+                           const double *rec_beta, const int *len,
+                           double *S_out);
+
+/* ----------------------------------------------------- Kimi Delta Attention
+ * Gated delta rule with a per-key-channel decay: alpha [T][B][H][DK] (and
+ * rec_alpha [B][H][cap][DK]); other layouts as for Gated DeltaNet. */
+
+int oracle_kda_conventional(int T, int B, int H, int DK, int DV, double scale,
+                            double *S, const double *q, const double *k,
+                            const double *v, const double *alpha,
+                            const double *beta, double *o,
+                            long long *reads, long long *writes);
+
+int oracle_kda_replay(int T, int B, int H, int DK, int DV, int L, int cap,
+                      double scale, double *h0, double *rec_q, double *rec_k,
+                      double *rec_v, double *rec_alpha, double *rec_beta,
+                      int *len, const double *q, const double *k,
+                      const double *v, const double *alpha, const double *beta,
+                      double *o, int *len_trace, int *flush_trace,
+                      long long *reads, long long *writes);
+
+int oracle_kda_flush(int B, int H, int DK, int DV, int L, int cap, int force,
+                     double *h0, const double *rec_k, const double *rec_v,
+                     const double *rec_alpha, const double *rec_beta, int *len);
+
+int oracle_kda_materialize(int B, int H, int DK, int DV, int cap,
                            const double *h0, const double *rec_k,
                            const double *rec_v, const double *rec_alpha,
                            const double *rec_beta, const int *len,

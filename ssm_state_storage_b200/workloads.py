@@ -24,12 +24,14 @@ Workloads (sizes of the SSM layer decode step):
   m2_readcopy  m2_serving shapes at batch 64 over 8192 steps.
   m2_verify    m2_serving heads at batch 512, 4 drafts per round, 256 rounds.
   gdn_verify   gdn_serving heads at batch 256, 4 drafts per round, 256 rounds.
+  kda_serving  Kimi Delta Attention on the gdn_serving shapes (batch 256, 32
+               heads, d_k = d_v = 128), one decay per key channel.
 
 Distributions: x, B, C ~ N(0,1); dt = softplus(N(0,1) - 2);
 A_h = -exp(U(0, ln 16)); D_h ~ N(0,1); initial state 0.1 * N(0,1) (standard
 deviation 0.1); GDN q, k ~ N(0,1) then L2-normalised; v ~ N(0,1);
-alpha = exp(-softplus(N(0,1))); beta = sigmoid(N(0,1)); verify acceptance
-length ~ Uniform{0..n_draft}.
+alpha = exp(-softplus(N(0,1))) (KDA: drawn per key channel); beta =
+sigmoid(N(0,1)); verify acceptance length ~ Uniform{0..n_draft}.
 """
 from __future__ import annotations
 
@@ -69,6 +71,8 @@ WORKLOADS = {
                           n_draft=4),
     "gdn_verify": Workload("gdn_verify", "gdn", B=256, H=32, P=128, N=128, G=32, T=256,
                            seed=1005, n_draft=4),
+    "kda_serving": Workload("kda_serving", "kda", B=256, H=32, P=128, N=128, G=32, T=512,
+                            seed=1006),
 }
 
 
@@ -112,7 +116,7 @@ class _Seq:
         q = self.n(w.H, w.N)
         k = self.n(w.H, w.N)
         v = self.n(w.H, w.P)
-        a = torch.exp(-_softplus(self.n(w.H)))
+        a = torch.exp(-_softplus(self.n(w.H, w.N) if w.kind == "kda" else self.n(w.H)))
         be = torch.sigmoid(self.n(w.H))
         q = q / q.norm(dim=-1, keepdim=True)
         k = k / k.norm(dim=-1, keepdim=True)

@@ -357,6 +357,8 @@ def run_ours(args, rank, world):
         torch.cuda.empty_cache()
         line["gdn"] = bench_gdn(args, dev, peak, rs, bm, wl, torch)
         torch.cuda.empty_cache()
+        line["kda"] = bench_kda(args, dev, peak, rs, bm, wl, torch)
+        torch.cuda.empty_cache()
         line["verify"] = bench_verify(args, dev, peak, rs, bm, wl, torch)
         torch.cuda.empty_cache()
         line["verify_gdn"] = bench_verify_gdn(args, dev, peak, rs, bm, wl, torch)
@@ -513,6 +515,59 @@ def bench_gdn(args, dev, peak, rs, bm, wl, torch):
             "step_times": steps_us,
             "bytes_per_head_token": {"replay": wb / (w.B * w.H * L),
                                      "replay_input_records_only": wb_rec / (w.B * w.H * L),
+                                     "full_state": fb / (w.B * w.H * L)},
+            "gpu_launches": n * L}
+
+
+def bench_kda(args, dev, peak, rs, bm, wl, torch):
+    """kda_serving: Kimi Delta Attention, batch 256, 32 heads, 128 x 128
+    state, one decay per key channel; replay against the conventional step."""
+    w = wl.make("kda_serving")
+    L, pool = w.L, 4 * w.L
+    g = wl.Generator(w)
+    S0 = g.initial_state()
+    st = {k: v.to(dev) for k, v in g.steps(pool).items()}
+    layer = rs.Layer("kda", w.B, w.H, w.P, w.N, window=L, in_dtype=w.in_dtype)
+    state = rs.ReplayState(layer, device=dev)
+    rs.replayssm_init(layer, state, S0.to(dev))
+    S = S0.to(dev)
+    o = torch.empty(w.B, w.H, w.P, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    step_in = [{k: st[k][t] for k in st} for t in range(pool)]
+
+    def replay_window(wi):
+        for j in range(L):
+            rs.replayssm_decode_step(layer, state, step_in[(wi * L + j) % pool], o, stream)
+
+    def full_window(wi):
+        for j in range(L):
+            rs.replayssm_full_decode_step(layer, S, step_in[(wi * L + j) % pool], o, stream=stream)
+
+    n = args.sub_steps
+    for i in range(3):
+        replay_window(i)
+        full_window(i)
+    ms_r = _events_ms(replay_window, n, stream, torch, dev)
+    ms_f = _events_ms(full_window, n, stream, torch, dev)
+    steps_us = per_launch_us(lambda i: rs.replayssm_decode_step(layer, state, step_in[i % pool], o,
+                                                                stream), L, 10, stream, torch, dev)
+    if state.status() != 0:
+        raise RuntimeError(f"device status {state.status()} after the KDA run")
+    wb = bm.kda_replay_window_bytes(L, w.N, w.P, 2) * w.B * w.H
+    fb = bm.kda_conventional_bytes(w.N, w.P, 2) * w.B * w.H * L
+    ach_r = wb / (ms_r / n * 1e-3) / 1e9
+    ach_f = fb / (ms_f / n * 1e-3) / 1e9
+    tok = w.B * L * n
+    return {"workload": "kda_serving", "value": tok / (ms_r * 1e-3), "unit": "tokens/s",
+            "ms_per_window": ms_r / n,
+            "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
+                         "frac": ach_r / peak, "kernel": "kda_kernel<decode>"},
+            "full_state": {"value": tok / (ms_f * 1e-3), "unit": "tokens/s",
+                           "achieved_gbs": ach_f, "frac": ach_f / peak,
+                           "kernel": "kda_kernel<full>"},
+            "replay_over_full": ms_f / ms_r,
+            "step_times": steps_us,
+            "bytes_per_head_token": {"replay": wb / (w.B * w.H * L),
                                      "full_state": fb / (w.B * w.H * L)},
             "gpu_launches": n * L}
 

@@ -53,6 +53,10 @@
  *            Step inputs q, k [B][H][DK], v [B][H][DV] of in_dtype (q, k
  *            already L2-normalised); alpha, beta [B][H] fp32.
  *            Output o [B][H][DV] fp32 = scale * S^T q.
+ *   KDA:     Kimi Delta Attention [hamidun §Why hybrid models became the
+ *            norm], the gated delta rule with one decay per key channel,
+ *            S <- (I - beta k k^T) Diag(alpha) S + beta k v^T, o = scale S^T q:
+ *            layouts as for GDN except alpha [B][H][DK] fp32.
  *   Buffer capacity per (sequence, head): cap = window + max(draft_max-1, 0).
  */
 #ifndef REPLAYSSM_H
@@ -78,7 +82,7 @@ typedef enum {
   RSSM_ERR_STATE = 9        /* device: buffer state out of range (status)    */
 } rssm_status;
 
-typedef enum { RSSM_MAMBA2 = 0, RSSM_GDN = 1 } rssm_kind;
+typedef enum { RSSM_MAMBA2 = 0, RSSM_GDN = 1, RSSM_KDA = 2 } rssm_kind;
 typedef enum { RSSM_F32 = 0, RSSM_BF16 = 1 } rssm_dtype;
 typedef enum { RSSM_FMT_NONE = 0, RSSM_FMT_FP8 = 1, RSSM_FMT_NVFP4 = 2 } rssm_fmt;
 
@@ -91,7 +95,7 @@ typedef struct {
   int32_t dstate;    /* Mamba-2 N (64 or 128); GDN DK (128)                      */
   int32_t ngroups;   /* Mamba-2 G (H % G == 0, H/G <= 16); GDN: ignored          */
   int32_t window;    /* records per flush, 1..16 (the pages use 16)              */
-  int32_t draft_max; /* most drafts per verify round, 0..4                      */
+  int32_t draft_max; /* most drafts per verify round, 0..4 (KDA: 0)             */
   int32_t in_dtype;  /* rssm_dtype of the step inputs                            */
   int32_t read_fmt;  /* rssm_fmt of the read copy (Mamba-2 only)                 */
   int32_t ckpt_fmt;  /* rssm_fmt the checkpoint is rounded to at each fold: the
@@ -110,7 +114,8 @@ typedef struct {
  *            buf[2] v  [B][H][cap][DV] in_dtype
  *            buf[3] alpha [B][H][cap]  fp32
  *            buf[4] beta  [B][H][cap]  fp32
- *            buf[5] u  [B][H][cap][DV] fp32: per record i, the delta-rule
+ *   KDA:     as GDN, with buf[3] alpha [B][H][cap][DK] fp32 (per channel)
+ *   GDN/KDA: buf[5] u  [B][H][cap][DV] fp32: per record i, the delta-rule
  *                   correction u_i = beta_i (v_i - (state before i)^T k_i)
  *                   expressed from h0 and records 0..i (see replayssm_decode_step);
  *                   it depends only on h0 and those records, so it is computed

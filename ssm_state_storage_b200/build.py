@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 OBJDIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libreplayssm.so")
 
-SOURCES = ["api.cu", "m2.cu", "m2_verify.cu", "gdn.cu", "quant.cu"]
+SOURCES = ["api.cu", "m2.cu", "m2_verify.cu", "gdn.cu", "kda.cu", "quant.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE,

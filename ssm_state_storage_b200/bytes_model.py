@@ -121,3 +121,28 @@ def gdn_verify_round_bytes(n1, fold, nd, DK, DV, in_bytes):
     draft = (2 * DK + DV) * in_bytes + 8
     return (state + n1 * rec + nd * draft + nd * (draft + DV * 4) + nd * DV * 4
             + (state if fold else 0))
+
+
+def kda_conventional_bytes(DK, DV, in_bytes):
+    """Kimi Delta Attention full-state step: read + write the state, read q,
+    k, v, the per-channel decay (fp32) and beta, write the output."""
+    state = DK * DV * 4
+    return 2 * state + (2 * DK + DV) * in_bytes + DK * 4 + 4 + DV * 4
+
+
+def kda_replay_bytes(k, L, DK, DV, in_bytes):
+    """Kimi Delta Attention replay step as the kernel runs it: every past
+    record contributes its key, its per-channel decay and its cached
+    correction; this step reads q, k, v, alpha, beta, appends them with the
+    correction (not on the flush step), writes the output, and on the flush
+    step writes the checkpoint."""
+    state = DK * DV * 4
+    rec_read = DK * in_bytes + DK * 4 + DV * 4
+    cur = (2 * DK + DV) * in_bytes + DK * 4 + 4
+    flush = k == L
+    append = 0 if flush else cur + DV * 4
+    return state + (k - 1) * rec_read + cur + append + DV * 4 + (state if flush else 0)
+
+
+def kda_replay_window_bytes(L, DK, DV, in_bytes):
+    return sum(kda_replay_bytes(k, L, DK, DV, in_bytes) for k in range(1, L + 1))

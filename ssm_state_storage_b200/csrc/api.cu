@@ -23,7 +23,8 @@ inline size_t es_of(const rssm_desc *d) { return d->in_dtype == RSSM_BF16 ? 2 : 
 
 rssm_status check_desc(const rssm_desc *d) {
   if (!d) return RSSM_ERR_INVALID_ARG;
-  if (d->kind != RSSM_MAMBA2 && d->kind != RSSM_GDN) return RSSM_ERR_INVALID_ARG;
+  if (d->kind != RSSM_MAMBA2 && d->kind != RSSM_GDN && d->kind != RSSM_KDA)
+    return RSSM_ERR_INVALID_ARG;
   if (d->batch < 0 || d->nheads <= 0 || d->headdim <= 0 || d->dstate <= 0)
     return RSSM_ERR_INVALID_ARG;
   if (d->in_dtype != RSSM_F32 && d->in_dtype != RSSM_BF16) return RSSM_ERR_DTYPE;
@@ -41,6 +42,7 @@ rssm_status check_desc(const rssm_desc *d) {
   } else {
     if (!gdn_supported(d->dstate, d->headdim)) return RSSM_ERR_SHAPE;
     if (d->read_fmt != RSSM_FMT_NONE || d->ckpt_fmt != RSSM_FMT_NONE) return RSSM_ERR_UNSUPPORTED;
+    if (d->kind == RSSM_KDA && d->draft_max != 0) return RSSM_ERR_UNSUPPORTED;
     if ((int64_t)d->batch * d->nheads > INT32_MAX) return RSSM_ERR_SHAPE;
   }
   return RSSM_OK;
@@ -143,6 +145,7 @@ GDNParams gdn_params(const rssm_desc *d, const rssm_state *s) {
   p.cap = cap_of(d);
   p.in_bf16 = d->in_dtype == RSSM_BF16;
   p.scale = d->scale;
+  p.kda = d->kind == RSSM_KDA;
   p.draft_max = d->draft_max;
   p.wait_ns = g_wait_ns.load();
   p.hold_item = g_hold_item.load();
@@ -173,7 +176,7 @@ rssm_status gdn_inputs(GDNParams &p, const rssm_step_in *in, int nd = 1) {
   p.bs_q = stride_or(in->batch_stride[0], (int64_t)nd * p.H * p.DK);
   p.bs_k = stride_or(in->batch_stride[1], (int64_t)nd * p.H * p.DK);
   p.bs_v = stride_or(in->batch_stride[2], (int64_t)nd * p.H * p.DV);
-  p.bs_a = stride_or(in->batch_stride[3], (int64_t)nd * p.H);
+  p.bs_a = stride_or(in->batch_stride[3], (int64_t)nd * p.H * (p.kda ? p.DK : 1));
   p.bs_b = stride_or(in->batch_stride[4], (int64_t)nd * p.H);
   p.bs_y = stride_or(in->y_batch_stride, (int64_t)nd * p.H * p.DV);
   return RSSM_OK;
@@ -202,7 +205,8 @@ size_t replayssm_state_bytes(const rssm_desc *d, int32_t which) {
     case RSSM_BYTES_BUF0 + 0: return m2 ? B * H * cap * P * es : B * H * cap * N * es;
     case RSSM_BYTES_BUF0 + 1: return m2 ? B * H * cap * 4 : B * H * cap * N * es;
     case RSSM_BYTES_BUF0 + 2: return m2 ? B * G * cap * N * es : B * H * cap * P * es;
-    case RSSM_BYTES_BUF0 + 3: return m2 ? B * G * cap * N * es : B * H * cap * 4;
+    case RSSM_BYTES_BUF0 + 3:
+      return m2 ? B * G * cap * N * es : B * H * cap * (d->kind == RSSM_KDA ? N : 1) * 4;
     case RSSM_BYTES_BUF0 + 4: return m2 ? 0 : B * H * cap * 4;
     case RSSM_BYTES_BUF0 + 5: return m2 ? 0 : B * H * cap * P * 4;
     case RSSM_BYTES_LEN: return B * H * 4;
@@ -281,6 +285,7 @@ rssm_status replayssm_decode_step(const rssm_desc *d, rssm_state *s, const rssm_
   GDNParams p = gdn_params(d, s);
   if ((st = gdn_inputs(p, in)) != RSSM_OK) return st;
   p.y = y;
+  if (p.kda) return from_cuda(kda_launch(p, 0, to_stream(stream)));
   return from_cuda(gdn_launch_decode(p, to_stream(stream)));
 }
 
@@ -299,6 +304,7 @@ rssm_status replayssm_flush(const rssm_desc *d, rssm_state *s, const float *A, i
   }
   GDNParams p = gdn_params(d, s);
   p.force = force != 0;
+  if (p.kda) return from_cuda(kda_launch(p, 1, to_stream(stream)));
   return from_cuda(gdn_launch_fold(p, kFoldFlush, to_stream(stream)));
 }
 
@@ -308,6 +314,7 @@ rssm_status replayssm_verify_commit(const rssm_desc *d, rssm_state *s,
   rssm_status st = check_desc(d);
   if (st != RSSM_OK) return st;
   if (d->read_fmt != RSSM_FMT_NONE || d->ckpt_fmt != RSSM_FMT_NONE) return RSSM_ERR_UNSUPPORTED;
+  if (d->kind == RSSM_KDA) return RSSM_ERR_UNSUPPORTED;
   if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
   if ((st = check_state(d, s)) != RSSM_OK) return st;
   if (n_draft < 1 || n_draft > d->draft_max) return RSSM_ERR_CAPACITY;
@@ -342,6 +349,7 @@ rssm_status replayssm_commit(const rssm_desc *d, rssm_state *s, const int32_t *a
                              const float *A, void *stream) {
   rssm_status st = check_desc(d);
   if (st != RSSM_OK) return st;
+  if (d->kind == RSSM_KDA) return RSSM_ERR_UNSUPPORTED;
   if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
   if ((st = check_state(d, s)) != RSSM_OK) return st;
   if (!accepted) return RSSM_ERR_INVALID_ARG;
@@ -381,6 +389,7 @@ rssm_status replayssm_full_decode_step(const rssm_desc *d, float *S, const rssm_
   p.y = y;
   p.limit = limit;
   p.step_index = step_index;
+  if (p.kda) return from_cuda(kda_launch(p, 3, to_stream(stream)));
   return from_cuda(gdn_launch_full(p, to_stream(stream)));
 }
 
@@ -401,6 +410,7 @@ rssm_status replayssm_materialize(const rssm_desc *d, const rssm_state *s, const
   }
   GDNParams p = gdn_params(d, s);
   p.S_out = S_out;
+  if (p.kda) return from_cuda(kda_launch(p, 2, to_stream(stream)));
   return from_cuda(gdn_launch_fold(p, kFoldMaterialize, to_stream(stream)));
 }
 

@@ -46,6 +46,7 @@ struct M2Params {
 struct GDNParams {
   int B, H, DK, DV, L, cap;
   int in_bf16;
+  int kda;  // Kimi Delta Attention: alpha and its records carry one decay per key channel
   float scale;
   float *h0;
   void *qbuf, *kbuf, *vbuf;
@@ -81,6 +82,10 @@ cudaError_t gdn_launch_decode(const GDNParams &p, cudaStream_t s);
 cudaError_t gdn_launch_fold(const GDNParams &p, int mode, cudaStream_t s);
 cudaError_t gdn_launch_full(const GDNParams &p, cudaStream_t s);
 cudaError_t gdn_launch_verify(const GDNParams &p, cudaStream_t s);
+
+// Kimi Delta Attention (GDNParams with alpha and its records per key channel):
+// mode 0 decode step, 1 flush, 2 materialise, 3 conventional step.
+cudaError_t kda_launch(const GDNParams &p, int mode, cudaStream_t s);
 bool gdn_supported(int DK, int DV);
 
 // Read copy of ntile tiles [rows][cols]; fmt 1 = FP8, 2 = NVFP4.  With

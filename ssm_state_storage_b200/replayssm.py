@@ -39,7 +39,7 @@ STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "unsu
                 4: "pointer not 16-byte aligned", 5: "buffer capacity exceeded",
                 6: "CUDA launch error", 7: "device wait timed out",
                 8: "unsupported by this build", 9: "buffer state out of range"}
-KIND = {"m2": 0, "gdn": 1}
+KIND = {"m2": 0, "gdn": 1, "kda": 2}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 FMT = {"none": 0, "fp8": 1, "nvfp4": 2}
 BYTES = {"h0": 0, "buf0": 1, "buf1": 2, "buf2": 3, "buf3": 4, "buf4": 5, "buf5": 6, "len": 7,
@@ -124,7 +124,7 @@ def _ok(rc: int, what: str):
 @dataclass
 class Layer:
     """One SSM layer's decode-state description (rssm_desc)."""
-    kind: str            # "m2" | "gdn"
+    kind: str            # "m2" | "gdn" | "kda"
     batch: int
     nheads: int
     headdim: int         # M2 P; GDN d_v
@@ -175,10 +175,11 @@ class ReplayState:
                         torch.zeros(B, G, cap, N, dtype=dt_in, device=device)]
         else:
             self.h0 = torch.zeros(B, H, N, P, dtype=f32, device=device)
+            alpha_shape = (B, H, cap, N) if layer.kind == "kda" else (B, H, cap)
             self.buf = [torch.zeros(B, H, cap, N, dtype=dt_in, device=device),
                         torch.zeros(B, H, cap, N, dtype=dt_in, device=device),
                         torch.zeros(B, H, cap, P, dtype=dt_in, device=device),
-                        torch.zeros(B, H, cap, dtype=f32, device=device),
+                        torch.zeros(*alpha_shape, dtype=f32, device=device),
                         torch.zeros(B, H, cap, dtype=f32, device=device),
                         torch.zeros(B, H, cap, P, dtype=f32, device=device)]
         for i, t in enumerate(self.buf):

@@ -12,7 +12,7 @@ def layer_for(w: wl.Workload, **kw) -> rs.Layer:
     if w.kind == "m2":
         return rs.Layer("m2", w.B, w.H, w.P, w.N, ngroups=w.G, window=w.L,
                         draft_max=kw.pop("draft_max", w.n_draft), in_dtype=w.in_dtype, **kw)
-    return rs.Layer("gdn", w.B, w.H, w.P, w.N, window=w.L,
+    return rs.Layer(w.kind, w.B, w.H, w.P, w.N, window=w.L,
                     draft_max=kw.pop("draft_max", w.n_draft), in_dtype=w.in_dtype, **kw)
 
 

@@ -160,3 +160,14 @@ def test_test_hooks_entry_point_validates_and_resets():
         rs.replayssm_set_test_hooks(1000, -2)
     rs.replayssm_set_test_hooks(1000, 3)
     rs.replayssm_set_test_hooks()  # back to the defaults
+
+
+def test_kda_descriptor_and_sizes():
+    from ssm_state_storage_b200 import replayssm as rs
+    L = rs.Layer("kda", 4, 8, 128, 128)
+    assert rs.replayssm_validate(L) == 0
+    assert L.nbytes("buf3") == 4 * 8 * 16 * 128 * 4     # one decay per key channel
+    assert L.nbytes("buf4") == 4 * 8 * 16 * 4
+    assert L.nbytes("buf5") == 4 * 8 * 16 * 128 * 4
+    assert rs.replayssm_validate(rs.Layer("kda", 4, 8, 128, 128, draft_max=2)) == 8
+    assert rs.replayssm_validate(rs.Layer("kda", 4, 8, 64, 128)) == 2

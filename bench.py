@@ -59,35 +59,45 @@ def parse():
     return ap.parse_args()
 
 
-# Sources of m2_decode_kernel: a DRAM-traffic figure recorded under profiles/
-# applies only while their content hash matches the one recorded with it.
-DECODE_SOURCES = ("m2.cu", "m2_device.cuh", "common.cuh", "pipeline.cuh", "codec.cuh",
-                  "internal.h")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "m2_decode_kernel_m2_serving_traffic.txt")
+# Per-kernel DRAM traffic recorded under profiles/ by ncu (one capture at batch 64,
+# scaled to the bench's batch by the number of work items): a figure applies only
+# while the content hash of the kernel's sources equals the one recorded with it.
+KERNEL_SOURCES = {
+    "m2_decode_kernel_m2_serving": ("m2.cu", "m2_device.cuh", "common.cuh", "pipeline.cuh",
+                                    "codec.cuh", "internal.h", "umma.cuh"),
+    "gdn_decode_kernel_gdn_serving": ("gdn.cu", "common.cuh", "pipeline.cuh", "internal.h",
+                                      "umma.cuh"),
+    "kda_kernel_kda_serving": ("kda.cu", "common.cuh", "internal.h"),
+    "m2_verify_kernel_m2_verify": ("m2_verify.cu", "m2_device.cuh", "common.cuh", "pipeline.cuh",
+                                   "codec.cuh", "internal.h"),
+    "gdn_verify_kernel_gdn_verify": ("gdn.cu", "common.cuh", "pipeline.cuh", "internal.h",
+                                     "umma.cuh"),
+}
 
 
-def decode_sources_sha256():
+def sources_sha256(files):
     import hashlib
     h = hashlib.sha256()
-    for name in DECODE_SOURCES:
+    for name in files:
         with open(os.path.join(ROOT, "ssm_state_storage_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def recorded_traffic(batch):
-    """DRAM bytes (read + write) per decode launch at batch 256 from the
-    committed ncu summary, or None when absent, for another batch, or taken on
-    different kernel sources."""
-    if batch != 256 or not os.path.exists(TRAFFIC_FILE):
+def recorded_traffic(record, batch, bench_batch):
+    """DRAM bytes (read + write) per launch at the bench's batch from the
+    committed ncu summary profiles/<record>_traffic.txt, or None when absent,
+    for another batch, or taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", record + "_traffic.txt")
+    if batch != bench_batch or not os.path.exists(path):
         return None
     kv = {}
-    with open(TRAFFIC_FILE) as f:
+    with open(path) as f:
         for line in f:
             parts = line.split()
             if len(parts) == 2 and not line.startswith("#"):
                 kv[parts[0]] = parts[1]
-    if kv.get("source_sha256") != decode_sources_sha256():
+    if kv.get("source_sha256") != sources_sha256(KERNEL_SOURCES[record]):
         return None
     return float(kv["traffic_bytes_per_launch"])
 
@@ -336,7 +346,8 @@ def run_ours(args, rank, world):
                    "step": "one 16-token window = 15 non-flush + 1 flush decode steps",
                    "l2": "inputs larger than L2 (1 GiB checkpoint streamed every step)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic(w.B),
+                     "frac": achieved / peak,
+                     "traffic": recorded_traffic("m2_decode_kernel_m2_serving", w.B, 256),
                      "kernel": "m2_decode_kernel",
                      "peak_source": peak_src,
                      "algorithmic_bytes_per_launch": win_bytes / L},
@@ -505,6 +516,8 @@ def bench_gdn(args, dev, peak, rs, bm, wl, torch):
             "ms_per_window": ms_r / n,
             "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
                          "frac": ach_r / peak, "kernel": "gdn_decode_kernel",
+                         "traffic": recorded_traffic("gdn_decode_kernel_gdn_serving", w.B, 256),
+                         "algorithmic_bytes_per_launch": wb / L,
                          "bytes": "records with their cached corrections u (as stored)",
                          "frac_input_records_only": ach_rec / peak,
                          "achieved_input_records_only": ach_rec},
@@ -561,7 +574,9 @@ def bench_kda(args, dev, peak, rs, bm, wl, torch):
     return {"workload": "kda_serving", "value": tok / (ms_r * 1e-3), "unit": "tokens/s",
             "ms_per_window": ms_r / n,
             "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
-                         "frac": ach_r / peak, "kernel": "kda_kernel<decode>"},
+                         "frac": ach_r / peak, "kernel": "kda_kernel<decode>",
+                         "traffic": recorded_traffic("kda_kernel_kda_serving", w.B, 256),
+                         "algorithmic_bytes_per_launch": wb / L},
             "full_state": {"value": tok / (ms_f * 1e-3), "unit": "tokens/s",
                            "achieved_gbs": ach_f, "frac": ach_f / peak,
                            "kernel": "kda_kernel<full>"},
@@ -709,7 +724,9 @@ def bench_verify(args, dev, peak, rs, bm, wl, torch):
             "drafts_evaluated_per_s": w.B * w.n_draft * rounds / (ms_r * 1e-3),
             "committed_tokens_per_s": committed / (ms_r * 1e-3),
             "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
-                         "frac": ach_r / peak, "kernel": "m2_verify_kernel"},
+                         "frac": ach_r / peak, "kernel": "m2_verify_kernel",
+                         "traffic": recorded_traffic("m2_verify_kernel_m2_verify", w.B, 512),
+                         "algorithmic_bytes_per_launch": total / n},
             "snapshot_restore": {"rounds_per_s": rounds / (ms_s * 1e-3), "ms_per_round": ms_s / rounds,
                                  "achieved_gbs": ach_s, "frac": ach_s / peak,
                                  "kernels": "cudaMemcpyAsync x2 + m2_full_kernel x8"},
@@ -794,7 +811,9 @@ def bench_verify_gdn(args, dev, peak, rs, bm, wl, torch):
             "ms_per_round": ms_r / n,
             "drafts_evaluated_per_s": w.B * w.n_draft * n / (ms_r * 1e-3),
             "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
-                         "frac": ach_r / peak, "kernel": "gdn_verify_kernel"},
+                         "frac": ach_r / peak, "kernel": "gdn_verify_kernel",
+                         "traffic": recorded_traffic("gdn_verify_kernel_gdn_verify", w.B, 256),
+                         "algorithmic_bytes_per_launch": total / n},
             "snapshot_restore": {"rounds_per_s": n / (ms_s * 1e-3), "ms_per_round": ms_s / n,
                                  "achieved_gbs": ach_s, "frac": ach_s / peak,
                                  "kernels": "cudaMemcpyAsync x2 + gdn_kernel<full> x8"},

@@ -205,6 +205,29 @@ rssm_status replayssm_init(const rssm_desc *desc, rssm_state *state, const float
 rssm_status replayssm_decode_step(const rssm_desc *desc, rssm_state *state,
                                   const rssm_step_in *in, float *y, void *stream);
 
+/* A decode step whose record was written into the state by its producer:
+ * the kernel that computes a step's layer inputs (a projection's epilogue,
+ * say) stores them straight into slot len[b][h] of the record buffers instead
+ * of a separate step-input tensor, and this call then runs the step exactly
+ * like replayssm_decode_step with those inputs, minus their read and append
+ * [news.hamidun.com §Where the state problem appears: serving keeps per-
+ * sequence state; the record written once, where the replay reads it].
+ * Slots (elements; the producer reads len on the device; a sequence's heads
+ * share one length):
+ *   Mamba-2: x of head h at buf[0] + ((b*H + h)*cap + len)*P, dt (fp32) at
+ *            buf[1] + (b*H + h)*cap + len, Bm and Cm of group g at
+ *            buf[2|3] + ((b*G + g)*cap + len)*N;
+ *   GDN/KDA: q, k at buf[0|1] + ((b*H + h)*cap + len)*DK, v at
+ *            buf[2] + ((b*H + h)*cap + len)*DV, alpha at buf[3] +
+ *            (b*H + h)*cap + len (KDA: times DK, DK decays), beta at
+ *            buf[4] + (b*H + h)*cap + len.
+ * A, D: Mamba-2 per-head parameters (ignored for GDN/KDA).  y dense
+ * [B][H][P] / [B][H][DV].  Lengths out of range go to the status word, as
+ * for replayssm_decode_step. */
+rssm_status replayssm_decode_step_inplace(const rssm_desc *desc, rssm_state *state,
+                                          const float *A, const float *D, float *y,
+                                          void *stream);
+
 /* Fold the buffer into h0 for every (sequence, head) with len >= window, or
  * with len > 0 when force != 0; those get len = 0.  A: Mamba-2 decay rates
  * [H] (NULL for GDN). */

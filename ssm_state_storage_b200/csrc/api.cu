@@ -289,6 +289,41 @@ rssm_status replayssm_decode_step(const rssm_desc *d, rssm_state *s, const rssm_
   return from_cuda(gdn_launch_decode(p, to_stream(stream)));
 }
 
+rssm_status replayssm_decode_step_inplace(const rssm_desc *d, rssm_state *s, const float *A,
+                                          const float *D, float *y, void *stream) {
+  rssm_status st = check_desc(d);
+  if (st != RSSM_OK) return st;
+  if (d->batch == 0) return RSSM_OK;  // empty batch: no pointer is read, nothing runs
+  if ((st = check_state(d, s)) != RSSM_OK) return st;
+  if (!y) return RSSM_ERR_INVALID_ARG;
+  if (d->kind == RSSM_MAMBA2) {
+    if (!A || !D) return RSSM_ERR_INVALID_ARG;
+    M2Params p = m2_params(d, s);
+    // the step-input pointers are never read in place: point them at the buffers
+    p.x = s->buf[0];
+    p.dt = s->buf[1];
+    p.Bm = s->buf[2];
+    p.Cm = s->buf[3];
+    p.A = A;
+    p.D = D;
+    p.bs_y = (int64_t)p.H * p.P;
+    p.y = y;
+    p.inplace = 1;
+    return from_cuda(m2_launch_decode(p, to_stream(stream)));
+  }
+  GDNParams p = gdn_params(d, s);
+  p.q = s->buf[0];
+  p.k = s->buf[1];
+  p.v = s->buf[2];
+  p.alpha = static_cast<const float *>(s->buf[3]);
+  p.beta = static_cast<const float *>(s->buf[4]);
+  p.bs_y = (int64_t)p.H * p.DV;
+  p.y = y;
+  p.inplace = 1;
+  if (p.kda) return from_cuda(kda_launch(p, 0, to_stream(stream)));
+  return from_cuda(gdn_launch_decode(p, to_stream(stream)));
+}
+
 rssm_status replayssm_flush(const rssm_desc *d, rssm_state *s, const float *A, int32_t force,
                             void *stream) {
   rssm_status st = check_desc(d);

@@ -398,7 +398,18 @@ __device__ __forceinline__ bool gdn_stage(const GDNParams &p, const GdnLayout &l
   const TI *kin = static_cast<const TI *>(p.k) + b * p.bs_k + (size_t)h * DKc;
   const TI *vin = static_cast<const TI *>(p.v) + b * p.bs_v + (size_t)h * DVc;
   const int n0 = __ldcg(&p.len[bh]);
-  const float a_cur = p.alpha[b * p.bs_a + h], b_cur = p.beta[b * p.bs_b + h];
+  float a_cur, b_cur;
+  if (p.inplace) {  // the record is already in slot len: read it from there
+    const size_t slot = bh * p.cap + min(max(n0, 0), L - 1);  // stays in bounds
+    qin = static_cast<const TI *>(p.qbuf) + slot * DKc;
+    kin = static_cast<const TI *>(p.kbuf) + slot * DKc;
+    vin = static_cast<const TI *>(p.vbuf) + slot * DVc;
+    a_cur = __ldcg(&p.abuf[slot]);
+    b_cur = __ldcg(&p.bbuf[slot]);
+  } else {
+    a_cur = p.alpha[b * p.bs_a + h];
+    b_cur = p.beta[b * p.bs_b + h];
+  }
   const float a_rec = lane < L ? __ldcg(&p.abuf[bh * p.cap + lane]) : 0.f;
   TI qv[4], kv[4], vv[4];
 #pragma unroll
@@ -605,8 +616,9 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
     const bool flush = (k == L);
     const float beta = tail[0];
 
-    // ---- P1: appends, decay ratios, k_j.k and k_i.q, fp32 keys for the fold
-    if (!flush) {
+    // ---- P1: appends (an in-place step's record is in its slot already),
+    // decay ratios, k_j.k and k_i.q, fp32 keys for the fold
+    if (!flush && !p.inplace) {
       TI *qb = static_cast<TI *>(p.qbuf) + (bh * p.cap + k - 1) * DKc;
       TI *kb = static_cast<TI *>(p.kbuf) + (bh * p.cap + k - 1) * DKc;
       TI *vb = static_cast<TI *>(p.vbuf) + (bh * p.cap + k - 1) * DVc;

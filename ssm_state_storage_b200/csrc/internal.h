@@ -41,6 +41,8 @@ struct M2Params {
   // work item whose records the stager withholds, -1 for none
   uint64_t wait_ns;
   int hold_item;
+  // the step's record was written to slot len of the buffers by its producer
+  int inplace;
 };
 
 struct GDNParams {
@@ -67,6 +69,7 @@ struct GDNParams {
   // speculative rounds
   const int32_t *acc;
   int draft_max, n_draft;
+  int inplace;  // as in M2Params
 };
 
 enum FoldMode { kFoldFlush = 0, kFoldCommit = 1, kFoldMaterialize = 2 };

@@ -111,6 +111,15 @@ __global__ void __launch_bounds__(kThreads, 2) kda_kernel(const GDNParams p) {
     const TI *kin = static_cast<const TI *>(p.k) + b * p.bs_k + (size_t)h * KDc;
     const TI *vin = static_cast<const TI *>(p.v) + b * p.bs_v + (size_t)h * KVc;
     const float *ain = p.alpha + b * p.bs_a + (size_t)h * KDc;
+    const float *bin = p.beta + b * p.bs_b + h;
+    if (MODE == kKdaDecode && p.inplace) {  // the record is already in slot len
+      const size_t slot = bh * p.cap + last;
+      qin = static_cast<const TI *>(p.qbuf) + slot * KDc;
+      kin = static_cast<const TI *>(p.kbuf) + slot * KDc;
+      vin = static_cast<const TI *>(p.vbuf) + slot * KVc;
+      ain = p.abuf + slot * KDc;
+      bin = p.bbuf + slot;
+    }
     if (tid < KDc) {
       S.K[last][tid] = to_f32(kin[tid]);
       S.A[last][tid] = ain[tid];
@@ -118,7 +127,7 @@ __global__ void __launch_bounds__(kThreads, 2) kda_kernel(const GDNParams p) {
     } else {
       S.v[tid - KDc] = to_f32(vin[tid - KDc]);
     }
-    if (tid == 0) S.beta = p.beta[b * p.bs_b + h];
+    if (tid == 0) S.beta = *bin;
   }
   __syncthreads();
 
@@ -189,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 2) kda_kernel(const GDNParams p) {
       p.y[b * p.bs_y + (size_t)h * KVc + c] = p.scale * o;
       if (MODE == kKdaDecode && !fold) p.ubuf[(bh * p.cap + last) * KVc + c] = u;
     }
-    if (MODE == kKdaDecode && !fold) {
+    if (MODE == kKdaDecode && !fold && !p.inplace) {
       // append this step's record (input values, unrounded)
       const size_t slot = bh * p.cap + last;
       if (tid < KDc) {

@@ -194,22 +194,33 @@ __device__ __forceinline__ bool stage_item(const M2Params &p, const DecodeLayout
   const TI *__restrict__ Cin = static_cast<const TI *>(p.Cm) + b * p.bs_C + (size_t)g * N;
   const TI *__restrict__ xin = static_cast<const TI *>(p.x) + b * p.bs_x + (size_t)h_first * P;
 
-  // ---- phase 1: every load of the item, independent of one another
+  // ---- phase 1: every load of the item, independent of one another (with
+  // the record already in its buffer slot, the x/B/C loads wait for the length)
   const int my_len = lane < hc ? __ldcg(&p.len[bh0 + lane]) : 0;
   const float my_A = lane < hc ? p.A[h_first + lane] : 0.f;
   const float my_D = lane < hc ? p.D[h_first + lane] : 0.f;
-  const float my_dt = lane < hc ? ld_in<TI>(p.dt, b * p.bs_dt + h_first + lane) : 0.f;
+  const float my_dt = (lane < hc && !p.inplace) ? ld_in<TI>(p.dt, b * p.bs_dt + h_first + lane) : 0.f;
+  const TI *xsrc = xin, *bsrc = Bin, *csrc = Cin;
+  int xstride = P;  // elements between consecutive heads' x
+  if (p.inplace) {
+    const int slot = min(max(__shfl_sync(0xffffffffu, my_len, 0), 0), L - 1);  // stays in bounds
+    const size_t bg = (size_t)b * p.G + g;
+    xsrc = static_cast<const TI *>(p.xbuf) + (bh0 * p.cap + slot) * P;
+    xstride = p.cap * P;
+    bsrc = static_cast<const TI *>(p.Bbuf) + (bg * p.cap + slot) * N;
+    csrc = static_cast<const TI *>(p.Cbuf) + (bg * p.cap + slot) * N;
+  }
   TI bv[NPL], cv[NPL], xv[XPL];
   float dtv[DPL];
 #pragma unroll
   for (int u = 0; u < NPL; ++u) {
-    bv[u] = Bin[lane + 32 * u];
-    cv[u] = Cin[lane + 32 * u];
+    bv[u] = bsrc[lane + 32 * u];
+    cv[u] = csrc[lane + 32 * u];
   }
 #pragma unroll
   for (int u = 0; u < XPL; ++u) {
     const int e = lane + 32 * u;
-    xv[u] = e < hc * P ? xin[e] : TI{};
+    xv[u] = e < hc * P ? xsrc[(e / P) * xstride + e % P] : TI{};
   }
 #pragma unroll
   for (int u = 0; u < DPL; ++u) {
@@ -240,7 +251,7 @@ __device__ __forceinline__ bool stage_item(const M2Params &p, const DecodeLayout
   for (int u = 0; u < DPL; ++u) {
     const int e = lane + 32 * u, j = e / L, i = e - j * L;
     const float cur = __shfl_sync(0xffffffffu, my_dt, j < 32 ? j : 0);
-    if (e < hc * L) st.dt[e] = i == k - 1 ? cur : dtv[u];
+    if (e < hc * L) st.dt[e] = (i == k - 1 && !p.inplace) ? cur : dtv[u];
   }
   if (lane < hc) {
     st.A[lane] = my_A;
@@ -541,8 +552,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) m2_decode_kernel(const M2Pa
     const bool flush = (k == L);
 
     // ---- append this step's record to the global buffer (a flush empties
-    // the buffer, so its record is not kept); one CTA per group writes B, C
-    if (!flush) {
+    // the buffer, so its record is not kept; an in-place step's record is
+    // already there); one CTA per group writes B, C
+    if (!flush && !p.inplace) {
       const size_t bg = (size_t)b * p.G + g;
       if (chunk == 0) {
         for (int n = tid; n < N; n += kThreads) {

@@ -75,6 +75,8 @@ ENTRY_POINTS = {
                                         C.c_void_p, C.c_void_p]),
     "replayssm_flush": (C.c_int, [C.POINTER(Desc), C.POINTER(State), C.c_void_p, C.c_int32,
                                   C.c_void_p]),
+    "replayssm_decode_step_inplace": (C.c_int, [C.POINTER(Desc), C.POINTER(State), C.c_void_p,
+                                                C.c_void_p, C.c_void_p, C.c_void_p]),
     "replayssm_verify_commit": (C.c_int, [C.POINTER(Desc), C.POINTER(State), C.c_void_p,
                                           C.POINTER(StepIn), C.c_int32, C.c_void_p, C.c_void_p]),
     "replayssm_commit": (C.c_int, [C.POINTER(Desc), C.POINTER(State), C.c_void_p, C.c_void_p,
@@ -284,6 +286,19 @@ def replayssm_decode_step(layer: Layer, state: ReplayState, inp: dict, y: torch.
     si = _step_in(layer, inp, y)
     _ok(lib().replayssm_decode_step(C.byref(d), C.byref(cs), C.byref(si), y.data_ptr(),
                                     _stream(stream)), "replayssm_decode_step")
+
+
+def replayssm_decode_step_inplace(layer: Layer, state: ReplayState, y: torch.Tensor,
+                                  A: torch.Tensor | None = None, D: torch.Tensor | None = None,
+                                  stream=None):
+    """A decode step whose record the caller already wrote into slot len of
+    the record buffers (state.buf[i][..., len, ...])."""
+    d, cs = layer.desc(), state.cstate()
+    a = _dense(A, torch.float32, "A") if A is not None else None
+    dd = _dense(D, torch.float32, "D") if D is not None else None
+    _ok(lib().replayssm_decode_step_inplace(C.byref(d), C.byref(cs), a, dd,
+                                            _dense(y, torch.float32, "y"), _stream(stream)),
+        "replayssm_decode_step_inplace")
 
 
 def replayssm_flush(layer: Layer, state: ReplayState, A: torch.Tensor | None = None,

@@ -911,9 +911,27 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_verify_kernel(const GDNParams
   // ---- stage committed records and the drafts (fp32)
   const TI *kb = static_cast<const TI *>(p.kbuf) + bh * p.cap * DKc;
   const float *ub = p.ubuf + bh * p.cap * DVc;
-  for (int e = tid; e < n1 * DKc; e += kThreads) {
-    S.Kc[e / DKc][e % DKc] = to_f32(kb[e]);
-    S.U[e / DVc][e % DVc] = ub[e];
+  {
+    // every load first (one memory latency for all committed records), then the
+    // shared-memory stores
+    constexpr int PER = kMaxRec * DKc / kThreads;
+    float kv[PER], uv[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int e = tid + u * kThreads;
+      if (e < n1 * DKc) {
+        kv[u] = to_f32(kb[e]);
+        uv[u] = ub[e];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int e = tid + u * kThreads;
+      if (e < n1 * DKc) {
+        S.Kc[e / DKc][e % DKc] = kv[u];
+        S.U[e / DVc][e % DVc] = uv[u];
+      }
+    }
   }
   for (int e = tid; e < nd * DKc; e += kThreads) {
     const int d = e / DKc, c = e % DKc;

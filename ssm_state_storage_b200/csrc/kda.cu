@@ -99,13 +99,22 @@ __global__ void __launch_bounds__(kThreads, 2) kda_kernel(const GDNParams p) {
   const TI *kb = static_cast<const TI *>(p.kbuf) + bh * p.cap * KDc;
   const float *ab = p.abuf + bh * p.cap * KDc;
   const float *ub = p.ubuf + bh * p.cap * KVc;
-  if (MODE != kKdaFull)
-    for (int e = tid; e < nbuf * KDc; e += kThreads) {
-      const int i = e / KDc, c = e - i * KDc;
-      S.K[i][c] = to_f32(kb[e]);
-      S.A[i][c] = ab[e];
-      S.U[i][c] = ub[e];
+  // every load first (one memory latency for the buffered records and this
+  // step's), then the shared-memory stores
+  constexpr int PER = kKRec * KDc / kThreads;
+  float kv[PER], av[PER], uv[PER];
+  if (MODE != kKdaFull) {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int e = tid + u * kThreads;
+      if (e < nbuf * KDc) {
+        kv[u] = to_f32(kb[e]);
+        av[u] = ab[e];
+        uv[u] = ub[e];
+      }
     }
+  }
+  float cur0 = 0.f, cur1 = 0.f, cur2 = 0.f, beta = 0.f;
   if (kOut) {
     const TI *qin = static_cast<const TI *>(p.q) + b * p.bs_q + (size_t)h * KDc;
     const TI *kin = static_cast<const TI *>(p.k) + b * p.bs_k + (size_t)h * KDc;
@@ -121,13 +130,35 @@ __global__ void __launch_bounds__(kThreads, 2) kda_kernel(const GDNParams p) {
       bin = p.bbuf + slot;
     }
     if (tid < KDc) {
-      S.K[last][tid] = to_f32(kin[tid]);
-      S.A[last][tid] = ain[tid];
-      S.q[tid] = to_f32(qin[tid]);
+      cur0 = to_f32(kin[tid]);
+      cur1 = ain[tid];
+      cur2 = to_f32(qin[tid]);
     } else {
-      S.v[tid - KDc] = to_f32(vin[tid - KDc]);
+      cur0 = to_f32(vin[tid - KDc]);
     }
-    if (tid == 0) S.beta = *bin;
+    if (tid == 0) beta = *bin;
+  }
+  if (MODE != kKdaFull) {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int e = tid + u * kThreads;
+      if (e < nbuf * KDc) {
+        const int i = e / KDc, c = e - i * KDc;
+        S.K[i][c] = kv[u];
+        S.A[i][c] = av[u];
+        S.U[i][c] = uv[u];
+      }
+    }
+  }
+  if (kOut) {
+    if (tid < KDc) {
+      S.K[last][tid] = cur0;
+      S.A[last][tid] = cur1;
+      S.q[tid] = cur2;
+    } else {
+      S.v[tid - KDc] = cur0;
+    }
+    if (tid == 0) S.beta = beta;
   }
   __syncthreads();
 

@@ -523,7 +523,7 @@ def bench_gdn(args, dev, peak, rs, bm, wl, torch):
                          "achieved_input_records_only": ach_rec},
             "full_state": {"value": tok / (ms_f * 1e-3), "unit": "tokens/s",
                            "achieved_gbs": ach_f, "frac": ach_f / peak,
-                           "kernel": "gdn_kernel<full>"},
+                           "kernel": "kda_kernel<full> (scalar decay)"},
             "replay_over_full": ms_f / ms_r,
             "step_times": steps_us,
             "bytes_per_head_token": {"replay": wb / (w.B * w.H * L),
@@ -816,7 +816,7 @@ def bench_verify_gdn(args, dev, peak, rs, bm, wl, torch):
                          "algorithmic_bytes_per_launch": total / n},
             "snapshot_restore": {"rounds_per_s": n / (ms_s * 1e-3), "ms_per_round": ms_s / n,
                                  "achieved_gbs": ach_s, "frac": ach_s / peak,
-                                 "kernels": "cudaMemcpyAsync x2 + gdn_kernel<full> x8"},
+                                 "kernels": "cudaMemcpyAsync x2 + kda_kernel<full> x8"},
             "replay_over_snapshot": ms_s / ms_r,
             "gpu_launches": n}
 

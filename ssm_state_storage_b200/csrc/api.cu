@@ -424,8 +424,9 @@ rssm_status replayssm_full_decode_step(const rssm_desc *d, float *S, const rssm_
   p.y = y;
   p.limit = limit;
   p.step_index = step_index;
-  if (p.kda) return from_cuda(kda_launch(p, 3, to_stream(stream)));
-  return from_cuda(gdn_launch_full(p, to_stream(stream)));
+  // the delta-rule conventional step (per-channel decays for KDA, one decay
+  // broadcast over the channels for GDN)
+  return from_cuda(kda_launch(p, 3, to_stream(stream)));
 }
 
 rssm_status replayssm_materialize(const rssm_desc *d, const rssm_state *s, const float *A,

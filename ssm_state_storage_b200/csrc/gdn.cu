@@ -1,6 +1,7 @@
-// gdn.cu -- Gated DeltaNet decode kernels for sm_100a: replay decode step with
-// fused flush fold, standalone fold (flush / materialise), and the conventional
-// full-state step.
+// gdn.cu -- Gated DeltaNet kernels for sm_100a: replay decode step with fused
+// flush fold, standalone fold (flush / materialise / commit), and the
+// speculative verify round.  (The conventional full-state step is the
+// one-decay case of the delta-rule step in kda.cu.)
 //
 // Method: checkpoint h0 plus a buffer of the latest (q, k, v, alpha, beta)
 // records per (sequence, head); outputs are evaluated from h0 and the buffer
@@ -1144,11 +1145,6 @@ cudaError_t gdn_launch_fold(const GDNParams &p, int mode, cudaStream_t s) {
   if (mode == kFoldMaterialize) return launch_dt<kGdnMaterialize>(p, s);
   if (mode == kFoldCommit) return launch_dt<kGdnCommit>(p, s);
   return cudaErrorInvalidValue;
-}
-
-cudaError_t gdn_launch_full(const GDNParams &p, cudaStream_t s) {
-  if (p.B * p.H == 0) return cudaSuccess;
-  return launch_dt<kGdnFull>(p, s);
 }
 
 cudaError_t gdn_launch_verify(const GDNParams &p, cudaStream_t s) {

@@ -83,11 +83,11 @@ bool m2_heads_supported(int hpg);  // heads per group: <= 8 or a multiple of 8
 
 cudaError_t gdn_launch_decode(const GDNParams &p, cudaStream_t s);
 cudaError_t gdn_launch_fold(const GDNParams &p, int mode, cudaStream_t s);
-cudaError_t gdn_launch_full(const GDNParams &p, cudaStream_t s);
 cudaError_t gdn_launch_verify(const GDNParams &p, cudaStream_t s);
 
 // Kimi Delta Attention (GDNParams with alpha and its records per key channel):
-// mode 0 decode step, 1 flush, 2 materialise, 3 conventional step.
+// mode 0 decode step, 1 flush, 2 materialise, 3 conventional step; mode 3 with
+// kda == 0 is the conventional Gated DeltaNet step (scalar alpha [B][H]).
 cudaError_t kda_launch(const GDNParams &p, int mode, cudaStream_t s);
 bool gdn_supported(int DK, int DV);
 

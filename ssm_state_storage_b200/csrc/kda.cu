@@ -22,7 +22,8 @@
 // it is computed once, when the record is appended, and cached in the buffer
 // (buf[5]); a step then needs two products with h0 (Gamma o k, Gamma o q)
 // and O(t) decay-weighted key dots.  The conventional step is the same
-// algebra with one record and the state written back.
+// algebra with one record and the state written back; it also serves as the
+// conventional step of Gated DeltaNet (a scalar decay is the all-equal case).
 //
 // One CTA of 256 threads per (sequence, head); lane l of warp w holds rows
 // 16w..16w+15 and columns 4l..4l+3 of the 128 x 128 tile in registers.  The
@@ -131,7 +132,9 @@ __global__ void __launch_bounds__(kThreads, 2) kda_kernel(const GDNParams p) {
     }
     if (tid < KDc) {
       cur0 = to_f32(kin[tid]);
-      cur1 = ain[tid];
+      // Gated DeltaNet's conventional step runs here too: one decay for every
+      // channel, alpha [B][H] (Diag(alpha) = alpha I commutes with the rule)
+      cur1 = p.kda ? ain[tid] : p.alpha[b * p.bs_a + h];
       cur2 = to_f32(qin[tid]);
     } else {
       cur0 = to_f32(vin[tid - KDc]);

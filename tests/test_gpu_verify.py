@@ -66,6 +66,7 @@ def test_verify_rounds_match_oracle():
     (64, 64, torch.float32, 12, 2),     # 6 heads per group
     (128, 64, torch.bfloat16, 8, 8),    # one head per group
     (64, 128, torch.bfloat16, 6, 2),    # 3 heads per group
+    (128, 128, torch.bfloat16, 8, 2),   # 128 x 128 tiles, tensor-core commit fold
 ])
 def test_verify_shapes_match_oracle(P, N, dtype, H, G):
     w, A, D, S0, rd = _draw(20, B=3, H=H, G=G, P=P, N=N, in_dtype=dtype)

@@ -616,6 +616,9 @@ def bench_readcopy(args, dev, peak, rs, bm, wl, torch, ms_fp32):
         for i in range(3):
             window(i)
         ms = _events_ms(window, n, stream, torch, dev)
+        steps_us = per_launch_us(lambda i: rs.replayssm_decode_step(layer, state,
+                                                                    step_in[i % pool], y, stream),
+                                 L, 10, stream, torch, dev)
         if state.status() != 0:
             raise RuntimeError(f"device status {state.status()} after the {fmt} read-copy run")
         wb = bm.m2_replay_window_bytes_rc(L, w.P, w.N, w.H // w.G, 2, fmt) * w.B * w.H
@@ -624,7 +627,8 @@ def bench_readcopy(args, dev, peak, rs, bm, wl, torch, ms_fp32):
                     "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                                  "frac": ach / peak, "kernel": "m2_decode_kernel (read copy)"},
                     "bytes_per_head_token": wb / (w.B * w.H * L),
-                    "over_fp32_replay": ms_fp32 / (ms / n), "gpu_launches": n * L}
+                    "over_fp32_replay": ms_fp32 / (ms / n), "step_times": steps_us,
+                    "gpu_launches": n * L}
         del state
         torch.cuda.empty_cache()
     return out

@@ -363,9 +363,12 @@ __device__ __forceinline__ void build_fold_b(unsigned char *dst, const TI *xj, c
 // Epilogue of head bh's fold by the WPH warps of one head group (`sub` = warp
 // in group): the new checkpoint, and for a read copy its new codes.  The old
 // tile comes from the ring slot (QM 0) or, with a read copy in the slot, from
-// the fp32 checkpoint in global memory.  NVFP4 (QM 2) takes a second pass
-// over the values this thread stored, after the group agrees on the tile
-// maximum (named barrier 2 + hq, `red` = the group's 8 maxima).
+// the fp32 checkpoint in global memory.  FP8 codes are written with the new
+// values; NVFP4 first agrees on the tile maximum over the group (`red` = the
+// group's 8 maxima), then forms the codes from the rows the group just stored
+// (re-read after named barrier 2 + hq, while they are in L2) in the row
+// layout of the output dots, four values per lane, so a 16-column block spans
+// four lanes.
 template <int P, int N, int QM, int WPH>
 __device__ __forceinline__ void fold_epilogue(const M2Params &p, size_t bh, const float *tile,
                                               float lam, uint32_t tcol, int sub, int lane,
@@ -401,33 +404,21 @@ __device__ __forceinline__ void fold_epilogue(const M2Params &p, size_t bh, cons
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if (lane == 0) red[sub] = amax;
-    bar_sync(2 + hq, WPH * 32);
+    bar_sync(2 + hq, WPH * 32);  // also orders the group's h0 stores before the re-reads
     float tmax = red[0];
     for (int w2 = 1; w2 < WPH; ++w2) tmax = fmaxf(tmax, red[w2]);
     const float sg = nvfp4_tile_scale(tmax);
-    uint8_t *rc = p.rc + bh * (size_t)(P * N / 2);
-    uint8_t *sc = p.rc_scale + bh * (size_t)(P * N / 16);
-#pragma unroll 1
-    for (int c = 0; c < CW; c += 32) {
-      float hv[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) hv[i] = hg[(r0 + c + i) * N + n];  // this thread's own stores
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = r0 + c + i;
-        const float hn = hv[i];
-        float bm = fabsf(hn);
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
-        const uint32_t scode = nvfp4_block_code(bm, sg);
-        const float dstep = nvfp4_step(scode, sg);
-        const float qv = dstep > 0.f ? __fdiv_rn(hn, dstep) : 0.f;
-        const float qn = __shfl_xor_sync(0xffffffffu, qv, 1);
-        if ((lane & 1) == 0) rc[r * (N / 2) + n / 2] = (uint8_t)e2m1x2_encode(qv, qn);
-        if ((lane & 15) == 0) sc[r * (N / 16) + n / 16] = (uint8_t)scode;
-      }
+    // codes from the rows just stored (L2-resident), in the row layout of the
+    // output dots: lane (rs, c8) takes four consecutive columns of a row, so
+    // a 16-column block spans four lanes
+    constexpr int RW = P / WPH, RG = RW / 4;
+    const int rs = lane >> 3, c8 = lane & 7;
+    for (int g4 = 0; g4 < RG; ++g4) {
+      const int r = sub * RW + 4 * g4 + rs;
+      float4 v[N / 32];
+      load_row<N>(hg, r, c8, v);
+      nvfp4_row<P, N>(v, sg, false, p.rc + bh * (size_t)(P * N / 2),
+                      p.rc_scale + bh * (size_t)(P * N / 16), r, c8);
     }
     if (sub == 0 && lane == 0) p.rc_gscale[bh] = sg;
     bar_sync(2 + hq, WPH * 32);  // red[] is reused by the group's next head

@@ -40,21 +40,17 @@ constexpr int DKc = 128, DVc = 128;
 constexpr int kMaxRec = kMaxCap;     // a window plus the tail of a speculative round
 constexpr int kRows = DKc / 8;       // rows per warp
 
-enum GdnMode { kGdnDecode = 0, kGdnFlush = 1, kGdnMaterialize = 2, kGdnFull = 3, kGdnCommit = 4 };
+enum GdnMode { kGdnFlush = 1, kGdnMaterialize = 2, kGdnCommit = 4 };
 
-// Shared memory of gdn_kernel for at most MR records (the conventional step
-// has exactly one).
-template <int MR>
+// Shared memory of the fold-only kernel: up to kMaxRec records.
 struct GdnSmem {
-  static constexpr int kZ = MR + 1;  // records + q
-  float k[kZ][DKc];       // k_0..k_{n-1}, then q
-  float u[MR][DVc];       // v_i, overwritten by u_i
-  float part[8][kZ][DVc];
-  float z[kZ][DVc];
-  float alpha[MR], beta[MR], gamma[MR];
-  float ratio[MR][MR];
-  float gram[MR][MR];
-  float kq[MR];
+  float k[kMaxRec][DKc];  // keys
+  float u[kMaxRec][DVc];  // v_i, overwritten by u_i
+  float part[8][kMaxRec][DVc];
+  float z[kMaxRec][DVc];
+  float alpha[kMaxRec], beta[kMaxRec], gamma[kMaxRec];
+  float ratio[kMaxRec][kMaxRec];
+  float gram[kMaxRec][kMaxRec];
   int n, act;
 };
 
@@ -64,143 +60,90 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Fold-only kernel, one CTA of 256 threads per (sequence, head): the buffered
+// records' corrections u_i by forward substitution from h0, then the fold
+// h0 <- gamma h0 + sum_i R(n-1,i) k_i u_i^T.  MODE kGdnFlush: where len >= L
+// (or len > 0 with force); kGdnCommit: len += accepted, fold where it reaches
+// L; kGdnMaterialize: S_out = the fold, state untouched.
 template <typename TI, int MODE>
 __global__ void __launch_bounds__(kThreads, 2) gdn_kernel(const GDNParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  using Smem = GdnSmem<MODE == kGdnFull ? 1 : kMaxRec>;
-  Smem &S = *reinterpret_cast<Smem *>(smem_raw);
+  GdnSmem &S = *reinterpret_cast<GdnSmem *>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh_i = blockIdx.x;
-  const int b = bh_i / p.H, h = bh_i - b * p.H;
+  const int b = bh_i / p.H;
   const size_t bh = (size_t)bh_i;
 
-  // ---- record count n (records 0..n-1), whether to fold, whether to output
+  // ---- record count n (records 0..n-1), whether to fold
   if (tid == 0) {
-    int n = 1, act = 1, ok = 1;
-    if (MODE == kGdnFull) {
-      ok = 1;
-      act = !(p.limit && p.step_index >= p.limit[b]);
+    int n, act, ok;
+    const int n0 = p.len[bh];
+    if (MODE == kGdnCommit) {  // len += accepted; fold when it reaches the window
+      const int a = p.acc[b];
+      ok = n0 >= 0 && n0 < p.L && a >= 0 && a <= p.draft_max && n0 + a <= p.cap;
+      n = n0 + a;
+      act = n >= p.L;
+      if (ok && !act) p.len[bh] = n;
     } else {
-      const int n0 = p.len[bh];
-      if (MODE == kGdnDecode) {
-        ok = n0 >= 0 && n0 < p.L;
-        n = n0 + 1;
-        act = 1;
-      } else if (MODE == kGdnCommit) {  // len += accepted; fold when it reaches the window
-        const int a = p.acc[b];
-        ok = n0 >= 0 && n0 < p.L && a >= 0 && a <= p.draft_max && n0 + a <= p.cap;
-        n = n0 + a;
-        act = n >= p.L;
-        if (ok && !act) p.len[bh] = n;
-      } else {
-        ok = n0 >= 0 && n0 <= p.cap;
-        n = n0;
-        act = MODE == kGdnMaterialize ? 1 : (n0 >= p.L || (p.force && n0 > 0));
-      }
-      if (!ok) report(p.status, RSSM_ERR_STATE);
+      ok = n0 >= 0 && n0 <= p.cap;
+      n = n0;
+      act = MODE == kGdnMaterialize ? 1 : (n0 >= p.L || (p.force && n0 > 0));
     }
+    if (!ok) report(p.status, RSSM_ERR_STATE);
     S.n = ok ? n : -1;
     S.act = act;
   }
   __syncthreads();
   const int n = S.n;
   if (n < 0 || !S.act) return;
-  constexpr bool kOut = (MODE == kGdnDecode || MODE == kGdnFull);
-  const bool fold = (MODE == kGdnDecode) ? (n == p.L) : true;
-  const int nz = kOut ? n + 1 : n;  // rows of Z: records (+ q)
 
   // ---- checkpoint tile into registers (rows 16w+rho, cols 4l..4l+3)
-  float *state = (MODE == kGdnFull) ? p.S + bh * (DKc * DVc) : p.h0 + bh * (DKc * DVc);
+  float *state = p.h0 + bh * (DKc * DVc);
   float4 hv[kRows];
 #pragma unroll
   for (int rho = 0; rho < kRows; ++rho)
     hv[rho] = ld_stream(state + (size_t)(kRows * warp + rho) * DVc + 4 * lane);
 
-  // ---- stage records (fp32) and append this step's
-  const TI *qin = static_cast<const TI *>(p.q) + b * p.bs_q + (size_t)h * DKc;
-  const TI *kin = static_cast<const TI *>(p.k) + b * p.bs_k + (size_t)h * DKc;
-  const TI *vin = static_cast<const TI *>(p.v) + b * p.bs_v + (size_t)h * DVc;
-  TI *qb = static_cast<TI *>(p.qbuf) + bh * p.cap * DKc;
-  TI *kb = static_cast<TI *>(p.kbuf) + bh * p.cap * DKc;
-  TI *vb = static_cast<TI *>(p.vbuf) + bh * p.cap * DVc;
-  const bool append = (MODE == kGdnDecode) && !fold;
+  // ---- stage the records (fp32)
+  const TI *kb = static_cast<const TI *>(p.kbuf) + bh * p.cap * DKc;
+  const TI *vb = static_cast<const TI *>(p.vbuf) + bh * p.cap * DVc;
   for (int idx = tid; idx < n * DKc; idx += kThreads) {
     const int i = idx / DKc, c = idx - i * DKc;
-    const bool cur = kOut && i == n - 1;
-    if (cur) {
-      const TI kv = kin[c], vv = vin[c];
-      S.k[i][c] = to_f32(kv);
-      S.u[i][c] = to_f32(vv);
-      if (append) {
-        kb[(size_t)i * DKc + c] = kv;
-        vb[(size_t)i * DVc + c] = vv;
-        qb[(size_t)i * DKc + c] = qin[c];
-      }
-    } else {
-      S.k[i][c] = to_f32(kb[(size_t)i * DKc + c]);
-      S.u[i][c] = to_f32(vb[(size_t)i * DVc + c]);
-    }
+    S.k[i][c] = to_f32(kb[(size_t)i * DKc + c]);
+    S.u[i][c] = to_f32(vb[(size_t)i * DVc + c]);
   }
-  if (kOut)
-    for (int c = tid; c < DKc; c += kThreads) S.k[n][c] = to_f32(qin[c]);
   if (tid < n) {
-    float a, be;
-    if (kOut && tid == n - 1) {
-      a = p.alpha[b * p.bs_a + h];
-      be = p.beta[b * p.bs_b + h];
-      if (append) {
-        p.abuf[bh * p.cap + tid] = a;
-        p.bbuf[bh * p.cap + tid] = be;
-      }
-    } else {
-      a = p.abuf[bh * p.cap + tid];
-      be = p.bbuf[bh * p.cap + tid];
-    }
-    S.alpha[tid] = a;
-    S.beta[tid] = be;
+    S.alpha[tid] = p.abuf[bh * p.cap + tid];
+    S.beta[tid] = p.bbuf[bh * p.cap + tid];
   }
   __syncthreads();
 
-  // ---- partial Z over this warp's 16 rows; key Gram matrix, k.q, decays
-  for (int i = 0; i < nz; ++i) {
+  // ---- partial Z = [k_0..k_{n-1}]^T h0 over this warp's 16 rows; key Gram
+  // matrix and decay ratios
+  for (int i = 0; i < n; ++i) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int t = 0; t < kRows / 4; ++t) {
       const float4 kr = *reinterpret_cast<const float4 *>(&S.k[i][kRows * warp + 4 * t]);
       const float kk[4] = {kr.x, kr.y, kr.z, kr.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float4 hr = hv[4 * t + e];
-        acc.x = fmaf(kk[e], hr.x, acc.x);
-        acc.y = fmaf(kk[e], hr.y, acc.y);
-        acc.z = fmaf(kk[e], hr.z, acc.z);
-        acc.w = fmaf(kk[e], hr.w, acc.w);
-      }
+      for (int e = 0; e < 4; ++e) acc = fma4x(kk[e], hv[4 * t + e], acc);
     }
     *reinterpret_cast<float4 *>(&S.part[warp][i][4 * lane]) = acc;
   }
-  // pairs (j, i), j < i < n: k_j.k_i ; and (i, q): k_i.q
-  const int npair = n * (n - 1) / 2 + (kOut ? n : 0);
+  // pairs (j, i), j < i < n, row-major over the strict lower triangle
+  const int npair = n * (n - 1) / 2;
   for (int pr = warp; pr < npair; pr += 8) {
-    int i, j;
-    bool isq = false;
-    if (pr < n * (n - 1) / 2) {  // row-major over the strict lower triangle
-      i = 1;
-      int rem = pr;
-      while (rem >= i) { rem -= i; ++i; }
-      j = rem;
-    } else {
-      i = pr - n * (n - 1) / 2;
-      j = n;  // q
-      isq = true;
+    int i = 1, rem = pr;
+    while (rem >= i) {
+      rem -= i;
+      ++i;
     }
+    const int j = rem;
     float acc = 0.f;
     for (int c = lane; c < DKc; c += 32) acc = fmaf(S.k[j][c], S.k[i][c], acc);
     acc = warp_sum(acc);
-    if (lane == 0) {
-      if (isq) S.kq[i] = acc;
-      else S.gram[i][j] = acc;
-    }
+    if (lane == 0) S.gram[i][j] = acc;
   }
   for (int e = tid; e < n * n; e += kThreads) {
     const int i = e / n, j = e - (e / n) * n;
@@ -218,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_kernel(const GDNParams p) {
   __syncthreads();
 
   // ---- Z = sum of the 8 warp partials (fixed order)
-  for (int idx = tid; idx < nz * DVc; idx += kThreads) {
+  for (int idx = tid; idx < n * DVc; idx += kThreads) {
     const int i = idx / DVc, c = idx - i * DVc;
     float z = 0.f;
 #pragma unroll
@@ -227,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_kernel(const GDNParams p) {
   }
   __syncthreads();
 
-  // ---- u by forward substitution, one column per thread; then the output
+  // ---- u by forward substitution, one column per thread
   if (tid < DVc) {
     const int c = tid;
     for (int i = 0; i < n; ++i) {
@@ -235,48 +178,29 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_kernel(const GDNParams p) {
       for (int j = 0; j < i; ++j) u -= S.ratio[i][j] * S.gram[i][j] * S.u[j][c];
       S.u[i][c] = S.beta[i] * u;
     }
-    if (kOut) {
-      float o = S.gamma[n - 1] * S.z[n][c];
-      for (int i = 0; i < n; ++i) o = fmaf(S.ratio[n - 1][i] * S.kq[i], S.u[i][c], o);
-      p.y[b * p.bs_y + (size_t)h * DVc + c] = p.scale * o;
-    }
   }
+  __syncthreads();
 
-  if (fold) {
-    __syncthreads();
-    // h0 <- gamma_{n-1} h0 + sum_i R(n-1,i) k_i u_i^T
-    const float gl = n > 0 ? S.gamma[n - 1] : 1.f;
+  // ---- h0 <- gamma_{n-1} h0 + sum_i R(n-1,i) k_i u_i^T
+  const float gl = n > 0 ? S.gamma[n - 1] : 1.f;
 #pragma unroll
-    for (int rho = 0; rho < kRows; ++rho) {
-      hv[rho].x *= gl;
-      hv[rho].y *= gl;
-      hv[rho].z *= gl;
-      hv[rho].w *= gl;
-    }
-    for (int i = 0; i < n; ++i) {
-      const float r = S.ratio[n - 1][i];
-      const float4 ui = *reinterpret_cast<const float4 *>(&S.u[i][4 * lane]);
+  for (int rho = 0; rho < kRows; ++rho) hv[rho] = mul4x(gl, hv[rho]);
+  for (int i = 0; i < n; ++i) {
+    const float r = S.ratio[n - 1][i];
+    const float4 ui = *reinterpret_cast<const float4 *>(&S.u[i][4 * lane]);
 #pragma unroll
-      for (int rho = 0; rho < kRows; ++rho) {
-        const float kr = r * S.k[i][kRows * warp + rho];
-        hv[rho].x = fmaf(kr, ui.x, hv[rho].x);
-        hv[rho].y = fmaf(kr, ui.y, hv[rho].y);
-        hv[rho].z = fmaf(kr, ui.z, hv[rho].z);
-        hv[rho].w = fmaf(kr, ui.w, hv[rho].w);
-      }
-    }
-    float *dst = (MODE == kGdnMaterialize) ? p.S_out + bh * (DKc * DVc) : state;
-#pragma unroll
-    for (int rho = 0; rho < kRows; ++rho)
-      st_stream(dst + (size_t)(kRows * warp + rho) * DVc + 4 * lane, hv[rho]);
+    for (int rho = 0; rho < kRows; ++rho) hv[rho] = fma4x(r * S.k[i][kRows * warp + rho], ui, hv[rho]);
   }
-  if (tid == 0 && (MODE == kGdnDecode || MODE == kGdnFlush || MODE == kGdnCommit))
-    p.len[bh] = fold ? 0 : n;
+  float *dst = (MODE == kGdnMaterialize) ? p.S_out + bh * (DKc * DVc) : state;
+#pragma unroll
+  for (int rho = 0; rho < kRows; ++rho)
+    st_stream(dst + (size_t)(kRows * warp + rho) * DVc + 4 * lane, hv[rho]);
+  if (tid == 0 && (MODE == kGdnFlush || MODE == kGdnCommit)) p.len[bh] = 0;
 }
 
 template <typename TI, int MODE>
 cudaError_t launch(const GDNParams &p, cudaStream_t s) {
-  const size_t smem = sizeof(GdnSmem<MODE == kGdnFull ? 1 : kMaxRec>);
+  const size_t smem = sizeof(GdnSmem);
   cudaError_t e = cudaFuncSetAttribute(gdn_kernel<TI, MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

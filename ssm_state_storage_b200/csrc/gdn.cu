@@ -42,6 +42,23 @@ constexpr int kRows = DKc / 8;       // rows per warp
 
 enum GdnMode { kGdnFlush = 1, kGdnMaterialize = 2, kGdnCommit = 4 };
 
+// Eight consecutive shared-memory elements (16-byte aligned for bf16, 32 for
+// fp32) as fp32.
+template <typename T>
+__device__ __forceinline__ void ld8_smem(const T *p, float (&v)[8]) {
+  if constexpr (sizeof(T) == 4) {
+    const float4 a = *reinterpret_cast<const float4 *>(p);
+    const float4 b = *reinterpret_cast<const float4 *>(p + 4);
+    v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w;
+    v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+  } else {
+    const uint4 raw = *reinterpret_cast<const uint4 *>(p);
+    const T *e = reinterpret_cast<const T *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = to_f32(e[i]);
+  }
+}
+
 // Shared memory of the fold-only kernel: up to kMaxRec records.
 struct GdnSmem {
   float k[kMaxRec][DKc];  // keys
@@ -262,8 +279,8 @@ struct GdnLayout {
       o += a128(d.NR * d.stage_floats * 4);
       d.off_db = o;
       o += a128(2 * d.db_floats * 4);
-      d.off_single = o;  // part [8][2][128] | z [2][128] | ucur [128] | opart [128]
-      o += a128((8 * 2 * 128 + 2 * 128 + 2 * 128) * 4);
+      d.off_single = o;  // part [8][2][128] | ucur [128]
+      o += a128((8 * 2 * 128 + 128) * 4);
       d.off_umma = o;
       o += mma ? 4 * 128 * 32 : 0;
       d.off_ring = o;
@@ -283,7 +300,7 @@ struct GdnPtrs {
   uint64_t *full, *empty, *rfull, *rempty, *mma;
   uint32_t *tmem_slot;
   unsigned char *recK, *ring, *umma;
-  float *recU, *stage, *db, *part, *z, *ucur, *opart;
+  float *recU, *stage, *db, *part, *ucur;
   __device__ GdnPtrs(unsigned char *smem, const GdnLayout &l) {
     full = reinterpret_cast<uint64_t *>(smem + l.off_bars);
     empty = full + 8;
@@ -297,9 +314,7 @@ struct GdnPtrs {
     stage = reinterpret_cast<float *>(smem + l.off_stage);
     db = reinterpret_cast<float *>(smem + l.off_db);
     part = reinterpret_cast<float *>(smem + l.off_single);
-    z = part + 8 * 2 * 128;
-    ucur = z + 2 * 128;
-    opart = ucur + 128;
+    ucur = part + 8 * 2 * 128;
     ring = smem + l.off_ring;
   }
 };
@@ -571,10 +586,11 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
     }
     {
       // 2k-1 dot products of 128: k_j.k_{k-1} (j < k-1) then k_i.q (i < k);
-      // 16 threads per dot, trip count uniform across each warp
+      // 8 threads per dot (one pass for up to 32 dots), thread j of a dot
+      // takes the 8-element chunks j and j + 8 with 16-byte key loads
       const int ndot = 2 * k - 1;
-      for (int base = 0; base < ndot; base += kThreads / 16) {
-        const int d = base + (tid >> 4), c0 = (tid & 15) * 8;
+      for (int base = 0; base < ndot; base += kThreads / 8) {
+        const int d = base + (tid >> 3), j = tid & 7;
         // products in fp32 (exact for bf16 inputs: 8 x 8 significant bits),
         // sums in fp64 over two independent chains
         double acc = 0.0, acc1 = 0.0;
@@ -582,17 +598,23 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
           const int i = d < k - 1 ? d : d - (k - 1);
           const float *other = d < k - 1 ? ks : qs;
 #pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            acc += (double)(to_f32(rK[i * DKc + c0 + e]) * other[c0 + e]);
-            acc1 += (double)(to_f32(rK[i * DKc + c0 + e + 1]) * other[c0 + e + 1]);
+          for (int m = 0; m < 2; ++m) {
+            const int c0 = 8 * (j + 8 * m);
+            float kv[8], ov[8];
+            ld8_smem(rK + i * DKc + c0, kv);
+            ld8_smem(other + c0, ov);
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              acc += (double)(kv[e] * ov[e]);
+              acc1 += (double)(kv[e + 1] * ov[e + 1]);
+            }
           }
           acc += acc1;
         }
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
         acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-        if (d < ndot && (tid & 15) == 0) {
+        if (d < ndot && j == 0) {
           if (d < k - 1) kk[d] = (float)acc;
           else kq[d - (k - 1)] = (float)acc;
         }
@@ -641,46 +663,39 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
       *reinterpret_cast<float4 *>(&S.part[(warp * 2 + 1) * 128 + 4 * lane]) = pq;
     }
     bar_sync(1, kThreads);
-    // ---- P3 (fused into P4): each thread sums the 8 warps' partials of its
-    // own column, z = h0^T k for threads 0-127, zq = h0^T q for 128-255, in a
-    // fixed order, so no barrier is needed between the two
-    // ---- P4: threads 0-127 form u of this record (column c), threads 128-255
-    // the output's terms over the older records; then the output's last term
-    // needs u, exchanged through shared memory.
+    // ---- P3 + P4: thread pair (2c, 2c+1) owns column c.  The even thread
+    // sums the 8 warps' partials of z = h0^T k, the odd one those of
+    // zq = h0^T q (fixed order), and they swap; each then runs over the
+    // older records of its parity, one load of u_j serving both the
+    // correction's and the output's sum, and the pair adds the two halves.
+    // Both threads hold u and o; no barrier is needed (the next item starts
+    // with one).
     {
-      const int vsel = tid >> 7, c = tid & 127;
+      const int c = tid >> 1, par = tid & 1;
       const float g = gam[0];
       float zc = 0.f;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) zc += S.part[(w * 2 + vsel) * 128 + c];
-      if (tid < 128) {
-        float a0 = vs[c] - g * zc, a1 = 0.f;
-        int j = 0;
-        for (; j + 1 < k - 1; j += 2) {
-          a0 = fmaf(-R[j] * kk[j], rU[j * DVc + c], a0);
-          a1 = fmaf(-R[j + 1] * kk[j + 1], rU[(j + 1) * DVc + c], a1);
-        }
-        if (j < k - 1) a0 = fmaf(-R[j] * kk[j], rU[j * DVc + c], a0);
-        const float u = beta * (a0 + a1);
+      for (int w = 0; w < 8; ++w) zc += S.part[(w * 2 + par) * 128 + c];
+      const float zo = __shfl_xor_sync(0xffffffffu, zc, 1);
+      const float z = par ? zo : zc, zq = par ? zc : zo;
+      float su = 0.f, so = 0.f;
+      for (int j = par; j < k - 1; j += 2) {
+        const float uj = rU[j * DVc + c], rj = R[j];
+        su = fmaf(rj * kk[j], uj, su);
+        so = fmaf(rj * kq[j], uj, so);
+      }
+      su += __shfl_xor_sync(0xffffffffu, su, 1);
+      so += __shfl_xor_sync(0xffffffffu, so, 1);
+      const float u = beta * ((vs[c] - g * z) - su);
+      const float o = fmaf(kq[k - 1], u, fmaf(g, zq, so));  // R_{k-1} = 1
+      if (par == 0) {
         if (!flush) p.ubuf[(bh * p.cap + k - 1) * DVc + c] = u;
         S.ucur[c] = u;
       } else {
-        float o0 = g * zc, o1 = 0.f;
-        int i = 0;
-        for (; i + 1 < k - 1; i += 2) {
-          o0 = fmaf(R[i] * kq[i], rU[i * DVc + c], o0);
-          o1 = fmaf(R[i + 1] * kq[i + 1], rU[(i + 1) * DVc + c], o1);
-        }
-        if (i < k - 1) o0 = fmaf(R[i] * kq[i], rU[i * DVc + c], o0);
-        S.opart[c] = o0 + o1;
+        p.y[b * p.bs_y + (size_t)h * DVc + c] = p.scale * o;
       }
     }
-    bar_sync(1, kThreads);
-    if (tid >= 128) {
-      const int c = tid - 128;
-      const float o = fmaf(kq[k - 1], S.ucur[c], S.opart[c]);  // R_{k-1} = 1
-      p.y[b * p.bs_y + (size_t)h * DVc + c] = p.scale * o;
-    }
+    if (flush) bar_sync(1, kThreads);  // the fold reads every column's u
     if constexpr (MMA) {
       if (mma_fold) {
         // ---- P5 on the tensor cores: the previous fold's accumulator reads
@@ -872,6 +887,20 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_verify_kernel(const GDNParams
   }
   __syncthreads();
 
+  // ---- append the drafts at slots nb .. nb+nd-1 (input values: the fp32
+  // copies convert back exactly); every committed record is in shared memory
+  for (int e = tid; e < nd * DKc; e += kThreads) {
+    const int d = e / DKc, c = e % DKc;
+    const size_t slot = (bh * p.cap + nb + d) * DKc + c;
+    static_cast<TI *>(p.qbuf)[slot] = from_f32<TI>(S.Qd[d][c]);
+    static_cast<TI *>(p.kbuf)[slot] = from_f32<TI>(S.Kd[d][c]);
+    static_cast<TI *>(p.vbuf)[(bh * p.cap + nb + d) * DVc + c] = from_f32<TI>(S.Vd[d][c]);
+  }
+  if (tid < nd) {
+    p.abuf[bh * p.cap + nb + tid] = S.ad[tid];
+    p.bbuf[bh * p.cap + nb + tid] = S.bd[tid];
+  }
+
   // ---- decay factors (warps 0, 1) and key dots (16 threads per dot)
   if (warp == 0) {  // fold: R_i = prod_{i<m<n1} alpha_m, gamma = prod_{m<n1} alpha_m
     double pr = lane < n1 ? (double)S.af[lane] : 1.0;  // inclusive prefix product
@@ -904,8 +933,9 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_verify_kernel(const GDNParams
     // dots: (d, j < e_d) keys . k_d, then (d, i <= e_d) keys . q_d
     const int nkk = nd * nb + nd * (nd - 1) / 2, nkq = nd * nb + nd * (nd + 1) / 2;
     const int ndot = nkk + nkq;
-    for (int base = 0; base < ndot; base += kThreads / 16) {
-      const int t = base + (tid >> 4), c0 = (tid & 15) * 8;
+    // 8 threads per dot, thread jt of a dot taking the 4-element chunks jt + 8m
+    for (int base = 0; base < ndot; base += kThreads / 8) {
+      const int t = base + (tid >> 3), jt = tid & 7;
       double acc = 0.0, acc1 = 0.0;
       int d = 0, j = 0;
       bool isq = false;
@@ -922,17 +952,21 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_verify_kernel(const GDNParams
         const float *kj = j < nb ? S.Kc[j] : S.Kd[j - nb];
         const float *other = isq ? S.Qd[d] : S.Kd[d];
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          acc += (double)(kj[c0 + e] * other[c0 + e]);
-          acc1 += (double)(kj[c0 + e + 1] * other[c0 + e + 1]);
+        for (int m = 0; m < DKc / 32; ++m) {
+          const int c0 = 4 * (jt + 8 * m);
+          const float4 a4 = *reinterpret_cast<const float4 *>(kj + c0);
+          const float4 o4 = *reinterpret_cast<const float4 *>(other + c0);
+          acc += (double)(a4.x * o4.x);
+          acc1 += (double)(a4.y * o4.y);
+          acc += (double)(a4.z * o4.z);
+          acc1 += (double)(a4.w * o4.w);
         }
         acc += acc1;
       }
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-      if (t < ndot && (tid & 15) == 0) {
+      if (t < ndot && jt == 0) {
         if (isq) S.KQ[d][j] = (float)acc;
         else S.G[d][j] = (float)acc;
       }
@@ -975,44 +1009,32 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_verify_kernel(const GDNParams
   }
   __syncthreads();
 
-  // ---- drafts in order: correction u_e, output o_d (one thread per column)
-  if (tid < DVc) {
-    const int c = tid;
+  // ---- drafts in order: correction u_e, output o_d.  Thread pair (2c, 2c+1)
+  // owns column c and splits the older records by parity (one load of u_j for
+  // both sums); the pair adds the two halves, so both hold u_e and o_d.
+  {
+    const int c = tid >> 1, par = tid & 1;
     for (int d = 0; d < nd; ++d) {
       const int e = nb + d;
-      float a0 = S.Vd[d][c] - S.gam[d] * S.z[d][c], a1 = 0.f;
-      int j = 0;
-      for (; j + 1 < e; j += 2) {
-        a0 = fmaf(-S.R[d][j] * S.G[d][j], S.U[j][c], a0);
-        a1 = fmaf(-S.R[d][j + 1] * S.G[d][j + 1], S.U[j + 1][c], a1);
+      float su = 0.f, so = 0.f;
+      for (int j = par; j < e; j += 2) {
+        const float uj = S.U[j][c], rj = S.R[d][j];
+        su = fmaf(rj * S.G[d][j], uj, su);
+        so = fmaf(rj * S.KQ[d][j], uj, so);
       }
-      if (j < e) a0 = fmaf(-S.R[d][j] * S.G[d][j], S.U[j][c], a0);
-      const float u = S.bd[d] * (a0 + a1);
-      S.U[e][c] = u;
-      p.ubuf[(bh * p.cap + e) * DVc + c] = u;
-      float o0 = S.gam[d] * S.z[nd + d][c], o1 = 0.f;
-      int i = 0;
-      for (; i + 1 <= e; i += 2) {
-        o0 = fmaf(S.R[d][i] * S.KQ[d][i], S.U[i][c], o0);
-        o1 = fmaf(S.R[d][i + 1] * S.KQ[d][i + 1], S.U[i + 1][c], o1);
+      su += __shfl_xor_sync(0xffffffffu, su, 1);
+      so += __shfl_xor_sync(0xffffffffu, so, 1);
+      const float g = S.gam[d];
+      const float u = S.bd[d] * ((S.Vd[d][c] - g * S.z[d][c]) - su);
+      if (par == 0) {
+        S.U[e][c] = u;
+        p.ubuf[(bh * p.cap + e) * DVc + c] = u;
+      } else {
+        const float o = fmaf(S.R[d][e] * S.KQ[d][e], u, fmaf(g, S.z[nd + d][c], so));
+        p.y[b * p.bs_y + (size_t)(d * p.H + h) * DVc + c] = p.scale * o;
       }
-      if (i <= e) o0 = fmaf(S.R[d][i] * S.KQ[d][i], S.U[i][c], o0);
-      p.y[b * p.bs_y + (size_t)(d * p.H + h) * DVc + c] = p.scale * (o0 + o1);
+      __syncwarp();  // u_e is read by both threads of the pair for later drafts
     }
-  }
-  // ---- append the drafts at slots nb .. nb+nd-1 (input values, unrounded)
-  for (int e = tid; e < nd * DKc; e += kThreads) {
-    const int d = e / DKc, c = e % DKc;
-    const int64_t o = (int64_t)(d * p.H + h) * DKc + c;
-    const size_t slot = (bh * p.cap + nb + d) * DKc + c;
-    static_cast<TI *>(p.qbuf)[slot] = static_cast<const TI *>(p.q)[b * p.bs_q + o];
-    static_cast<TI *>(p.kbuf)[slot] = static_cast<const TI *>(p.k)[b * p.bs_k + o];
-    static_cast<TI *>(p.vbuf)[(bh * p.cap + nb + d) * DVc + c] =
-        static_cast<const TI *>(p.v)[b * p.bs_v + (int64_t)(d * p.H + h) * DVc + c];
-  }
-  if (tid < nd) {
-    p.abuf[bh * p.cap + nb + tid] = S.ad[tid];
-    p.bbuf[bh * p.cap + nb + tid] = S.bd[tid];
   }
   if (tid == 0) p.len[bh] = nb;
 }

@@ -183,24 +183,48 @@ __global__ void __launch_bounds__(kThreads, 2) kda_kernel(const GDNParams p) {
 
   const int row0 = kKRows * warp;
   if constexpr (kOut) {
-    // decay-weighted key dots, 16 threads per dot, fp64 sums:
+    // decay-weighted key dots, fp64 sums:
     // G_j = k_j . (R_j o k_last) (j < last), KQ_i = k_i . (R_i o q) (i <= last)
     const int ndot = 2 * n - 1;
-    for (int base = 0; base < ndot; base += kThreads / 16) {
-      const int d = base + (tid >> 4), c0 = (tid & 15) * 8;
+    if constexpr (MODE == kKdaFull) {  // one dot (n = 1): 16 threads
+      const int c0 = (tid & 15) * 8;
       double acc = 0.0;
-      if (d < ndot) {
-        const int i = d < last ? d : d - last;
-        const float *other = d < last ? S.K[last] : S.q;
+      if (tid < 16) {
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          acc += (double)(S.K[i][c0 + e] * S.R[i][c0 + e]) * (double)other[c0 + e];
+          acc += (double)(S.K[0][c0 + e] * S.R[0][c0 + e]) * (double)S.q[c0 + e];
       }
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       acc += __shfl_xor_sync(0xffffffffu, acc, 4);
       acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-      if (d < ndot && (tid & 15) == 0) {
+      if (tid == 0) S.KQ[0] = (float)acc;
+    } else
+    // 8 threads per dot (one pass for up to 32 dots), thread j of a dot
+    // taking the 4-element chunks j + 8m
+    for (int base = 0; base < ndot; base += kThreads / 8) {
+      const int d = base + (tid >> 3), j = tid & 7;
+      double acc = 0.0, acc1 = 0.0;
+      if (d < ndot) {
+        const int i = d < last ? d : d - last;
+        const float *other = d < last ? S.K[last] : S.q;
+#pragma unroll
+        for (int m = 0; m < KDc / 32; ++m) {
+          const int c0 = 4 * (j + 8 * m);
+          const float4 kv = *reinterpret_cast<const float4 *>(&S.K[i][c0]);
+          const float4 rv = *reinterpret_cast<const float4 *>(&S.R[i][c0]);
+          const float4 ov = *reinterpret_cast<const float4 *>(&other[c0]);
+          acc += (double)(kv.x * rv.x) * (double)ov.x;
+          acc1 += (double)(kv.y * rv.y) * (double)ov.y;
+          acc += (double)(kv.z * rv.z) * (double)ov.z;
+          acc1 += (double)(kv.w * rv.w) * (double)ov.w;
+        }
+        acc += acc1;
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      if (d < ndot && j == 0) {
         if (d < last) S.G[d] = (float)acc;
         else S.KQ[d - last] = (float)acc;
       }
@@ -215,22 +239,33 @@ __global__ void __launch_bounds__(kThreads, 2) kda_kernel(const GDNParams p) {
     *reinterpret_cast<float4 *>(&S.part[warp][0][4 * lane]) = pk;
     *reinterpret_cast<float4 *>(&S.part[warp][1][4 * lane]) = pq;
     __syncthreads();
-    if (tid < KVc) {
-      const int c = tid;
-      float z = 0.f, zq = 0.f;
+    {
+      // thread pair (2c, 2c+1) owns column c: the even thread sums the
+      // partials of z, the odd one those of zq, and they swap; each runs over
+      // the older records of its parity (one load of u_j for both sums) and
+      // the pair adds the two halves
+      const int c = tid >> 1, par = tid & 1;
+      float zc = 0.f;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        z += S.part[w][0][c];
-        zq += S.part[w][1][c];
+      for (int w = 0; w < 8; ++w) zc += S.part[w][par][c];
+      const float zo = __shfl_xor_sync(0xffffffffu, zc, 1);
+      const float z = par ? zo : zc, zq = par ? zc : zo;
+      float su = 0.f, so = 0.f;
+      for (int j = par; j < last; j += 2) {
+        const float uj = S.U[j][c];
+        su = fmaf(S.G[j], uj, su);
+        so = fmaf(S.KQ[j], uj, so);
       }
-      float a0 = S.v[c] - z;
-      for (int j = 0; j < last; ++j) a0 = fmaf(-S.G[j], S.U[j][c], a0);
-      const float u = S.beta * a0;
-      S.U[last][c] = u;
-      float o = zq;
-      for (int i = 0; i <= last; ++i) o = fmaf(S.KQ[i], S.U[i][c], o);
-      p.y[b * p.bs_y + (size_t)h * KVc + c] = p.scale * o;
-      if (MODE == kKdaDecode && !fold) p.ubuf[(bh * p.cap + last) * KVc + c] = u;
+      su += __shfl_xor_sync(0xffffffffu, su, 1);
+      so += __shfl_xor_sync(0xffffffffu, so, 1);
+      const float u = S.beta * ((S.v[c] - z) - su);
+      if (par == 0) {
+        S.U[last][c] = u;
+        if (MODE == kKdaDecode && !fold) p.ubuf[(bh * p.cap + last) * KVc + c] = u;
+      } else {
+        const float o = fmaf(S.KQ[last], u, zq + so);
+        p.y[b * p.bs_y + (size_t)h * KVc + c] = p.scale * o;
+      }
     }
     if (MODE == kKdaDecode && !fold && !p.inplace) {
       // append this step's record (input values, unrounded)

@@ -294,6 +294,40 @@ struct GdnLayout {
     d.NS = 0;
     return d;
   }
+  // Two consumer groups (bf16 keys, tensor-core fold): per group the decay
+  // ratios and key dots R | kk | kq | gamma, the partial sums [4][2][128] and
+  // the current correction [128], and a fold operand area; a ring of exactly
+  // 4 half-tiles and an even number of record buffers (4, else 2), so that
+  // each group owns its slots and buffers and waits on them in its own order.
+  __host__ static GdnLayout make2(int L, int budget) {
+    GdnLayout d;
+    d.L = L;
+    d.stage_floats = 3 * 128 + ((L + 3) & ~3) + 4;
+    d.db_floats = 3 * ((L + 3) & ~3) + 4;
+    for (d.NR = 4; d.NR >= 2; d.NR -= 2) {
+      int o = 0;
+      d.off_bars = o;
+      o += a128(8 * (2 * 8 + 2 * 4) + 2 * 8 + 4);  // ring, records, two fold MMAs, TMEM base
+      d.off_recK = o;
+      o += a128(d.NR * L * DKc * 2);
+      d.off_recU = o;
+      o += a128(d.NR * L * DVc * 4);
+      d.off_stage = o;
+      o += a128(d.NR * d.stage_floats * 4);
+      d.off_db = o;
+      o += a128(2 * d.db_floats * 4);
+      d.off_single = o;
+      o += a128(2 * (4 * 2 * 128 + 128) * 4);
+      d.off_umma = o;
+      o += 2 * 4 * 128 * 32;
+      d.off_ring = o;
+      d.NS = 4;
+      d.total = o + d.NS * kHalfBytes;
+      if (d.total <= budget) return d;
+    }
+    d.NS = 0;
+    return d;
+  }
 };
 
 struct GdnPtrs {
@@ -319,12 +353,36 @@ struct GdnPtrs {
   }
 };
 
+// Shared memory of the two-group decode kernel (GdnLayout::make2).
+struct Gdn2Ptrs {
+  uint64_t *full, *empty, *rfull, *rempty, *mma;  // mma[2]: one per group
+  uint32_t *tmem_slot;
+  unsigned char *recK, *ring, *umma;
+  float *recU, *stage, *db, *part, *ucur;
+  __device__ Gdn2Ptrs(unsigned char *smem, const GdnLayout &l) {
+    full = reinterpret_cast<uint64_t *>(smem + l.off_bars);
+    empty = full + 8;
+    rfull = empty + 8;
+    rempty = rfull + 4;
+    mma = rempty + 4;
+    tmem_slot = reinterpret_cast<uint32_t *>(mma + 2);
+    umma = smem + l.off_umma;
+    recK = smem + l.off_recK;
+    recU = reinterpret_cast<float *>(smem + l.off_recU);
+    stage = reinterpret_cast<float *>(smem + l.off_stage);
+    db = reinterpret_cast<float *>(smem + l.off_db);
+    part = reinterpret_cast<float *>(smem + l.off_single);  // [2][4][2][128]
+    ucur = part + 2 * 4 * 2 * 128;                           // [2][128]
+    ring = smem + l.off_ring;
+  }
+};
+
 // Stager warp: all loads of item `it` first (none depends on the length:
 // every alpha slot of the window is read), then shared-memory writes, then
 // (lane 0) the bulk copies of the buffered k and u records.
-template <typename TI>
+template <typename TI, typename Ptrs>
 __device__ __forceinline__ bool gdn_stage(const GDNParams &p, const GdnLayout &lay,
-                                          const GdnPtrs &S, int item, int it, int lane,
+                                          const Ptrs &S, int item, int it, int lane,
                                           volatile int *abort_flag) {
   const int L = lay.L;
   const int rb = it % lay.NR;
@@ -400,9 +458,10 @@ __device__ __forceinline__ bool gdn_stage(const GDNParams &p, const GdnLayout &l
 template <typename TI>
 __device__ __forceinline__ void gdn_build_fold_operands(unsigned char *ua, const float *rU,
                                                         const float *ucur, const float *R,
-                                                        const TI *rK, int k, int tid) {
+                                                        const TI *rK, int k, int tid,
+                                                        int nthr = kThreads) {
   unsigned char *ub = ua + 3 * 128 * 32;
-  for (int e = tid; e < 128 * 8; e += kThreads) {
+  for (int e = tid; e < 128 * 8; e += nthr) {
     const int c = e % 128, q = e / 128, i0 = 2 * q, i1 = i0 + 1;
     auto uval = [&](int i) -> float {
       return i < k - 1 ? rU[i * DVc + c] : (i == k - 1 ? ucur[c] : 0.f);
@@ -776,6 +835,350 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
 }
 
 
+// Two consumer groups (bf16 keys, tensor-core fold).  Warps 0-3 and 4-7 take
+// alternate work items of this CTA (group g: items it = g, g + 2, ...), so one
+// item's latency chain (key dots, partial products, u and output, fold)
+// overlaps the other group's.  Same producer, stager and ring as the kernel
+// above with exactly 4 half-tile slots: item it fills slots 2(it%2) and
+// 2(it%2)+1, so each group owns one pair; with an even number of record
+// buffers each group also owns its buffers.  A group therefore never waits on
+// a barrier phase beyond the next one of its own slots and buffers.  Within a group warp w (0-3) reads
+// rows 32w..32w+31 of the tile straight from its slot (no register copy: the
+// tile is used once on non-flush steps, and the fold epilogue reads it again
+// from the slot); thread c of the group forms u and the output of column c;
+// the fold's accumulator is this group's 128 of 256 tensor-memory columns.
+template <typename TI>
+__global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode2_kernel(const GDNParams p,
+                                                                    const GdnLayout lay) {
+  static_assert(std::is_same<TI, __nv_bfloat16>::value, "tensor-core fold: bf16 keys");
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int abort_word;
+  volatile int *abort_flag = &abort_word;
+  const Gdn2Ptrs S(smem, lay);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nitems = p.B * p.H;
+  const int L = lay.L;
+
+  if (tid == 0) {
+    for (int s = 0; s < 8; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 4);  // the 4 warps of the group that owns the slot
+    }
+    for (int r = 0; r < 4; ++r) {
+      mbar_init(&S.rfull[r], 1);
+      mbar_init(&S.rempty[r], 4);
+    }
+    mbar_init(&S.mma[0], 1);
+    mbar_init(&S.mma[1], 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) umma::alloc(S.tmem_slot, 256);
+  umma::fence_before_sync();
+  __syncthreads();
+
+  if (warp == 8) {  // tile producer: half-tiles in (item, half) order, 4 slots
+    if (lane != 0) return;
+    int slot = 0;
+    uint32_t sphase = 0, issued = 0, parity = 0;
+    bool failed = false;
+    for (int item = blockIdx.x; item < nitems && !failed; item += gridDim.x) {
+      for (int half = 0; half < 2; ++half) {
+        if (*abort_flag || !mbar_wait(&S.empty[slot], sphase ^ 1, kWaitLimitNs, abort_flag) ||
+            *abort_flag) {
+          failed = true;
+          break;
+        }
+        mbar_arrive_expect_tx(&S.full[slot], kHalfBytes);
+        bulk_g2s(S.ring + slot * kHalfBytes,
+                 p.h0 + (size_t)item * DKc * DVc + (size_t)half * kHalfRows * DVc, kHalfBytes,
+                 &S.full[slot]);
+        issued |= 1u << slot;
+        parity = (parity & ~(1u << slot)) | (sphase << slot);
+        if (++slot == lay.NS) {
+          slot = 0;
+          sphase ^= 1;
+        }
+      }
+    }
+    if (failed) {
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    // every copy issued here lands before the warp returns
+    for (int s2 = 0; s2 < lay.NS; ++s2)
+      if (issued & (1u << s2)) mbar_wait(&S.full[s2], (parity >> s2) & 1u);
+    return;
+  }
+  if (warp == 9) {  // stager
+    int it = 0;
+    ArmedRecords armed;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+      const bool abort_now = __any_sync(0xffffffffu, *abort_flag != 0);
+      if (!abort_now && item == p.hold_item) continue;  // test hook: never staged
+      if (abort_now || !gdn_stage<TI>(p, lay, S, item, it, lane, abort_flag)) {
+        if (lane == 0 && !*abort_flag) {
+          report(p.status, RSSM_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      armed.arm(it % lay.NR, (it / lay.NR) & 1);
+    }
+    if (lane == 0) armed.drain(S.rfull, lay.NR);  // no record copy outlives the warp
+    __syncwarp();
+    return;
+  }
+
+  // Consumer group grp (warps 4grp .. 4grp+3), thread gt = column c.
+  constexpr int kG = 128;  // threads per group
+  const int grp = warp >> 2, gw = warp & 3, gt = tid & (kG - 1);
+  const uint32_t gbar = 1 + grp;  // the group's named barrier
+  umma::fence_after_sync();
+  const uint32_t tmem_base = *S.tmem_slot;
+  const uint32_t tmem = tmem_base + 128u * grp;  // this group's accumulator columns
+  uint32_t n_mma = 0;
+  float *part = S.part + grp * (4 * 2 * 128);
+  float *ucur = S.ucur + grp * 128;
+  unsigned char *ua = S.umma + grp * (4 * 128 * 32);
+  uint64_t *mbar_mma = &S.mma[grp];
+  float *db = S.db + grp * lay.db_floats;
+  float *R = db, *kk = db + ((L + 3) & ~3), *kq = kk + ((L + 3) & ~3);
+  float *gam = kq + ((L + 3) & ~3);
+
+  int it = grp;
+  for (int item = blockIdx.x + grp * gridDim.x; item < nitems; item += 2 * gridDim.x, it += 2) {
+    const int rb = it % lay.NR;
+    const uint32_t rphase = (it / lay.NR) & 1;
+    const int b = item / p.H, h = item - (item / p.H) * p.H;
+    const size_t bh = (size_t)item;
+    const float *st = S.stage + rb * lay.stage_floats;
+    const float *qs = st, *ks = st + 128, *vs = st + 256, *alpha = st + 384;
+    const float *tail = alpha + ((L + 3) & ~3);
+    const TI *rK = reinterpret_cast<const TI *>(S.recK) + (size_t)rb * L * DKc;
+    const float *rU = S.recU + (size_t)rb * L * DVc;
+    // this item's two half-tiles: slots 2 (it % 2) and 2 (it % 2) + 1, phase it / 2
+    const int sl0 = 2 * (it & 1), sl1 = sl0 + 1;
+    const uint32_t tphase = (it >> 1) & 1;
+
+    const bool got = mbar_wait(&S.rfull[rb], rphase, p.wait_ns, abort_flag);
+    if (!got) {
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    if (bar_or(gbar, kG, !got || *abort_flag)) break;
+    const int n0 = reinterpret_cast<const int *>(tail)[1];
+    if (reinterpret_cast<const int *>(tail)[2]) {
+      if (gt == 0) report(p.status, RSSM_ERR_STATE);
+      const int sl = gw < 2 ? sl0 : sl1;
+      if (!mbar_wait(&S.full[sl], tphase, p.wait_ns, abort_flag)) {
+        if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&S.empty[sl0]);
+        mbar_arrive(&S.empty[sl1]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.rempty[rb]);
+      continue;
+    }
+    const int k = n0 + 1;
+    const bool flush = (k == L);
+    const float beta = tail[0];
+
+    // ---- P1: appends (an in-place step's record is in its slot already),
+    // decay ratios, k_j.k and k_i.q
+    if (!flush && !p.inplace) {
+      const size_t slot = bh * p.cap + k - 1;
+      static_cast<TI *>(p.qbuf)[slot * DKc + gt] = from_f32<TI>(qs[gt]);
+      static_cast<TI *>(p.kbuf)[slot * DKc + gt] = rK[(k - 1) * DKc + gt];
+      static_cast<TI *>(p.vbuf)[slot * DVc + gt] = from_f32<TI>(vs[gt]);
+      if (gt == 0) {
+        p.abuf[slot] = alpha[k - 1];
+        p.bbuf[slot] = beta;
+      }
+    }
+    if (gw == 3) {  // R_i = prod_{i<m<k} alpha_m (lane i), gamma: fp64 suffix-product scan
+      double pr = lane < k ? (double)alpha[lane] : 1.0;  // inclusive: prod_{m >= lane}
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_down_sync(0xffffffffu, pr, o);
+        if (lane + o < 32) pr *= t;
+      }
+      const double nxt = __shfl_down_sync(0xffffffffu, pr, 1);  // prod_{m > lane}
+      if (lane < k) R[lane] = (float)(lane + 1 < 32 ? nxt : 1.0);
+      if (lane == 0) gam[0] = (float)pr;
+    }
+    {
+      // 2k-1 <= 31 dot products of 128 (the window is at most 16):
+      // k_j.k_{k-1} (j < k-1) then k_i.q (i < k); 4 threads per dot, thread j
+      // of a dot takes the 8-element chunks j + 4m (16-byte key loads);
+      // products in fp32 (exact for bf16 inputs), sums in fp64 over two chains
+      const int ndot = 2 * k - 1, d = gt >> 2, j = gt & 3;
+      double acc = 0.0, acc1 = 0.0;
+      if (d < ndot) {
+        const int i = d < k - 1 ? d : d - (k - 1);
+        const float *other = d < k - 1 ? ks : qs;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int c0 = 8 * (j + 4 * m);
+          float kv[8], ov[8];
+          ld8_smem(rK + i * DKc + c0, kv);
+          ld8_smem(other + c0, ov);
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            acc += (double)(kv[e] * ov[e]);
+            acc1 += (double)(kv[e + 1] * ov[e + 1]);
+          }
+        }
+        acc += acc1;
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (d < ndot && j == 0) {
+        if (d < k - 1) kk[d] = (float)acc;
+        else kq[d - (k - 1)] = (float)acc;
+      }
+    }
+
+    // ---- P2: partial h0^T k and h0^T q over this warp's 32 rows, read from
+    // the slot (rows 64 half + 32 (gw % 2) ..)
+    const int half = gw >> 1, sl = half ? sl1 : sl0;
+    if (!mbar_wait(&S.full[sl], tphase, p.wait_ns, abort_flag)) {
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    {
+      const float *tile = reinterpret_cast<const float *>(S.ring + sl * kHalfBytes) +
+                          (size_t)(32 * (gw & 1)) * DVc + 4 * lane;
+      const int row0 = 32 * gw;  // = 64 half + 32 (gw % 2)
+      float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+#pragma unroll 2
+      for (int t = 0; t < 8; ++t) {
+        const float4 k4 = *reinterpret_cast<const float4 *>(&ks[row0 + 4 * t]);
+        const float4 q4 = *reinterpret_cast<const float4 *>(&qs[row0 + 4 * t]);
+        const float kr[4] = {k4.x, k4.y, k4.z, k4.w}, qr[4] = {q4.x, q4.y, q4.z, q4.w};
+        float4 x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = *reinterpret_cast<const float4 *>(tile + (4 * t + e) * DVc);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          pk = fma4x(kr[e], x[e], pk);
+          pq = fma4x(qr[e], x[e], pq);
+        }
+      }
+      *reinterpret_cast<float4 *>(&part[(gw * 2 + 0) * 128 + 4 * lane]) = pk;
+      *reinterpret_cast<float4 *>(&part[(gw * 2 + 1) * 128 + 4 * lane]) = pq;
+    }
+    if (!flush) {  // the fold epilogue reads both half-tiles again
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&S.empty[sl0]);
+        mbar_arrive(&S.empty[sl1]);
+      }
+    }
+    bar_sync(gbar, kG);
+
+    // ---- P3 + P4: thread c sums the 4 warps' partials of z = h0^T k and
+    // zq = h0^T q for column c (fixed order), then one pass over the older
+    // records gives both the correction's and the output's sums (one load of
+    // u_j each, even and odd records in separate accumulators)
+    {
+      const int c = gt;
+      const float g = gam[0];
+      float z = 0.f, zq = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        z += part[(w * 2 + 0) * 128 + c];
+        zq += part[(w * 2 + 1) * 128 + c];
+      }
+      float su0 = 0.f, su1 = 0.f, so0 = 0.f, so1 = 0.f;
+      int jj = 0;
+      for (; jj + 1 < k - 1; jj += 2) {
+        const float u0 = rU[jj * DVc + c], u1 = rU[(jj + 1) * DVc + c];
+        const float r0 = R[jj], r1 = R[jj + 1];
+        su0 = fmaf(r0 * kk[jj], u0, su0);
+        so0 = fmaf(r0 * kq[jj], u0, so0);
+        su1 = fmaf(r1 * kk[jj + 1], u1, su1);
+        so1 = fmaf(r1 * kq[jj + 1], u1, so1);
+      }
+      if (jj < k - 1) {
+        const float u0 = rU[jj * DVc + c], r0 = R[jj];
+        su0 = fmaf(r0 * kk[jj], u0, su0);
+        so0 = fmaf(r0 * kq[jj], u0, so0);
+      }
+      const float u = beta * ((vs[c] - g * z) - (su0 + su1));
+      const float o = fmaf(kq[k - 1], u, fmaf(g, zq, so0 + so1));  // R_{k-1} = 1
+      if (!flush) p.ubuf[(bh * p.cap + k - 1) * DVc + c] = u;
+      else ucur[c] = u;
+      p.y[b * p.bs_y + (size_t)h * DVc + c] = p.scale * o;
+    }
+
+    if (flush) {
+      // ---- P5 on the tensor cores: h0 <- gamma h0 + sum_i R_i k_i u_i^T
+      bar_sync(gbar, kG);  // every column's u; the previous fold's reads are done
+      gdn_build_fold_operands<TI>(ua, rU, ucur, R, rK, k, gt, kG);
+      fence_proxy_async_smem();
+      umma::fence_before_sync();
+      bar_sync(gbar, kG);
+      if (gt == 0) {
+        umma::fence_after_sync();
+        const uint32_t id = umma::idesc_bf16_f32(128, 128);
+        const uint64_t bd = umma::smem_desc(ua + 3 * 128 * 32);
+#pragma unroll
+        for (int t3 = 0; t3 < 3; ++t3)
+          umma::mma_bf16(tmem, umma::smem_desc(ua + t3 * 128 * 32), bd, id, t3 > 0);
+        umma::commit(mbar_mma);
+      }
+      const bool done = mbar_wait(mbar_mma, n_mma & 1u, p.wait_ns, abort_flag);
+      ++n_mma;
+      if (!done) {
+        if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      umma::fence_after_sync();
+      // epilogue: lane = column c = 32 gw + lane, all 128 rows, 32 at a time
+      if (!mbar_wait(&S.full[half ? sl0 : sl1], tphase, p.wait_ns, abort_flag)) {
+        if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);  // the other half-tile
+        *abort_flag = 1;
+      }
+      const int c = 32 * gw + lane;
+      const uint32_t taddr = tmem + ((uint32_t)(32 * gw) << 16);
+      const float g = gam[0];
+      float *dst = p.h0 + bh * (DKc * DVc);
+#pragma unroll 1
+      for (int r0 = 0; r0 < DKc; r0 += 32) {
+        const float *tile = reinterpret_cast<const float *>(S.ring + (r0 < 64 ? sl0 : sl1) * kHalfBytes);
+        float dv[32];
+        umma::ld32(taddr + (uint32_t)r0, dv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int r = r0 + i;
+          dst[(size_t)r * DVc + c] = fmaf(g, tile[(r & 63) * DVc + c], dv[i]);
+        }
+      }
+      umma::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&S.empty[sl0]);
+        mbar_arrive(&S.empty[sl1]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.rempty[rb]);
+    if (gt == 0) p.len[bh] = flush ? 0 : k;
+  }
+  if (gt == 0 && n_mma > 0) mbar_wait(mbar_mma, (n_mma - 1) & 1u);  // no MMA outlives the memory
+  umma::fence_before_sync();
+  bar_sync(3, kThreads);
+  umma::fence_after_sync();
+  if (warp == 0) umma::dealloc(tmem_base, 256);
+}
+
 // ============================================================ verify round
 // Speculative verify round of Gated DeltaNet [sitech.ge, "NVIDIA ו-Dao AI Lab
 // הציגו ReplaySSM…", §Reducing state traffic and simplifying rollback], one
@@ -1062,6 +1465,18 @@ int gdn_sm_count() {
 template <typename TI>
 cudaError_t gdn_launch_persistent(const GDNParams &p, cudaStream_t s) {
   constexpr bool kMma = std::is_same<TI, __nv_bfloat16>::value;
+  if constexpr (kMma) {  // two consumer groups when their layout fits
+    const GdnLayout lay2 = GdnLayout::make2(p.L, 227 * 1024);
+    if (lay2.NS == 4) {
+      cudaError_t e = cudaFuncSetAttribute(gdn_decode2_kernel<TI>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, lay2.total);
+      if (e != cudaSuccess) return e;
+      const int nitems = p.B * p.H;
+      const int grid = nitems < gdn_sm_count() ? nitems : gdn_sm_count();
+      gdn_decode2_kernel<TI><<<grid, kThreads + 64, lay2.total, s>>>(p, lay2);
+      return cudaGetLastError();
+    }
+  }
   GdnLayout lay = GdnLayout::make(p.L, (int)sizeof(TI), 220 * 1024, kMma);
   const bool mma = kMma && lay.NS >= 4;
   if (!mma) lay = GdnLayout::make(p.L, (int)sizeof(TI), 220 * 1024);

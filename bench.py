@@ -65,7 +65,7 @@ def parse():
 KERNEL_SOURCES = {
     "m2_decode_kernel_m2_serving": ("m2.cu", "m2_device.cuh", "common.cuh", "pipeline.cuh",
                                     "codec.cuh", "internal.h", "umma.cuh"),
-    "gdn_decode_kernel_gdn_serving": ("gdn.cu", "common.cuh", "pipeline.cuh", "internal.h",
+    "gdn_decode2_kernel_gdn_serving": ("gdn.cu", "common.cuh", "pipeline.cuh", "internal.h",
                                       "umma.cuh"),
     "kda_kernel_kda_serving": ("kda.cu", "common.cuh", "internal.h"),
     "m2_verify_kernel_m2_verify": ("m2_verify.cu", "m2_device.cuh", "common.cuh", "pipeline.cuh",
@@ -515,8 +515,8 @@ def bench_gdn(args, dev, peak, rs, bm, wl, torch):
     return {"workload": "gdn_serving", "value": tok / (ms_r * 1e-3), "unit": "tokens/s",
             "ms_per_window": ms_r / n,
             "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
-                         "frac": ach_r / peak, "kernel": "gdn_decode_kernel",
-                         "traffic": recorded_traffic("gdn_decode_kernel_gdn_serving", w.B, 256),
+                         "frac": ach_r / peak, "kernel": "gdn_decode2_kernel",
+                         "traffic": recorded_traffic("gdn_decode2_kernel_gdn_serving", w.B, 256),
                          "algorithmic_bytes_per_launch": wb / L,
                          "bytes": "records with their cached corrections u (as stored)",
                          "frac_input_records_only": ach_rec / peak,

@@ -30,6 +30,7 @@
 // per-channel decay products are taken in fp64 (one thread per channel).
 #include "common.cuh"
 #include "internal.h"
+#include "pipeline.cuh"
 
 namespace rssm {
 namespace {
@@ -303,6 +304,439 @@ __global__ void __launch_bounds__(kThreads, 2) kda_kernel(const GDNParams p) {
   if (tid == 0 && (MODE == kKdaDecode || MODE == kKdaFlush)) p.len[bh] = fold ? 0 : n;
 }
 
+// ============================================================ persistent decode step
+// Persistent replay decode step (one CTA of 320 threads per SM), structured as
+// the two-group Gated DeltaNet kernel: warp 8 streams each item's checkpoint
+// as two 32 KiB half-tiles into a ring of exactly 4 slots, warp 9 stages the
+// item's inputs and bulk-copies its buffered keys, corrections and decay
+// vectors, and two consumer groups of 4 warps take alternate items (item it
+// uses slots 2(it%2), 2(it%2)+1 and record buffer it % NR with NR even, so
+// each group owns its slots and buffers).  Per item, in a group:
+//   * thread c (one key channel) runs the fp64 suffix products of the decays
+//     over the records and overwrites each staged decay with the record's
+//     weighted key w_i[c] = k_i[c] * R_i[c] (the fp32 product both the dots
+//     and the fold use), and forms Gamma o k and Gamma o q;
+//   * 4 threads per key dot: G_j = w_j . k_last, KQ_i = w_i . q (fp64 sums);
+//   * warp w: partial h0^T (Gamma o k), h0^T (Gamma o q) over rows 32w.. from
+//     the slot; thread c: u and the output of column c;
+//   * flush: h0[r] <- Gamma[r] h0[r] + sum_i w_i[r] u_i, rows read from the
+//     slot, written once.
+constexpr int kKHalfRows = KDc / 2, kKHalfBytes = kKHalfRows * KVc * 4;  // 32 KiB
+
+struct KdaLayout {
+  int NR, L, stage_floats, db_floats;
+  int off_bars, off_recK, off_recU, off_recW, off_stage, off_db, off_single, off_ring, total;
+  __host__ static int a128(int v) { return (v + 127) & ~127; }
+  // stage: q, v [128] fp32 | beta, n0, bad, pad; per group: Gamma, kg, qg
+  // [128] | G, KQ [L]; per group: partial sums [4][2][128] | u [128]
+  __host__ static KdaLayout make(int L, int es, int budget) {
+    KdaLayout d;
+    d.L = L;
+    d.stage_floats = 2 * 128 + 4;
+    d.db_floats = 3 * 128 + 2 * ((L + 3) & ~3);
+    for (d.NR = 4; d.NR >= 2; d.NR -= 2) {
+      int o = 0;
+      d.off_bars = o;
+      o += a128(8 * (2 * 8 + 2 * 4));
+      d.off_recK = o;
+      o += a128(d.NR * L * KDc * es);
+      d.off_recU = o;
+      o += a128(d.NR * L * KVc * 4);
+      d.off_recW = o;
+      o += a128(d.NR * L * KDc * 4);
+      d.off_stage = o;
+      o += a128(d.NR * d.stage_floats * 4);
+      d.off_db = o;
+      o += a128(2 * d.db_floats * 4);
+      d.off_single = o;
+      o += a128(2 * (4 * 2 * 128 + 128) * 4);
+      d.off_ring = o;
+      d.total = o + 4 * kKHalfBytes;
+      if (d.total <= budget) return d;
+    }
+    d.NR = 0;
+    return d;
+  }
+};
+
+template <typename TI>
+__device__ __forceinline__ float4 ld4_in(const TI *p) {
+  if constexpr (sizeof(TI) == 4) {
+    return *reinterpret_cast<const float4 *>(p);
+  } else {
+    const uint2 raw = *reinterpret_cast<const uint2 *>(p);
+    const TI *e = reinterpret_cast<const TI *>(&raw);
+    return make_float4(to_f32(e[0]), to_f32(e[1]), to_f32(e[2]), to_f32(e[3]));
+  }
+}
+
+template <typename TI>
+__global__ void __launch_bounds__(kThreads + 64, 1) kda_decode2_kernel(const GDNParams p,
+                                                                    const KdaLayout lay) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int abort_word;
+  volatile int *abort_flag = &abort_word;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.off_bars);
+  uint64_t *empty = full + 8, *rfull = empty + 8, *rempty = rfull + 4;
+  unsigned char *ring = smem + lay.off_ring;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nitems = p.B * p.H;
+  const int L = lay.L, NR = lay.NR;
+
+  if (tid == 0) {
+    for (int s = 0; s < 8; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4);  // the 4 warps of the group that owns the slot
+    }
+    for (int r = 0; r < 4; ++r) {
+      mbar_init(&rfull[r], 1);
+      mbar_init(&rempty[r], 4);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == 8) {  // tile producer: half-tiles in (item, half) order, 4 slots
+    if (lane != 0) return;
+    int slot = 0;
+    uint32_t sphase = 0, issued = 0, parity = 0;
+    bool failed = false;
+    for (int item = blockIdx.x; item < nitems && !failed; item += gridDim.x) {
+      for (int half = 0; half < 2; ++half) {
+        if (*abort_flag || !mbar_wait(&empty[slot], sphase ^ 1, kWaitLimitNs, abort_flag) ||
+            *abort_flag) {
+          failed = true;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[slot], kKHalfBytes);
+        bulk_g2s(ring + slot * kKHalfBytes,
+                 p.h0 + (size_t)item * KDc * KVc + (size_t)half * kKHalfRows * KVc, kKHalfBytes,
+                 &full[slot]);
+        issued |= 1u << slot;
+        parity = (parity & ~(1u << slot)) | (sphase << slot);
+        if (++slot == 4) {
+          slot = 0;
+          sphase ^= 1;
+        }
+      }
+    }
+    if (failed) {
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    for (int s2 = 0; s2 < 4; ++s2)  // every copy issued here lands before the warp returns
+      if (issued & (1u << s2)) mbar_wait(&full[s2], (parity >> s2) & 1u);
+    return;
+  }
+
+  if (warp == 9) {  // stager: all loads of an item first, then shared-memory writes and copies
+    int it = 0;
+    ArmedRecords armed;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+      const bool abort_now = __any_sync(0xffffffffu, *abort_flag != 0);
+      if (!abort_now && item == p.hold_item) continue;  // test hook: never staged
+      const int rb = it % NR;
+      bool ok = !abort_now;
+      if (ok && lane == 0)
+        ok = mbar_wait(&rempty[rb], ((it / NR) & 1) ^ 1, kWaitLimitNs, abort_flag) && !*abort_flag;
+      if (!__shfl_sync(0xffffffffu, (int)ok, 0)) {
+        if (lane == 0 && !*abort_flag) {
+          report(p.status, RSSM_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      const int b = item / p.H, h = item - (item / p.H) * p.H;
+      const size_t bh = (size_t)item;
+      const int n0 = __ldcg(&p.len[bh]);
+      const TI *qin = static_cast<const TI *>(p.q) + b * p.bs_q + (size_t)h * KDc;
+      const TI *kin = static_cast<const TI *>(p.k) + b * p.bs_k + (size_t)h * KDc;
+      const TI *vin = static_cast<const TI *>(p.v) + b * p.bs_v + (size_t)h * KVc;
+      const float *ain = p.alpha + b * p.bs_a + (size_t)h * KDc;
+      const float *bin = p.beta + b * p.bs_b + h;
+      if (p.inplace) {  // the record is already in slot len: read it from there
+        const size_t slot = bh * p.cap + min(max(n0, 0), L - 1);  // stays in bounds
+        qin = static_cast<const TI *>(p.qbuf) + slot * KDc;
+        kin = static_cast<const TI *>(p.kbuf) + slot * KDc;
+        vin = static_cast<const TI *>(p.vbuf) + slot * KVc;
+        ain = p.abuf + slot * KDc;
+        bin = p.bbuf + slot;
+      }
+      TI qv[4], kv[4], vv[4];
+      float av[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        qv[u] = qin[lane + 32 * u];
+        kv[u] = kin[lane + 32 * u];
+        vv[u] = vin[lane + 32 * u];
+        av[u] = ain[lane + 32 * u];
+      }
+      const float b_cur = *bin;
+      const bool bad = n0 < 0 || n0 >= L;
+      const int k = min(max(n0 + 1, 1), L);  // copies stay in bounds even for a bad length
+      float *st = reinterpret_cast<float *>(smem + lay.off_stage) + rb * lay.stage_floats;
+      TI *rK = reinterpret_cast<TI *>(smem + lay.off_recK) + (size_t)rb * L * KDc;
+      float *rW = reinterpret_cast<float *>(smem + lay.off_recW) + (size_t)rb * L * KDc;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = lane + 32 * u;
+        st[c] = to_f32(qv[u]);
+        st[128 + c] = to_f32(vv[u]);
+        rK[(k - 1) * KDc + c] = kv[u];
+        rW[(k - 1) * KDc + c] = av[u];
+      }
+      if (lane == 0) {
+        st[256] = b_cur;
+        reinterpret_cast<int *>(st)[257] = n0;
+        reinterpret_cast<int *>(st)[258] = bad;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t bK = (k - 1) * KDc * sizeof(TI), bU = (k - 1) * KVc * 4, bW = (k - 1) * KDc * 4;
+        mbar_arrive_expect_tx(&rfull[rb], bK + bU + bW);
+        if (k > 1) {
+          bulk_g2s(rK, static_cast<const TI *>(p.kbuf) + bh * p.cap * KDc, bK, &rfull[rb]);
+          bulk_g2s(reinterpret_cast<float *>(smem + lay.off_recU) + (size_t)rb * L * KVc,
+                   p.ubuf + bh * p.cap * KVc, bU, &rfull[rb]);
+          bulk_g2s(rW, p.abuf + bh * p.cap * KDc, bW, &rfull[rb]);
+        }
+      }
+      armed.arm(rb, (it / NR) & 1);
+    }
+    if (lane == 0) armed.drain(rfull, NR);  // no record copy outlives the warp
+    __syncwarp();
+    return;
+  }
+
+  // Consumer group grp (warps 4grp .. 4grp+3), thread gt = key channel / column.
+  constexpr int kG = 128;
+  const int grp = warp >> 2, gw = warp & 3, gt = tid & (kG - 1);
+  const uint32_t gbar = 1 + grp;
+  float *db = reinterpret_cast<float *>(smem + lay.off_db) + grp * lay.db_floats;
+  float *gamv = db, *kg = db + 128, *qg = db + 256, *G = db + 384, *KQ = G + ((L + 3) & ~3);
+  float *part = reinterpret_cast<float *>(smem + lay.off_single) + grp * (4 * 2 * 128 + 128);
+  float *ucur = part + 4 * 2 * 128;
+
+  int it = grp;
+  for (int item = blockIdx.x + grp * gridDim.x; item < nitems; item += 2 * gridDim.x, it += 2) {
+    const int rb = it % NR;
+    const int b = item / p.H, h = item - (item / p.H) * p.H;
+    const size_t bh = (size_t)item;
+    const float *st = reinterpret_cast<const float *>(smem + lay.off_stage) + rb * lay.stage_floats;
+    const float *qs = st, *vs = st + 128;
+    const TI *rK = reinterpret_cast<const TI *>(smem + lay.off_recK) + (size_t)rb * L * KDc;
+    const float *rU = reinterpret_cast<const float *>(smem + lay.off_recU) + (size_t)rb * L * KVc;
+    float *rW = reinterpret_cast<float *>(smem + lay.off_recW) + (size_t)rb * L * KDc;
+    const int sl0 = 2 * (it & 1), sl1 = sl0 + 1;
+    const uint32_t tphase = (it >> 1) & 1;
+
+    const bool got = mbar_wait(&rfull[rb], (it / NR) & 1, p.wait_ns, abort_flag);
+    if (!got) {
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    if (bar_or(gbar, kG, !got || *abort_flag)) break;
+    const int n0 = reinterpret_cast<const int *>(st)[257];
+    if (reinterpret_cast<const int *>(st)[258]) {
+      if (gt == 0) report(p.status, RSSM_ERR_STATE);
+      if (!mbar_wait(&full[gw < 2 ? sl0 : sl1], tphase, p.wait_ns, abort_flag)) {
+        if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&empty[sl0]);
+        mbar_arrive(&empty[sl1]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rempty[rb]);
+      continue;
+    }
+    const int k = n0 + 1, last = n0;
+    const bool fold = (k == L);
+    const float beta = st[256];
+
+    // ---- appends (an in-place step's record is in its slot already)
+    if (!fold && !p.inplace) {
+      const size_t slot = bh * p.cap + last;
+      static_cast<TI *>(p.qbuf)[slot * KDc + gt] = from_f32<TI>(qs[gt]);
+      static_cast<TI *>(p.kbuf)[slot * KDc + gt] = rK[last * KDc + gt];
+      static_cast<TI *>(p.vbuf)[slot * KVc + gt] = from_f32<TI>(vs[gt]);
+      p.abuf[slot * KDc + gt] = rW[last * KDc + gt];
+      if (gt == 0) p.bbuf[slot] = beta;
+    }
+    // ---- channel c: decay suffix products in fp64; each staged decay is
+    // replaced by the record's weighted key w_i[c] = k_i[c] * R_i[c]
+    {
+      const int c = gt;
+      double pr = 1.0;
+      for (int i = last; i >= 0; --i) {
+        const float a = rW[i * KDc + c];
+        rW[i * KDc + c] = to_f32(rK[i * KDc + c]) * (float)pr;
+        pr *= (double)a;
+      }
+      gamv[c] = (float)pr;
+      kg[c] = (float)(pr * (double)to_f32(rK[last * KDc + c]));
+      qg[c] = (float)(pr * (double)qs[c]);
+    }
+    bar_sync(gbar, kG);
+    // ---- 2k-1 <= 31 decay-weighted key dots (the window is at most 16):
+    // G_j = w_j . k_last (j < last), KQ_i = w_i . q (i <= last); 4 threads per
+    // dot, thread j4 takes the 4-element chunks j4 + 4m; fp64 sums
+    {
+      const int ndot = 2 * k - 1, d = gt >> 2, j4 = gt & 3;
+      double acc = 0.0, acc1 = 0.0;
+      if (d < ndot) {
+        const int i = d < last ? d : d - last;
+#pragma unroll
+        for (int m = 0; m < KDc / 16; ++m) {
+          const int c0 = 4 * (j4 + 4 * m);
+          const float4 w4 = *reinterpret_cast<const float4 *>(&rW[i * KDc + c0]);
+          const float4 o4 = d < last ? ld4_in<TI>(rK + last * KDc + c0)
+                                     : *reinterpret_cast<const float4 *>(&qs[c0]);
+          acc += (double)w4.x * (double)o4.x;
+          acc1 += (double)w4.y * (double)o4.y;
+          acc += (double)w4.z * (double)o4.z;
+          acc1 += (double)w4.w * (double)o4.w;
+        }
+        acc += acc1;
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (d < ndot && j4 == 0) {
+        if (d < last) G[d] = (float)acc;
+        else KQ[d - last] = (float)acc;
+      }
+    }
+    // ---- partial h0^T (Gamma o k) and h0^T (Gamma o q) over this warp's 32
+    // rows, read from the slot
+    const int half = gw >> 1, sl = half ? sl1 : sl0;
+    if (!mbar_wait(&full[sl], tphase, p.wait_ns, abort_flag)) {
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    {
+      const float *tile = reinterpret_cast<const float *>(ring + sl * kKHalfBytes) +
+                          (size_t)(32 * (gw & 1)) * KVc + 4 * lane;
+      const int row0 = 32 * gw;
+      float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+#pragma unroll 2
+      for (int t = 0; t < 8; ++t) {
+        const float4 k4 = *reinterpret_cast<const float4 *>(&kg[row0 + 4 * t]);
+        const float4 q4 = *reinterpret_cast<const float4 *>(&qg[row0 + 4 * t]);
+        const float kr[4] = {k4.x, k4.y, k4.z, k4.w}, qr[4] = {q4.x, q4.y, q4.z, q4.w};
+        float4 x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = *reinterpret_cast<const float4 *>(tile + (4 * t + e) * KVc);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          pk = fma4x(kr[e], x[e], pk);
+          pq = fma4x(qr[e], x[e], pq);
+        }
+      }
+      *reinterpret_cast<float4 *>(&part[(gw * 2 + 0) * 128 + 4 * lane]) = pk;
+      *reinterpret_cast<float4 *>(&part[(gw * 2 + 1) * 128 + 4 * lane]) = pq;
+    }
+    if (!fold) {  // the fold reads both half-tiles again
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&empty[sl0]);
+        mbar_arrive(&empty[sl1]);
+      }
+    }
+    bar_sync(gbar, kG);
+    // ---- column c: u and the output (one pass over the older records)
+    {
+      const int c = gt;
+      float z = 0.f, zq = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        z += part[(w * 2 + 0) * 128 + c];
+        zq += part[(w * 2 + 1) * 128 + c];
+      }
+      float su0 = 0.f, su1 = 0.f, so0 = 0.f, so1 = 0.f;
+      int j = 0;
+      for (; j + 1 < last; j += 2) {
+        const float u0 = rU[j * KVc + c], u1 = rU[(j + 1) * KVc + c];
+        su0 = fmaf(G[j], u0, su0);
+        so0 = fmaf(KQ[j], u0, so0);
+        su1 = fmaf(G[j + 1], u1, su1);
+        so1 = fmaf(KQ[j + 1], u1, so1);
+      }
+      if (j < last) {
+        const float u0 = rU[j * KVc + c];
+        su0 = fmaf(G[j], u0, su0);
+        so0 = fmaf(KQ[j], u0, so0);
+      }
+      const float u = beta * ((vs[c] - z) - (su0 + su1));
+      const float o = fmaf(KQ[last], u, zq + (so0 + so1));
+      if (!fold) p.ubuf[(bh * p.cap + last) * KVc + c] = u;
+      else ucur[c] = u;
+      p.y[b * p.bs_y + (size_t)h * KVc + c] = p.scale * o;
+    }
+    // ---- fold: h0[r] <- Gamma[r] h0[r] + sum_i w_i[r] u_i over this warp's
+    // rows 32gw.. (its half-tile's slot is still held), written once
+    if (fold) {
+      bar_sync(gbar, kG);  // every column's u
+      const float *tile = reinterpret_cast<const float *>(ring + sl * kKHalfBytes) +
+                          (size_t)(32 * (gw & 1)) * KVc + 4 * lane;
+      float *dst = p.h0 + bh * (KDc * KVc) + (size_t)(32 * gw) * KVc + 4 * lane;
+#pragma unroll 1
+      for (int r0 = 0; r0 < 32; r0 += 8) {
+        float4 acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          acc[e] = mul4x(gamv[32 * gw + r0 + e], *reinterpret_cast<const float4 *>(tile + (r0 + e) * KVc));
+        for (int i = 0; i <= last; ++i) {
+          const float4 ui = *reinterpret_cast<const float4 *>(i < last ? &rU[i * KVc + 4 * lane]
+                                                                        : &ucur[4 * lane]);
+          const float4 wa = *reinterpret_cast<const float4 *>(&rW[i * KDc + 32 * gw + r0]);
+          const float4 wb = *reinterpret_cast<const float4 *>(&rW[i * KDc + 32 * gw + r0 + 4]);
+          const float wr[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] = fma4x(wr[e], ui, acc[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) st_stream(dst + (size_t)(r0 + e) * KVc, acc[e]);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&empty[sl0]);
+        mbar_arrive(&empty[sl1]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&rempty[rb]);
+    if (gt == 0) p.len[bh] = fold ? 0 : k;
+  }
+}
+
+int kda_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n > 0 ? n : 148;
+}
+
+// The persistent decode step when its layout fits (window <= 16), else none.
+template <typename TI>
+bool kda_launch_persistent(const GDNParams &p, cudaStream_t s, cudaError_t &err) {
+  const KdaLayout lay = KdaLayout::make(p.L, (int)sizeof(TI), 227 * 1024);
+  if (lay.NR < 2 || p.L > 16) return false;
+  err = cudaFuncSetAttribute(kda_decode2_kernel<TI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             lay.total);
+  if (err != cudaSuccess) return true;
+  const int nitems = p.B * p.H;
+  const int grid = nitems < kda_sm_count() ? nitems : kda_sm_count();
+  kda_decode2_kernel<TI><<<grid, kThreads + 64, lay.total, s>>>(p, lay);
+  err = cudaGetLastError();
+  return true;
+}
+
 template <typename TI, int MODE>
 cudaError_t kda_launch_mode(const GDNParams &p, cudaStream_t s) {
   const size_t smem = sizeof(KdaSmem);
@@ -323,7 +757,13 @@ cudaError_t kda_launch_dt(const GDNParams &p, cudaStream_t s) {
 cudaError_t kda_launch(const GDNParams &p, int mode, cudaStream_t s) {
   if (p.B * p.H == 0) return cudaSuccess;
   switch (mode) {
-    case 0: return kda_launch_dt<kKdaDecode>(p, s);
+    case 0: {
+      cudaError_t e = cudaSuccess;
+      if (p.kda && (p.in_bf16 ? kda_launch_persistent<__nv_bfloat16>(p, s, e)
+                              : kda_launch_persistent<float>(p, s, e)))
+        return e;
+      return kda_launch_dt<kKdaDecode>(p, s);
+    }
     case 1: return kda_launch_dt<kKdaFlush>(p, s);
     case 2: return kda_launch_dt<kKdaMaterialize>(p, s);
     case 3: return kda_launch_dt<kKdaFull>(p, s);

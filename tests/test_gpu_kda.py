@@ -90,3 +90,33 @@ def test_kda_full_batch_sampled():
     orc, o, lt = _orc_decode(ws, S0s, sts)
     assert per_step_rel_err(got["y"][:, seqs], o) < TOL
     assert rel_err(_gpu.f64(got["state"].h0[seqs]), orc.h0) < TOL
+
+
+def test_kda_bad_buffer_length_sets_status():
+    """A corrupted length is caught on the device: RSSM_ERR_STATE in the status
+    word, the affected items untouched, every other item decoded as usual.
+    320 items on at most 148 CTAs: items of both consumer groups of CTA 0
+    (items 0 and 148) are hit."""
+    w, S0, st = _draw(1, B=10, H=32)
+    layer = _gpu.layer_for(w)
+    state = rs.ReplayState(layer)
+    rs.replayssm_init(layer, state, S0.cuda())
+    bad = [(0, 0), (148 // 32, 148 % 32), (7, 5)]
+    for b, h in bad:
+        state.len[b, h] = 16  # a full buffer on entry: invalid for a decode step
+    h0_before = state.h0.clone()
+    dev = _gpu.to_dev(st)
+    o = torch.zeros(w.B, w.H, w.P, device="cuda")
+    rs.replayssm_decode_step(layer, state, {k: dev[k][0] for k in ("q", "k", "v", "alpha", "beta")}, o)
+    torch.cuda.synchronize()
+    assert state.status() == 9
+    assert torch.equal(state.h0, h0_before)  # a first step folds nothing
+    _, oo, _ = _orc_decode(w, S0, {k: v[:1] for k, v in st.items()})
+    got = o.cpu().numpy().astype(np.float64)
+    good = np.ones((w.B, w.H), dtype=bool)
+    for b, h in bad:
+        good[b, h] = False
+        assert int(state.len[b, h]) == 16
+        assert np.all(got[b, h] == 0)
+    assert np.all(state.len.cpu().numpy()[good] == 1)
+    assert rel_err(got[good], oo[0][good]) < TOL

@@ -86,6 +86,32 @@ def test_gdn_decode_wait_runs_out_then_recovers():
     assert per_step_rel_err(og.cpu().numpy(), oo) < TOL
 
 
+def test_kda_decode_wait_runs_out_then_recovers():
+    w = wl.make("kda_serving", B=1, H=1)  # one (sequence, head) work item
+    g = wl.Generator(w)
+    S0 = g.initial_state()
+    st = g.steps(20)
+    layer = _gpu.layer_for(w)
+    state = rs.ReplayState(layer)
+    rs.replayssm_init(layer, state, S0.cuda())
+    dev = _gpu.to_dev(st)
+    o = torch.zeros(w.B, w.H, w.P, device="cuda")
+    inp = lambda t: {k: dev[k][t] for k in ("q", "k", "v", "alpha", "beta")}
+    _withheld_launch(lambda: rs.replayssm_decode_step(layer, state, inp(0), o))
+    assert state.status() == 7
+    assert int(state.len.abs().sum()) == 0 and torch.equal(state.h0.cpu(), S0)
+    state.clear_status()
+    og = torch.empty(20, w.B, w.H, w.P, device="cuda")
+    for t in range(20):
+        rs.replayssm_decode_step(layer, state, inp(t), og[t])
+    torch.cuda.synchronize()
+    assert state.status() == 0
+    orc = oracle.KDAReplay(S0, L=w.L)
+    oo, _, _ = orc.decode(st["q"], st["k"], st["v"], st["alpha"], st["beta"])
+    assert np.array_equal(state.len.cpu().numpy(), orc.len)
+    assert per_step_rel_err(og.cpu().numpy(), oo) < TOL
+
+
 def test_m2_verify_wait_runs_out_then_recovers():
     w = wl.make("m2_verify", B=1, H=8, G=1)
     g = wl.Generator(w)

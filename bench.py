@@ -67,7 +67,7 @@ KERNEL_SOURCES = {
                                     "codec.cuh", "internal.h", "umma.cuh"),
     "gdn_decode2_kernel_gdn_serving": ("gdn.cu", "common.cuh", "pipeline.cuh", "internal.h",
                                       "umma.cuh"),
-    "kda_kernel_kda_serving": ("kda.cu", "common.cuh", "internal.h"),
+    "kda_decode2_kernel_kda_serving": ("kda.cu", "common.cuh", "internal.h", "pipeline.cuh"),
     "m2_verify_kernel_m2_verify": ("m2_verify.cu", "m2_device.cuh", "common.cuh", "pipeline.cuh",
                                    "codec.cuh", "internal.h"),
     "gdn_verify_kernel_gdn_verify": ("gdn.cu", "common.cuh", "pipeline.cuh", "internal.h",
@@ -574,8 +574,8 @@ def bench_kda(args, dev, peak, rs, bm, wl, torch):
     return {"workload": "kda_serving", "value": tok / (ms_r * 1e-3), "unit": "tokens/s",
             "ms_per_window": ms_r / n,
             "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
-                         "frac": ach_r / peak, "kernel": "kda_kernel<decode>",
-                         "traffic": recorded_traffic("kda_kernel_kda_serving", w.B, 256),
+                         "frac": ach_r / peak, "kernel": "kda_decode2_kernel",
+                         "traffic": recorded_traffic("kda_decode2_kernel_kda_serving", w.B, 256),
                          "algorithmic_bytes_per_launch": wb / L},
             "full_state": {"value": tok / (ms_f * 1e-3), "unit": "tokens/s",
                            "achieved_gbs": ach_f, "frac": ach_f / peak,

@@ -25,8 +25,10 @@
 // algebra with one record and the state written back; it also serves as the
 // conventional step of Gated DeltaNet (a scalar decay is the all-equal case).
 //
-// One CTA of 256 threads per (sequence, head); lane l of warp w holds rows
-// 16w..16w+15 and columns 4l..4l+3 of the 128 x 128 tile in registers.  The
+// kda_kernel: one CTA of 256 threads per (sequence, head); lane l of warp w
+// holds rows 16w..16w+15 and columns 4l..4l+3 of the 128 x 128 tile in
+// registers (conventional step, standalone folds).  kda_decode2_kernel: the
+// persistent replay decode step with two consumer groups (below).  The
 // per-channel decay products are taken in fp64 (one thread per channel).
 #include "common.cuh"
 #include "internal.h"

@@ -1442,8 +1442,504 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_verify_kernel(const GDNParams
   if (tid == 0) p.len[bh] = nb;
 }
 
+// Persistent verify round with two consumer groups on alternate items, on the
+// structure of gdn_decode2_kernel: warp 8 streams each item's checkpoint as
+// two half-tiles into a ring of exactly 4 slots, warp 9 stages the item (the
+// draft inputs, the committed alphas) and bulk-copies its committed keys and
+// corrections into record buffer it % 4 (two per group, so the next item of a
+// group is staged while it works on this one).  Per item, in a group of 4 warps:
+//   * warp 0: fold factors (prefix products of the committed alphas); warp 1:
+//     the draft sequence's factors R(e, j) = Q_e / Q_j; 4 threads per key dot
+//     (k_j . k_e and k_i . q_d, fp32 products, fp64 sums);
+//   * commit fold (n1 reaches the window): warp w folds its 32 rows in its
+//     slot, writes them to h0 and leaves them in the slot for the products;
+//   * warp w: partial h^T k_d, then h^T q_d, over its 32 rows (two passes
+//     through one partial-sum buffer);
+//   * thread c: the drafts in order, u_e and o_d of column c (the earlier
+//     drafts' corrections of column c stay in its registers), then the
+//     drafts are appended.
+struct GdnV2Layout {
+  int L, off_bars, off_rec, rec_bytes, off_scr, scr_bytes, off_ring, total;
+  // record buffer: Kc [20][128] (input dtype) | Uc [20][128] | Qd, Kd, Vd [4][128]
+  // (input dtype) | af [20 -> 32] | ad, bd [4] | hdr [8]
+  int o_uc, o_qd, o_kd, o_vd, o_af, o_ad, o_bd, o_hdr;
+  // group scratch: part [4][4][128] | G, KQ, R [4][24] | gam [4] | Rf [20 -> 32] | gf
+  int s_part, s_g, s_kq, s_r, s_gam, s_rf, s_gf;
+  __host__ static int a128(int v) { return (v + 127) & ~127; }
+  __host__ static GdnV2Layout make(int L, int es, int budget) {
+    GdnV2Layout d;
+    d.L = L;
+    int o = 0;
+    d.o_uc = a128(kMaxRec * DKc * es);
+    d.o_qd = d.o_uc + kMaxRec * DVc * 4;
+    d.o_kd = d.o_qd + kVD * DKc * es;
+    d.o_vd = d.o_kd + kVD * DKc * es;
+    d.o_af = d.o_vd + kVD * DVc * es;
+    d.o_ad = d.o_af + 32 * 4;
+    d.o_bd = d.o_ad + kVD * 4;
+    d.o_hdr = d.o_bd + kVD * 4;
+    d.rec_bytes = a128(d.o_hdr + 8 * 4);
+    d.s_part = 0;
+    d.s_g = 4 * kVD * DVc * 4;
+    d.s_kq = d.s_g + kVD * kVSeq * 4;
+    d.s_r = d.s_kq + kVD * kVSeq * 4;
+    d.s_gam = d.s_r + kVD * kVSeq * 4;
+    d.s_rf = d.s_gam + kVD * 4;
+    d.s_gf = d.s_rf + 32 * 4;
+    d.scr_bytes = a128(d.s_gf + 4 * 4);
+    d.off_bars = o;
+    o += a128(8 * (2 * 8 + 2 * 4));
+    d.off_rec = o;
+    o += 4 * d.rec_bytes;
+    d.off_scr = o;
+    o += 2 * d.scr_bytes;
+    d.off_ring = o;
+    d.total = o + 4 * kHalfBytes;
+    if (d.total > budget) d.total = 0;
+    return d;
+  }
+};
+
+// Four consecutive shared-memory elements (8-byte aligned for bf16, 16 for
+// fp32) as fp32.
+template <typename T>
+__device__ __forceinline__ float4 ld4_smem(const T *p) {
+  if constexpr (sizeof(T) == 4) {
+    return *reinterpret_cast<const float4 *>(p);
+  } else {
+    const uint2 raw = *reinterpret_cast<const uint2 *>(p);
+    const T *e = reinterpret_cast<const T *>(&raw);
+    return make_float4(to_f32(e[0]), to_f32(e[1]), to_f32(e[2]), to_f32(e[3]));
+  }
+}
+
+template <typename TI>
+__global__ void __launch_bounds__(kThreads + 64, 1) gdn_verify2_kernel(const GDNParams p,
+                                                                    const GdnV2Layout lay) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int abort_word;
+  volatile int *abort_flag = &abort_word;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.off_bars);
+  uint64_t *empty = full + 8, *rfull = empty + 8, *rempty = rfull + 4;
+  unsigned char *ring = smem + lay.off_ring;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nitems = p.B * p.H;
+  const int L = lay.L, nd = p.n_draft;
+
+  if (tid == 0) {
+    for (int s = 0; s < 8; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4);  // the 4 warps of the group that owns the slot
+    }
+    for (int r = 0; r < 4; ++r) {
+      mbar_init(&rfull[r], 1);
+      mbar_init(&rempty[r], 4);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == 8) {  // tile producer: half-tiles in (item, half) order, 4 slots
+    if (lane != 0) return;
+    int slot = 0;
+    uint32_t sphase = 0, issued = 0, parity = 0;
+    bool failed = false;
+    for (int item = blockIdx.x; item < nitems && !failed; item += gridDim.x) {
+      for (int half = 0; half < 2; ++half) {
+        if (*abort_flag || !mbar_wait(&empty[slot], sphase ^ 1, kWaitLimitNs, abort_flag) ||
+            *abort_flag) {
+          failed = true;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[slot], kHalfBytes);
+        bulk_g2s(ring + slot * kHalfBytes,
+                 p.h0 + (size_t)item * DKc * DVc + (size_t)half * kHalfRows * DVc, kHalfBytes,
+                 &full[slot]);
+        issued |= 1u << slot;
+        parity = (parity & ~(1u << slot)) | (sphase << slot);
+        if (++slot == 4) {
+          slot = 0;
+          sphase ^= 1;
+        }
+      }
+    }
+    if (failed) {
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    for (int s2 = 0; s2 < 4; ++s2)  // every copy issued here lands before the warp returns
+      if (issued & (1u << s2)) mbar_wait(&full[s2], (parity >> s2) & 1u);
+    return;
+  }
+
+  if (warp == 9) {  // stager: the item's loads first, then shared-memory writes and copies
+    int it = 0;
+    ArmedRecords armed;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+      const bool abort_now = __any_sync(0xffffffffu, *abort_flag != 0);
+      if (!abort_now && item == p.hold_item) continue;  // test hook: never staged
+      const int rb = it & 3;
+      bool ok = !abort_now;
+      if (ok && lane == 0)
+        ok = mbar_wait(&rempty[rb], ((it >> 2) & 1) ^ 1, kWaitLimitNs, abort_flag) && !*abort_flag;
+      if (!__shfl_sync(0xffffffffu, (int)ok, 0)) {
+        if (lane == 0 && !*abort_flag) {
+          report(p.status, RSSM_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      const int b = item / p.H, h = item - (item / p.H) * p.H;
+      const size_t bh = (size_t)item;
+      const int n0 = __ldcg(&p.len[bh]);
+      const int a = p.acc ? __ldcg(&p.acc[b]) : 0;
+      const int n1 = n0 + a, fold = n1 >= L, nb = fold ? 0 : n1;
+      const int bad = n0 < 0 || n0 >= L || a < 0 || a > p.draft_max || n1 > p.cap ||
+                      nb + nd > p.cap;
+      const int n1c = min(max(n1, 0), p.cap);  // copies stay in this item's slots even when bad
+      const float af = lane < n1c ? __ldcg(&p.abuf[bh * p.cap + lane]) : 0.f;
+      TI qv[kVD][4], kv[kVD][4], vv[kVD][4];
+      float adv = 0.f, bdv = 0.f;
+#pragma unroll
+      for (int d = 0; d < kVD; ++d) {
+        if (d < nd) {
+          const int64_t o = (int64_t)(d * p.H + h) * DKc;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            qv[d][u] = static_cast<const TI *>(p.q)[b * p.bs_q + o + lane + 32 * u];
+            kv[d][u] = static_cast<const TI *>(p.k)[b * p.bs_k + o + lane + 32 * u];
+            vv[d][u] = static_cast<const TI *>(p.v)[b * p.bs_v + (int64_t)(d * p.H + h) * DVc + lane + 32 * u];
+          }
+        }
+      }
+      if (lane < nd) {
+        adv = p.alpha[b * p.bs_a + lane * p.H + h];
+        bdv = p.beta[b * p.bs_b + lane * p.H + h];
+      }
+      unsigned char *rec = smem + lay.off_rec + rb * lay.rec_bytes;
+      TI *Qd = reinterpret_cast<TI *>(rec + lay.o_qd), *Kd = reinterpret_cast<TI *>(rec + lay.o_kd);
+      TI *Vd = reinterpret_cast<TI *>(rec + lay.o_vd);
+#pragma unroll
+      for (int d = 0; d < kVD; ++d) {
+        if (d < nd) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            Qd[d * DKc + lane + 32 * u] = qv[d][u];
+            Kd[d * DKc + lane + 32 * u] = kv[d][u];
+            Vd[d * DVc + lane + 32 * u] = vv[d][u];
+          }
+        }
+      }
+      reinterpret_cast<float *>(rec + lay.o_af)[lane] = af;
+      if (lane < kVD) {
+        reinterpret_cast<float *>(rec + lay.o_ad)[lane] = adv;
+        reinterpret_cast<float *>(rec + lay.o_bd)[lane] = bdv;
+      }
+      if (lane == 0) {
+        int *hdr = reinterpret_cast<int *>(rec + lay.o_hdr);
+        hdr[0] = n1;
+        hdr[1] = nb;
+        hdr[2] = fold;
+        hdr[3] = bad;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t bK = n1c * DKc * sizeof(TI), bU = n1c * DVc * 4;
+        mbar_arrive_expect_tx(&rfull[rb], bK + bU);
+        if (n1c > 0) {
+          bulk_g2s(rec, static_cast<const TI *>(p.kbuf) + bh * p.cap * DKc, bK, &rfull[rb]);
+          bulk_g2s(rec + lay.o_uc, p.ubuf + bh * p.cap * DVc, bU, &rfull[rb]);
+        }
+      }
+      armed.arm(rb, (it >> 2) & 1);
+    }
+    if (lane == 0) armed.drain(rfull, 4);  // no record copy outlives the warp
+    __syncwarp();
+    return;
+  }
+
+  // Consumer group grp (warps 4grp .. 4grp+3), thread gt = column c.
+  constexpr int kG = 128;
+  const int grp = warp >> 2, gw = warp & 3, gt = tid & (kG - 1);
+  const uint32_t gbar = 1 + grp;
+  unsigned char *scr = smem + lay.off_scr + grp * lay.scr_bytes;
+  float *part = reinterpret_cast<float *>(scr + lay.s_part);
+  float *G = reinterpret_cast<float *>(scr + lay.s_g), *KQ = reinterpret_cast<float *>(scr + lay.s_kq);
+  float *Rd = reinterpret_cast<float *>(scr + lay.s_r), *gam = reinterpret_cast<float *>(scr + lay.s_gam);
+  float *Rf = reinterpret_cast<float *>(scr + lay.s_rf), *gf = reinterpret_cast<float *>(scr + lay.s_gf);
+  int it = grp;
+  for (int item = blockIdx.x + grp * gridDim.x; item < nitems; item += 2 * gridDim.x, it += 2) {
+    const int rb = it & 3;  // this group's buffers: grp and grp + 2
+    const unsigned char *rec = smem + lay.off_rec + rb * lay.rec_bytes;
+    const TI *Kc = reinterpret_cast<const TI *>(rec);
+    const float *Uc = reinterpret_cast<const float *>(rec + lay.o_uc);
+    const TI *Qd = reinterpret_cast<const TI *>(rec + lay.o_qd);
+    const TI *Kd = reinterpret_cast<const TI *>(rec + lay.o_kd);
+    const TI *Vd = reinterpret_cast<const TI *>(rec + lay.o_vd);
+    const float *afs = reinterpret_cast<const float *>(rec + lay.o_af);
+    const float *ads = reinterpret_cast<const float *>(rec + lay.o_ad);
+    const float *bds = reinterpret_cast<const float *>(rec + lay.o_bd);
+    const int *hdr = reinterpret_cast<const int *>(rec + lay.o_hdr);
+    const int b = item / p.H, h = item - (item / p.H) * p.H;
+    const size_t bh = (size_t)item;
+    const int sl0 = 2 * (it & 1), sl1 = sl0 + 1;
+    const uint32_t tphase = (it >> 1) & 1;
+    const int half = gw >> 1, sl = half ? sl1 : sl0;
+
+    const bool got = mbar_wait(&rfull[rb], (it >> 2) & 1, p.wait_ns, abort_flag);
+    if (!got) {
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    if (bar_or(gbar, kG, !got || *abort_flag)) break;
+    if (hdr[3]) {
+      if (gt == 0) report(p.status, RSSM_ERR_STATE);
+      if (!mbar_wait(&full[sl], tphase, p.wait_ns, abort_flag)) {
+        if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&empty[sl0]);
+        mbar_arrive(&empty[sl1]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rempty[rb]);
+      continue;
+    }
+    const int n1 = hdr[0], nb = hdr[1], ne = nb + nd;  // draft sequence: records 0..ne-1
+    const bool fold = hdr[2];
+
+    // ---- decay factors (warps 0, 1) and key dots (4 threads per dot)
+    if (gw == 0) {  // fold: R_i = prod_{i<m<n1} alpha_m, gamma = prod_{m<n1} alpha_m
+      double pr = lane < n1 ? (double)afs[lane] : 1.0;  // inclusive prefix product
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_up_sync(0xffffffffu, pr, o);
+        if (lane >= o) pr *= t;
+      }
+      const double lastp = __shfl_sync(0xffffffffu, pr, (n1 > 0 ? n1 : 1) - 1);
+      if (fold && lane < n1) Rf[lane] = (float)(lastp / pr);
+      if (lane == 0) gf[0] = (float)lastp;
+    } else if (gw == 1) {  // drafts: Q_m over the draft sequence, R(e,j) = Q_e / Q_j
+      const float am = lane < nb ? afs[lane] : (lane < ne ? ads[lane - nb] : 1.f);
+      double pr = am;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_up_sync(0xffffffffu, pr, o);
+        if (lane >= o) pr *= t;
+      }
+#pragma unroll
+      for (int d = 0; d < kVD; ++d) {
+        const double qe = __shfl_sync(0xffffffffu, pr, (nb + d) & 31);
+        if (d < nd) {
+          if (lane <= nb + d) Rd[d * kVSeq + lane] = (float)(qe / pr);
+          if (lane == 0) gam[d] = (float)qe;
+        }
+      }
+    }
+    {
+      // dots: (d, j < e_d) keys . k_d, then (d, i <= e_d) keys . q_d
+      const int nkk = nd * nb + nd * (nd - 1) / 2, nkq = nd * nb + nd * (nd + 1) / 2;
+      const int ndot = nkk + nkq;
+      for (int base = 0; base < ndot; base += kG / 4) {
+        const int t = base + (gt >> 2), j4 = gt & 3;
+        double acc = 0.0, acc1 = 0.0;
+        int d = 0, j = 0;
+        bool isq = false;
+        if (t < ndot) {
+          int r = t < nkk ? t : t - nkk;
+          isq = t >= nkk;
+          // enumerate (d, j): draft d has nb + d (keys) or nb + d + 1 (queries) partners
+          for (d = 0; d < nd; ++d) {
+            const int cnt = nb + d + (isq ? 1 : 0);
+            if (r < cnt) break;
+            r -= cnt;
+          }
+          j = r;
+          const TI *other = isq ? Qd + d * DKc : Kd + d * DKc;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int c0 = 8 * (j4 + 4 * m);
+            float kv[8], ov[8];
+            if (j < nb) ld8_smem(Kc + j * DKc + c0, kv);
+            else ld8_smem(Kd + (j - nb) * DKc + c0, kv);
+            ld8_smem(other + c0, ov);
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              acc += (double)(kv[e] * ov[e]);
+              acc1 += (double)(kv[e + 1] * ov[e + 1]);
+            }
+          }
+          acc += acc1;
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        if (t < ndot && j4 == 0) {
+          if (isq) KQ[d * kVSeq + j] = (float)acc;
+          else G[d * kVSeq + j] = (float)acc;
+        }
+      }
+    }
+    bar_sync(gbar, kG);
+
+    // ---- this warp's 32 rows: commit fold in the slot, then partial products
+    if (!mbar_wait(&full[sl], tphase, p.wait_ns, abort_flag)) {
+      if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    float *tile = reinterpret_cast<float *>(ring + sl * kHalfBytes) +
+                  (size_t)(32 * (gw & 1)) * DVc + 4 * lane;
+    const int row0 = 32 * gw;
+    if (fold) {  // h <- gamma h0 + sum_i R_i k_i u_i^T, written to h0 and to the slot
+      const float g = gf[0];
+      float *dst = p.h0 + bh * (DKc * DVc) + (size_t)row0 * DVc + 4 * lane;
+#pragma unroll 1
+      for (int r0 = 0; r0 < 32; r0 += 8) {
+        float4 acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = mul4x(g, *reinterpret_cast<const float4 *>(tile + (r0 + e) * DVc));
+        for (int i = 0; i < n1; ++i) {
+          const float4 ui = *reinterpret_cast<const float4 *>(&Uc[i * DVc + 4 * lane]);
+          const float ri = Rf[i];
+          float kr[8];
+          ld8_smem(Kc + i * DKc + row0 + r0, kr);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] = fma4x(ri * kr[e], ui, acc[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          *reinterpret_cast<float4 *>(tile + (r0 + e) * DVc) = acc[e];
+          st_stream(dst + (size_t)(r0 + e) * DVc, acc[e]);
+        }
+      }
+      __syncwarp();
+    }
+    // two passes through the partial-sum buffer: h^T k_d, then h^T q_d;
+    // thread c keeps the column sums in registers
+    float zk[kVD], zq[kVD];
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+      const TI *vecs = pass ? Qd : Kd;
+      float4 pa[kVD];
+#pragma unroll
+      for (int v = 0; v < kVD; ++v) pa[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+      for (int t = 0; t < 8; ++t) {
+        float4 x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = *reinterpret_cast<const float4 *>(tile + (4 * t + e) * DVc);
+#pragma unroll
+        for (int v = 0; v < kVD; ++v) {
+          if (v < nd) {
+            const float4 w4 = ld4_smem(vecs + v * DKc + row0 + 4 * t);
+            pa[v] = fma4x(w4.x, x[0], pa[v]);
+            pa[v] = fma4x(w4.y, x[1], pa[v]);
+            pa[v] = fma4x(w4.z, x[2], pa[v]);
+            pa[v] = fma4x(w4.w, x[3], pa[v]);
+          }
+        }
+      }
+      if (pass) bar_sync(gbar, kG);  // the first pass's sums have been read
+#pragma unroll
+      for (int v = 0; v < kVD; ++v)
+        *reinterpret_cast<float4 *>(&part[(gw * kVD + v) * DVc + 4 * lane]) = pa[v];
+      bar_sync(gbar, kG);
+#pragma unroll
+      for (int d = 0; d < kVD; ++d) {
+        float zs = 0.f;
+        if (d < nd) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) zs += part[(w * kVD + d) * DVc + gt];
+        }
+        if (pass) zq[d] = zs;
+        else zk[d] = zs;
+      }
+    }
+    fence_proxy_async_smem();  // the fold's slot writes before the slot's next bulk copy
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&empty[sl0]);
+      mbar_arrive(&empty[sl1]);
+    }
+
+    // ---- column c: the drafts in order (each needs the earlier ones' u)
+    {
+      const int c = gt;
+      float su[kVD], so[kVD], ud[kVD];
+#pragma unroll
+      for (int d = 0; d < kVD; ++d) su[d] = so[d] = ud[d] = 0.f;
+      // the committed records' terms, one load of u_j for every draft
+      for (int j = 0; j < nb; ++j) {
+        const float uj = Uc[j * DVc + c];
+#pragma unroll
+        for (int d = 0; d < kVD; ++d) {
+          if (d < nd) {
+            const float rj = Rd[d * kVSeq + j];
+            su[d] = fmaf(-rj * G[d * kVSeq + j], uj, su[d]);
+            so[d] = fmaf(rj * KQ[d * kVSeq + j], uj, so[d]);
+          }
+        }
+      }
+#pragma unroll
+      for (int d = 0; d < kVD; ++d) {
+        if (d < nd) {
+          const int e = nb + d;
+          float a0 = to_f32(Vd[d * DVc + c]) - gam[d] * zk[d] + su[d];
+#pragma unroll
+          for (int q = 0; q < kVD; ++q)  // earlier drafts' records
+            if (q < d) a0 = fmaf(-Rd[d * kVSeq + nb + q] * G[d * kVSeq + nb + q], ud[q], a0);
+          const float u = bds[d] * a0;
+          ud[d] = u;
+          float o0 = gam[d] * zq[d] + so[d];
+#pragma unroll
+          for (int q = 0; q < kVD; ++q)
+            if (q <= d) o0 = fmaf(Rd[d * kVSeq + nb + q] * KQ[d * kVSeq + nb + q], ud[q], o0);
+          p.ubuf[(bh * p.cap + e) * DVc + c] = u;
+          p.y[b * p.bs_y + (size_t)(d * p.H + h) * DVc + c] = p.scale * o0;
+        }
+      }
+      // ---- append the drafts at slots nb .. nb+nd-1 (their staged input values)
+#pragma unroll
+      for (int d = 0; d < kVD; ++d) {
+        if (d < nd) {
+          const size_t slot = bh * p.cap + nb + d;
+          static_cast<TI *>(p.qbuf)[slot * DKc + c] = Qd[d * DKc + c];
+          static_cast<TI *>(p.kbuf)[slot * DKc + c] = Kd[d * DKc + c];
+          static_cast<TI *>(p.vbuf)[slot * DVc + c] = Vd[d * DVc + c];
+        }
+      }
+      if (c < nd) {
+        p.abuf[bh * p.cap + nb + c] = ads[c];
+        p.bbuf[bh * p.cap + nb + c] = bds[c];
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&rempty[rb]);
+    if (gt == 0) p.len[bh] = nb;
+  }
+}
+
+int gdn_sm_count();
+
 template <typename TI>
 cudaError_t gdn_verify_launch(const GDNParams &p, cudaStream_t s) {
+  if (p.L <= 16) {  // two consumer groups when their layout fits
+    const GdnV2Layout lay = GdnV2Layout::make(p.L, (int)sizeof(TI), 227 * 1024);
+    if (lay.total > 0) {
+      cudaError_t e = cudaFuncSetAttribute(gdn_verify2_kernel<TI>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+      if (e != cudaSuccess) return e;
+      const int nitems = p.B * p.H;
+      const int grid = nitems < gdn_sm_count() ? nitems : gdn_sm_count();
+      gdn_verify2_kernel<TI><<<grid, kThreads + 64, lay.total, s>>>(p, lay);
+      return cudaGetLastError();
+    }
+  }
   const size_t smem = sizeof(GdnVerifySmem);
   cudaError_t e = cudaFuncSetAttribute(gdn_verify_kernel<TI>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

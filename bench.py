@@ -70,7 +70,7 @@ KERNEL_SOURCES = {
     "kda_decode2_kernel_kda_serving": ("kda.cu", "common.cuh", "internal.h", "pipeline.cuh"),
     "m2_verify_kernel_m2_verify": ("m2_verify.cu", "m2_device.cuh", "common.cuh", "pipeline.cuh",
                                    "codec.cuh", "internal.h"),
-    "gdn_verify_kernel_gdn_verify": ("gdn.cu", "common.cuh", "pipeline.cuh", "internal.h",
+    "gdn_verify2_kernel_gdn_verify": ("gdn.cu", "common.cuh", "pipeline.cuh", "internal.h",
                                      "umma.cuh"),
 }
 
@@ -815,8 +815,8 @@ def bench_verify_gdn(args, dev, peak, rs, bm, wl, torch):
             "ms_per_round": ms_r / n,
             "drafts_evaluated_per_s": w.B * w.n_draft * n / (ms_r * 1e-3),
             "roofline": {"bound": "hbm", "achieved": ach_r, "peak": peak, "unit": "GB/s",
-                         "frac": ach_r / peak, "kernel": "gdn_verify_kernel",
-                         "traffic": recorded_traffic("gdn_verify_kernel_gdn_verify", w.B, 256),
+                         "frac": ach_r / peak, "kernel": "gdn_verify2_kernel",
+                         "traffic": recorded_traffic("gdn_verify2_kernel_gdn_verify", w.B, 256),
                          "algorithmic_bytes_per_launch": total / n},
             "snapshot_restore": {"rounds_per_s": n / (ms_s * 1e-3), "ms_per_round": ms_s / n,
                                  "achieved_gbs": ach_s, "frac": ach_s / peak,

@@ -153,3 +153,32 @@ def test_gdn_verify_bad_acceptance_sets_status():
     rs.replayssm_verify_commit(layer, state, bad, drafts, y)
     assert state.status() == 9
     assert int(state.len[0, 0]) == 0 and int(state.len[1, 0]) == 1
+
+
+@pytest.mark.parametrize("dmax,nd", [(1, 1), (3, 2), (4, 3)])
+def test_gdn_verify_fewer_drafts(dmax, nd):
+    """Rounds of 1-3 drafts, with draft_max (and so the buffer capacity) both
+    equal to and above the round's count."""
+    w, S0, rd = _draw(12, B=3, H=4)
+    rd = {k: (v[:, :, :nd].contiguous() if k != "acc" else v.clamp(max=nd)) for k, v in rd.items()}
+    layer = _gpu.layer_for(w, draft_max=dmax)
+    state = rs.ReplayState(layer)
+    rs.replayssm_init(layer, state, S0.cuda())
+    dev = _gpu.to_dev(rd)
+    R = rd["q"].shape[0]
+    y = torch.empty(R, w.B, nd, w.H, w.P, device="cuda")
+    lens = []
+    for r in range(R):
+        drafts = {k: dev[k][r] for k in ("q", "k", "v", "alpha", "beta")}
+        rs.replayssm_verify_commit(layer, state, dev["acc"][r - 1] if r else None, drafts, y[r])
+        lens.append(state.len.clone())
+    rs.replayssm_commit(layer, state, dev["acc"][R - 1].contiguous())
+    lens.append(state.len.clone())
+    torch.cuda.synchronize()
+    orc = oracle.GDNReplay(S0, L=w.L, cap=w.L + max(dmax - 1, 0))
+    yo, lt = orc.verify(rd["q"], rd["k"], rd["v"], rd["alpha"], rd["beta"], rd["acc"])
+    yg = y.cpu().numpy()
+    assert state.status() == 0
+    assert np.array_equal(torch.stack(lens).cpu().numpy()[1:], lt)
+    assert per_step_rel_err(_flat(yg), _flat(yo)) < TOL
+    assert rel_err(_gpu.f64(state.h0), orc.h0) < TOL

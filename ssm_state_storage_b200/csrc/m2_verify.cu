@@ -528,7 +528,79 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
       report(p.status, RSSM_ERR_TIMEOUT);
       *abort_flag = 1;
     }
-    for (int j = 0; j < hc; ++j) {
+    bool paired = false;
+    if constexpr (NSP == 1) {
+      if (!fold) {
+        paired = true;
+        // no fold: heads in pairs, so the two heads' dot products and
+        // reductions interleave (independent chains)
+        int rows[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) rows[u] = gw * RW + 2 * u + h16;
+        for (int j = 0; j < hc; j += 2) {
+          const bool two = j + 1 < hc;
+          float4 v[2][2][S4];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            if (hh == 0 || two) {
+              const int jj = j + hh;
+              const uint32_t pos = (uint32_t)it * hc + jj;
+              const int sl = pos % lay.NS;
+              if (!mbar_wait(&full[sl], (pos / lay.NS) & 1, p.wait_ns, abort_flag)) {
+                if (!*abort_flag) report(p.status, RSSM_ERR_TIMEOUT);
+                *abort_flag = 1;
+              }
+              if (jj == hc - 1) pass_turn();
+              const float *tl = reinterpret_cast<const float *>(ring + sl * lay.tile_stride);
+#pragma unroll
+              for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int s4 = 0; s4 < S4; ++s4)
+                  v[hh][u][s4] = *reinterpret_cast<const float4 *>(tl + rows[u] * N + 64 * s4 + 4 * c16);
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&empty[sl]);
+            } else {  // no second head: its (unused) sums run on a copy of the first
+#pragma unroll
+              for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int s4 = 0; s4 < S4; ++s4) v[1][u][s4] = v[0][u][s4];
+            }
+          }
+          float q[2][2 * kMD];  // paired fp32 FMAs over this lane's 4 S4 columns
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+              for (int d = 0; d < kMD; ++d) {
+                float2 a = __fmul2_rn(make_float2(v[hh][u][0].x, v[hh][u][0].y),
+                                      make_float2(cr[d][0].x, cr[d][0].y));
+                a = __ffma2_rn(make_float2(v[hh][u][0].z, v[hh][u][0].w),
+                               make_float2(cr[d][0].z, cr[d][0].w), a);
+#pragma unroll
+                for (int s4 = 1; s4 < S4; ++s4) {
+                  a = __ffma2_rn(make_float2(v[hh][u][s4].x, v[hh][u][s4].y),
+                                 make_float2(cr[d][s4].x, cr[d][s4].y), a);
+                  a = __ffma2_rn(make_float2(v[hh][u][s4].z, v[hh][u][s4].w),
+                                 make_float2(cr[d][s4].z, cr[d][s4].w), a);
+                }
+                q[hh][u * kMD + d] = a.x + a.y;
+              }
+          HalfWarpReduce<2 * kMD, 8>::run(q[0], c16);  // every lane shuffles
+          HalfWarpReduce<2 * kMD, 8>::run(q[1], c16);
+          const int idx = c16 >> 1, u = idx / kMD, d = idx - u * kMD;
+          if ((c16 & 1) == 0 && d < nd) {
+            const int r = rows[u];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+              if (hh == 0 || two)
+                p.y[b * p.bs_y + ((size_t)d * p.H + h_first + j + hh) * P + r] =
+                    fmaf(lamd[d * hc + j + hh], q[hh][0], z[(d * hc + j + hh) * P + r]);
+          }
+        }
+      }
+    }
+    for (int j = 0; j < (paired ? 0 : hc); ++j) {
       const int h = h_first + j;
       const size_t bh = bh0 + j;
       const uint32_t pos = (uint32_t)it * hc + j;

@@ -498,7 +498,49 @@ __global__ void __maxnreg__(96) m2_verify_kernel(const M2Params p, const VerifyL
     // ---- S3 (one warp per (draft, head) row, RZ rows of the head per lane):
     // z[d][j][r] = sum_i c_i x_i[r] + D_j x_d[r], with the coefficient
     // c_i = w_{d,i} (B_i . C_d) rounded once by lane i and broadcast
-    for (int row = gw; row < nd * hc; row += kGWarps) {
+    // When the warp's two rows are the same head's (kGWarps a multiple of hc),
+    // one pass over the records serves both: one load of x_i, two chains.
+    const bool pair_rows = (kGWarps % hc) == 0 && nd * hc <= 2 * kGWarps;
+    if (pair_rows && gw < nd * hc) {
+      const int rowB = gw + kGWarps;
+      const bool hasB = rowB < nd * hc;
+      const int dA = gw / hc, j = gw - dA * hc, dB = dA + kGWarps / hc;
+      const float clA = lane <= nb + dA ? (float)(wd[(dA * hc + j) * R + lane] * bc[dA * R + lane]) : 0.f;
+      const float clB = hasB && lane <= nb + dB
+                            ? (float)(wd[(dB * hc + j) * R + lane] * bc[dB * R + lane]) : 0.f;
+      float accA[RZ], accB[RZ], xv[RZ];
+#pragma unroll
+      for (int k = 0; k < RZ; ++k) accA[k] = accB[k] = 0.f;
+      for (int i = 0; i < nb; ++i) {
+        ld_vec<TI, RZ>(recX + (j * cap + i) * P + RZ * lane, xv);
+        const float ca = __shfl_sync(0xffffffffu, clA, i), cb = __shfl_sync(0xffffffffu, clB, i);
+#pragma unroll
+        for (int k = 0; k < RZ; ++k) {
+          accA[k] = fmaf(ca, xv[k], accA[k]);
+          accB[k] = fmaf(cb, xv[k], accB[k]);
+        }
+      }
+      for (int i = nb; i <= nb + (hasB ? dB : dA); ++i) {
+        ld_vec<TI, RZ>(dX + ((i - nb) * hc + j) * P + RZ * lane, xv);
+        const float ca = __shfl_sync(0xffffffffu, clA, i), cb = __shfl_sync(0xffffffffu, clB, i);
+        if (i <= nb + dA) {
+#pragma unroll
+          for (int k = 0; k < RZ; ++k) accA[k] = fmaf(ca, xv[k], accA[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < RZ; ++k) accB[k] = fmaf(cb, xv[k], accB[k]);
+      }
+      const float Dj = Ds[j];
+      ld_vec<TI, RZ>(dX + (dA * hc + j) * P + RZ * lane, xv);
+#pragma unroll
+      for (int k = 0; k < RZ; ++k) z[(dA * hc + j) * P + RZ * lane + k] = fmaf(Dj, xv[k], accA[k]);
+      if (hasB) {
+        ld_vec<TI, RZ>(dX + (dB * hc + j) * P + RZ * lane, xv);
+#pragma unroll
+        for (int k = 0; k < RZ; ++k) z[(dB * hc + j) * P + RZ * lane + k] = fmaf(Dj, xv[k], accB[k]);
+      }
+    }
+    for (int row = pair_rows ? nd * hc : gw; row < nd * hc; row += kGWarps) {
       const int d = row / hc, j = row - d * hc;
       const float cl = lane <= nb + d ? (float)(wd[(d * hc + j) * R + lane] * bc[d * R + lane]) : 0.f;
       float acc[RZ], xv[RZ];

@@ -182,7 +182,8 @@ const char *replayssm_last_cuda_error(void);
  * withhold_item >= 0 makes the record-staging warp skip that work item, so the
  * compute warps' wait for it runs out (-1: none).  Work items: Mamba-2
  * decode and verify (sequence * G + group) * chunks + chunk, with chunks = 1
- * when a group has at most 8 heads; GDN and KDA decode sequence * H + head.  The
+ * when a group has at most 8 heads; GDN and KDA decode and GDN verify (bf16
+ * inputs) sequence * H + head.  The
  * values apply to every launch made after the call, from any host thread.
  * Returns RSSM_ERR_INVALID_ARG for withhold_item < -1. */
 rssm_status replayssm_set_test_hooks(int64_t consumer_wait_ns, int32_t withhold_item);

@@ -141,3 +141,31 @@ def test_m2_verify_wait_runs_out_then_recovers():
     assert np.array_equal(state.len.cpu().numpy(), orc.len)
     yg = yg.cpu().numpy()
     assert per_step_rel_err(yg.reshape(-1, *yg.shape[3:]), yo.reshape(-1, *yo.shape[3:])) < TOL
+
+
+def test_gdn_verify_wait_runs_out_then_recovers():
+    w = wl.make("gdn_verify", B=1, H=1)  # one (sequence, head) work item
+    g = wl.Generator(w)
+    S0 = g.initial_state()
+    rd = g.rounds(3)
+    layer = _gpu.layer_for(w)
+    state = rs.ReplayState(layer)
+    rs.replayssm_init(layer, state, S0.cuda())
+    dev = _gpu.to_dev(rd)
+    drafts = lambda r: {k: dev[k][r] for k in ("q", "k", "v", "alpha", "beta")}
+    y = torch.zeros(w.B, w.n_draft, w.H, w.P, device="cuda")
+    _withheld_launch(lambda: rs.replayssm_verify_commit(layer, state, None, drafts(0), y))
+    assert state.status() == 7
+    assert int(state.len.abs().sum()) == 0 and torch.equal(state.h0.cpu(), S0)
+    state.clear_status()
+    yg = torch.empty(3, w.B, w.n_draft, w.H, w.P, device="cuda")
+    for r in range(3):
+        rs.replayssm_verify_commit(layer, state, dev["acc"][r - 1] if r else None, drafts(r), yg[r])
+    rs.replayssm_commit(layer, state, dev["acc"][2].contiguous())
+    torch.cuda.synchronize()
+    assert state.status() == 0
+    orc = oracle.GDNReplay(S0, L=w.L, cap=w.L + w.n_draft - 1)
+    yo, lt = orc.verify(rd["q"], rd["k"], rd["v"], rd["alpha"], rd["beta"], rd["acc"])
+    assert np.array_equal(state.len.cpu().numpy(), orc.len)
+    yg = yg.cpu().numpy()
+    assert per_step_rel_err(yg.reshape(-1, *yg.shape[3:]), yo.reshape(-1, *yo.shape[3:])) < TOL

@@ -1453,8 +1453,8 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_verify_kernel(const GDNParams
 //     (k_j . k_e and k_i . q_d, fp32 products, fp64 sums);
 //   * commit fold (n1 reaches the window): warp w folds its 32 rows in its
 //     slot, writes them to h0 and leaves them in the slot for the products;
-//   * warp w: partial h^T k_d, then h^T q_d, over its 32 rows (two passes
-//     through one partial-sum buffer);
+//   * warp w: partial h^T k_d and h^T q_d over its 32 rows in one pass (the
+//     sums go through one partial-sum buffer in two halves);
 //   * thread c: the drafts in order, u_e and o_d of column c (the earlier
 //     drafts' corrections of column c stay in its registers), then the
 //     drafts are appended.
@@ -1818,45 +1818,53 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_verify2_kernel(const GDN
       }
       __syncwarp();
     }
-    // two passes through the partial-sum buffer: h^T k_d, then h^T q_d;
-    // thread c keeps the column sums in registers
+    // one pass over the rows for all 2 nd products; the partial sums go
+    // through one buffer in two halves (h^T k_d, then h^T q_d), thread c
+    // keeping its column's sums in registers
     float zk[kVD], zq[kVD];
+    {
+      float4 pa[2][kVD];
 #pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
-      const TI *vecs = pass ? Qd : Kd;
-      float4 pa[kVD];
+      for (int pass = 0; pass < 2; ++pass)
 #pragma unroll
-      for (int v = 0; v < kVD; ++v) pa[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int v = 0; v < kVD; ++v) pa[pass][v] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
       for (int t = 0; t < 8; ++t) {
         float4 x[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) x[e] = *reinterpret_cast<const float4 *>(tile + (4 * t + e) * DVc);
 #pragma unroll
-        for (int v = 0; v < kVD; ++v) {
-          if (v < nd) {
-            const float4 w4 = ld4_smem(vecs + v * DKc + row0 + 4 * t);
-            pa[v] = fma4x(w4.x, x[0], pa[v]);
-            pa[v] = fma4x(w4.y, x[1], pa[v]);
-            pa[v] = fma4x(w4.z, x[2], pa[v]);
-            pa[v] = fma4x(w4.w, x[3], pa[v]);
+        for (int pass = 0; pass < 2; ++pass) {
+          const TI *vecs = pass ? Qd : Kd;
+#pragma unroll
+          for (int v = 0; v < kVD; ++v) {
+            if (v < nd) {
+              const float4 w4 = ld4_smem(vecs + v * DKc + row0 + 4 * t);
+              pa[pass][v] = fma4x(w4.x, x[0], pa[pass][v]);
+              pa[pass][v] = fma4x(w4.y, x[1], pa[pass][v]);
+              pa[pass][v] = fma4x(w4.z, x[2], pa[pass][v]);
+              pa[pass][v] = fma4x(w4.w, x[3], pa[pass][v]);
+            }
           }
         }
       }
-      if (pass) bar_sync(gbar, kG);  // the first pass's sums have been read
 #pragma unroll
-      for (int v = 0; v < kVD; ++v)
-        *reinterpret_cast<float4 *>(&part[(gw * kVD + v) * DVc + 4 * lane]) = pa[v];
-      bar_sync(gbar, kG);
+      for (int pass = 0; pass < 2; ++pass) {
+        if (pass) bar_sync(gbar, kG);  // the first half's sums have been read
 #pragma unroll
-      for (int d = 0; d < kVD; ++d) {
-        float zs = 0.f;
-        if (d < nd) {
+        for (int v = 0; v < kVD; ++v)
+          *reinterpret_cast<float4 *>(&part[(gw * kVD + v) * DVc + 4 * lane]) = pa[pass][v];
+        bar_sync(gbar, kG);
 #pragma unroll
-          for (int w = 0; w < 4; ++w) zs += part[(w * kVD + d) * DVc + gt];
+        for (int d = 0; d < kVD; ++d) {
+          float zs = 0.f;
+          if (d < nd) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) zs += part[(w * kVD + d) * DVc + gt];
+          }
+          if (pass) zq[d] = zs;
+          else zk[d] = zs;
         }
-        if (pass) zq[d] = zs;
-        else zk[d] = zs;
       }
     }
     fence_proxy_async_smem();  // the fold's slot writes before the slot's next bulk copy

@@ -842,11 +842,12 @@ __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode_kernel(const GDNP
 // above with exactly 4 half-tile slots: item it fills slots 2(it%2) and
 // 2(it%2)+1, so each group owns one pair; with an even number of record
 // buffers each group also owns its buffers.  A group therefore never waits on
-// a barrier phase beyond the next one of its own slots and buffers.  Within a group warp w (0-3) reads
-// rows 32w..32w+31 of the tile straight from its slot (no register copy: the
-// tile is used once on non-flush steps, and the fold epilogue reads it again
-// from the slot); thread c of the group forms u and the output of column c;
-// the fold's accumulator is this group's 128 of 256 tensor-memory columns.
+// a barrier phase beyond the next one of its own slots and buffers.  Within a
+// group warp w (0-3) reads rows 32w..32w+31 of the tile straight from its slot
+// (no register copy: the tile is used once on non-flush steps, and the fold
+// epilogue reads it again from the slot); thread c of the group forms u and
+// the output of column c; the fold's accumulator is this group's 128 of 256
+// tensor-memory columns.
 template <typename TI>
 __global__ void __launch_bounds__(kThreads + 64, 1) gdn_decode2_kernel(const GDNParams p,
                                                                     const GdnLayout lay) {

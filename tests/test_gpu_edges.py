@@ -63,6 +63,23 @@ def test_gdn_windows_and_fp32_inputs(L, dtype):
     assert rel_err(_gpu.f64(got["state"].h0), orc.h0) < TOL
 
 
+@pytest.mark.parametrize("L,dtype", [(1, torch.bfloat16), (2, torch.bfloat16), (16, torch.float32)])
+def test_kda_windows_and_fp32_inputs(L, dtype):
+    """Kimi Delta Attention with a one-record window (a fold every step), a
+    two-record window, and fp32 inputs (two record buffers instead of four)."""
+    w = wl.make("kda_serving", B=2, H=4, L=L, in_dtype=dtype)
+    g = wl.Generator(w)
+    S0 = g.initial_state()
+    st = g.steps(20)
+    got = _gpu.gdn_replay_run(w, S0, st)
+    orc = oracle.KDAReplay(S0, L=L)
+    o, lt, _ = orc.decode(st["q"], st["k"], st["v"], st["alpha"], st["beta"])
+    assert got["state"].status() == 0
+    assert np.array_equal(got["len"], lt)
+    assert per_step_rel_err(got["y"], o) < TOL
+    assert rel_err(_gpu.f64(got["state"].h0), orc.h0) < TOL
+
+
 def test_empty_batch_is_a_no_op():
     for kind in ("m2", "gdn"):
         w = wl.make("m2_serving" if kind == "m2" else "gdn_serving", B=0, H=16 if kind == "m2" else 4,
